@@ -1,0 +1,407 @@
+"""Benchmark of the ZONOS2 sparse MoE feed-forward path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+A step is one pass of the whole MoE layer over one batch of synthetic tokens:
+zmoe_route -> zmoe_permute -> zmoe_grouped_swiglu -> zmoe_combine, all through libzmoe's
+C-ABI.  The default workload is the decode step (T = 64 tokens, d_model 2048, d_ff 3072,
+16 experts, top-1, bf16 weights with fp32 accumulation): memory-bound, every touched
+expert's weights are streamed from HBM once.  Four copies of the layer's weights (2.4 GB,
+far above the 126 MB L2) are used in rotation so that no step finds its weights in L2.
+
+Multi-GPU (torchrun, one rank per GPU): tokens are independent, so every rank runs its own
+batch against replicated weights with no data-path collective (weak scaling); the time is
+the max over ranks, taken from CUDA events.
+
+``--impl reference`` times the fp64 CPU oracle (the baseline arm) on the same workload.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from datetime import timedelta
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/sec on 1 B200 and % of roofline (HBM GB/s or tensor TFLOP/s)"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle timing leg")
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=FALLBACK_HBM_GBS, bf16_tflops=FALLBACK_BF16_TFLOPS,
+                    bf16_tflops_sustained=1400.0, source="fallback")
+
+
+WORKLOADS = {
+    2: "decode step: one MoE layer, T=64 tokens (64 streams x 1 position), d_model=2048, d_ff=3072, E=16, top-1, "
+       "bf16 weights/activations, fp32 accumulate",
+    3: "prefill MoE layer: T=16384 (8 x 2048), d_model=2048, d_ff=3072, E=16, top-1, b~N(0,0.5), bf16",
+    4: "final MoE layer: T=16384, d_model=2048, d_ff=3072, E=16, top-2, Zipf(1.2) logit skew, bf16",
+}
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"zmoe_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            with open(self.path) as fh:
+                for line in fh:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) < 9:
+                        continue
+                    try:
+                        sm.append(float(parts[1]))
+                        smax.append(float(parts[2]))
+                    except ValueError:
+                        continue
+                    for n, v in zip(names, parts[5:9]):
+                        if v.lower() == "active":
+                            reasons.add(n)
+            os.unlink(self.path)
+        except OSError:
+            pass
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [v for v in sm if v > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# the oracle leg (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_leg(L, budget_s: float, max_steps: int | None = None):
+    """Times oracle.moe_layer on the workload's layer; returns (tokens/s, steps, seconds, sample text)."""
+    import oracle
+    if L.T > 1024:
+        # bounded sample: the first 512 tokens of the batch (same weights, same routing rule)
+        T_s = 512
+        x = L.x[:T_s]
+    else:
+        T_s = L.T
+        x = L.x
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.moe_layer(x, L.w_router, L.w_gate, L.w_up, L.w_down, L.k, L.sel_bias, L.logit_bias)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or (max_steps is not None and steps >= max_steps):
+            break
+    sample = (f"oracle.moe_layer (numpy float64) on {T_s} of the workload's {L.T} tokens with the full "
+              f"16-expert weights, {steps} step(s), {el:.1f} s")
+    return T_s * steps / el, steps, el, sample
+
+
+def run_reference(args):
+    """The oracle as it stands, on the host cores: W untimed + K timed steps, each step a bounded
+    sample of the workload's tokens (rotating through the batch) sized so the run ends in ~2.5 min."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from moe_inputs import make_config
+    L = make_config(args.config)
+
+    def one(lo, n):
+        idx = (np.arange(n) + lo) % L.T
+        oracle.moe_layer(L.x[idx], L.w_router, L.w_gate, L.w_up, L.w_down, L.k, L.sel_bias, L.logit_bias)
+
+    t0 = time.perf_counter()
+    one(0, min(L.T, 64))                                  # calibration on up to 64 tokens
+    t_cal = (time.perf_counter() - t0) / min(L.T, 64)
+    per_step = 150.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(L.T, per_step / max(t_cal, 1e-9))))
+    for i in range(args.warmup):
+        one(i * n, n)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one((args.warmup + i) * n, n)
+    el = time.perf_counter() - t0
+    v = n * args.steps / el
+    cores = blas_threads()
+    sample = (f"oracle.moe_layer (numpy float64), {n} of the workload's {L.T} tokens per step "
+              f"(rotating through the batch), full 16-expert weights, {args.steps} timed steps, {el:.1f} s")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.config], "T": L.T, "d_model": L.d, "d_ff": L.f, "E": L.E,
+                       "k": L.k, "tokens_per_step": n},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+
+def traffic_from_profiles(kernel_key: str):
+    """Per-launch DRAM bytes recorded from an ncu capture, if the kernel source is unchanged since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        entries = {}
+        with open(path) as fh:
+            for line in fh:
+                if line.startswith("#") or "=" not in line:
+                    continue
+                k, v = line.strip().split("=", 1)
+                entries[k.strip()] = v.strip()
+        src = entries.get(f"{kernel_key}.source")
+        want_hash = entries.get(f"{kernel_key}.sha256")
+        if not src or not want_hash:
+            return None
+        with open(os.path.join(ROOT, src), "rb") as fh:
+            if hashlib.sha256(fh.read()).hexdigest() != want_hash:
+                return None
+        return float(entries[f"{kernel_key}.bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    from moe_inputs import make_config
+    from sparse_moe_decoder_b200 import MoELayerRunner, MoEWeights, zmoe_get_device_errors
+
+    L = make_config(args.config)
+    if rank > 0:
+        # each rank its own tokens, replicated weights
+        from moe_inputs import round_to_bf16
+        rng = np.random.default_rng(1000 + rank)
+        L.x = round_to_bf16(rng.standard_normal(L.x.shape, dtype=np.float32))
+    dt = torch.bfloat16
+    W0 = MoEWeights.from_host(L)
+    n_copies = 4 if args.config == 2 else 1
+    Ws = [W0] + [MoEWeights(W0.w_router.clone(), W0.w_gate.clone(), W0.w_up.clone(), W0.w_down.clone(),
+                            W0.sel_bias, W0.logit_bias, None, W0.k) for _ in range(n_copies - 1)]
+    R = MoELayerRunner(L.T, L.E, L.d, L.f, L.k, dt)
+    x = torch.from_numpy(L.x).to("cuda", dt)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        return R.run(x, Ws[i % n_copies])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    counts = R.perm_outs["counts"].cpu().numpy()
+    experts_touched = int((counts > 0).sum())
+
+    # timed region: K steps, per-step events around the grouped-SwiGLU call (dominant kernels)
+    import sparse_moe_decoder_b200.zmoe as Z
+    ev_ffn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        for i in range(args.steps):
+            W = Ws[i % n_copies]
+            Z.zmoe_route(x, W.w_router, W.k, W.logit_bias, W.sel_bias, outs=(R.idx, R.gates, R.margin))
+            Z.zmoe_permute(R.idx, x, W.E, outs=R.perm_outs, workspace=R.perm_ws)
+            ev_ffn[i][0].record(stream)
+            Z.zmoe_grouped_swiglu(R.perm_outs["x_perm"], R.perm_outs["offsets"], W.w_gate, W.w_up, W.w_down,
+                                  h=R.h, y_perm=R.y_perm, workspace=R.ffn_ws)
+            ev_ffn[i][1].record(stream)
+            Z.zmoe_combine(R.y_perm, R.perm_outs["inv_perm"], R.gates, None, out=R.y)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    ffn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_ffn)
+    if world > 1:
+        t = torch.tensor([elapsed_ms, ffn_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, ffn_ms = float(t[0]), float(t[1])
+    ms_per_step = elapsed_ms / args.steps
+    tokens_total = L.T * world * args.steps
+    value = tokens_total / (elapsed_ms / 1e3)
+
+    # launches of libzmoe kernels per step
+    n_assign = L.T * L.k
+    launches_per_step = 1 + (1 if n_assign <= 1024 else 4) + 2 + 1
+
+    # e2e: the same steps through the public API from pinned host memory, result read back
+    x_host = torch.from_numpy(L.x).to(dt).pin_memory()
+    y_host = torch.empty((L.T, L.d), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x)
+    for i in range(min(3, args.warmup)):
+        x_dev.copy_(x_host, non_blocking=True)
+        R.run(x_dev, Ws[i % n_copies])
+        y_host.copy_(R.y, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        R.run(x_dev, Ws[i % n_copies])
+        y_host.copy_(R.y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_value = tokens_total / (e2e_ms / 1e3)
+    h2d = x_host.numel() * x_host.element_size()
+    d2h = y_host.numel() * y_host.element_size()
+
+    dev_errors = zmoe_get_device_errors()
+
+    # roofline of the dominant kernels (the grouped-SwiGLU launches: gate/up then down)
+    peaks = load_peaks()
+    bpe = 2
+    counts_all = R.perm_outs["counts"].cpu().numpy()
+    touched = int((counts_all > 0).sum())
+    M = int(counts_all.sum())
+    weight_bytes = touched * 3 * L.f * L.d * bpe
+    act_bytes = M * L.d * bpe + 2 * M * L.f * bpe + M * L.d * 4   # x_perm in, h out + in, y_perm out
+    alg_bytes = weight_bytes + act_bytes
+    flops = 2.0 * M * 3 * L.d * L.f
+    if args.config == 2:
+        achieved = alg_bytes / (ffn_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_from_profiles("grouped_swiglu_cfg2"),
+                "kernel": "zmoe_grouped_swiglu (stream_ffn gate/up + down launches)",
+                "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peaks["source"]}
+    else:
+        achieved = flops / (ffn_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "traffic": traffic_from_profiles(f"grouped_swiglu_cfg{args.config}"),
+                "kernel": "zmoe_grouped_swiglu", "algorithmic_flops_per_launch": flops,
+                "peak_source": peaks["source"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, steps, el, sample = oracle_leg(L, args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.config], "T": L.T, "d_model": L.d, "d_ff": L.f, "E": L.E,
+                       "k": L.k, "tokens_per_rank": L.T, "parallelism": f"dp{world} (replicated weights, no "
+                       "data-path collective)",
+                       "l2": ("weights rotated over 4 device copies (2.4 GB > 126 MB L2)" if n_copies > 1
+                              else "inputs larger than L2 (weights 604 MB, activations >= 67 MB)"),
+                       "experts_touched": experts_touched},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+            "ffn_ms_per_step": ffn_ms,
+            "device_errors": dev_errors,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

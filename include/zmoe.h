@@ -1,0 +1,198 @@
+/*
+ * libzmoe: the sparse mixture-of-experts feed-forward path of the ZONOS2
+ * autoregressive decoder, as hand-written CUDA kernels for NVIDIA B200 (sm_100a).
+ *
+ * Sources (the ZONOS2 pages):
+ *   [DIGEST]  "ZONOS2 Technical Report" digest (audio-paper-digest blog),
+ *             section "method overview and architecture": item 1 (delay pattern over
+ *             N = 9 DAC codebooks), item 5 (input = RMSNorm of the summed codebook
+ *             embeddings; 28 layers, MoE layers with 16 experts, top-1 routing,
+ *             top-2 in the last MoE layer), item 6 (per-layer bias b_l that steers
+ *             expert usage toward uniform).
+ *   [ABSTRACT] "ZONOS2 Technical Report" (mlsanity.com), Abstract (8B total, 900M
+ *             active) and "Builds on" (GLU Variants Improve Transformer; Root Mean
+ *             Square Layer Normalization; Auxiliary-Loss-Free Load Balancing).
+ *   [ROUTING] telknet.cc article on ZONOS2, section 2.1 (routing intuition: linear
+ *             router, SiLU, TopK; the printed equation was lost in extraction).
+ *
+ * Conventions for every call
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  No call
+ *     allocates or frees device memory; scratch comes from caller-provided
+ *     `workspace` / `ws_bytes`, sized by the matching *_workspace_size() query.
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default stream) and
+ *     never synchronises.  Results are valid once the stream reaches the call.
+ *   - Row-major layouts throughout.  Activations [T, d]; router W_r [E, d];
+ *     W_gate, W_up [E, f, d] and W_down [E, d, f] (every weight row is contiguous
+ *     along the contraction dimension, i.e. K-major).
+ *   - Arguments are checked on the host before anything is launched; a bad argument
+ *     returns ZMOE_ERR_INVALID_ARG (or ZMOE_ERR_UNSUPPORTED for a valid but unbuilt
+ *     shape) and launches nothing.  A launch failure returns ZMOE_ERR_CUDA;
+ *     zmoe_last_error() then gives the CUDA message (thread-local).
+ *   - Data errors found on the device (an id or expert index out of range) never
+ *     fault: the offending element is skipped and a device error counter is
+ *     incremented; read it with zmoe_get_device_errors().
+ *   - Sizes are int; T * max(d, f) and T * k must fit in int32.
+ */
+#ifndef ZMOE_H
+#define ZMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ZMOE_API __attribute__((visibility("default")))
+#else
+#define ZMOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* zmoe_stream_t;
+
+typedef enum {
+  ZMOE_OK = 0,
+  ZMOE_ERR_INVALID_ARG = 1,        /* checked on the host, nothing launched          */
+  ZMOE_ERR_UNSUPPORTED = 2,        /* valid arguments, shape or dtype not built      */
+  ZMOE_ERR_CUDA = 3,               /* CUDA runtime error; see zmoe_last_error()      */
+  ZMOE_ERR_WORKSPACE_TOO_SMALL = 4,
+  ZMOE_ERR_DEVICE_CHECK = 5,       /* device-side data check failed (counter > 0)    */
+  ZMOE_ERR_TIMEOUT = 6             /* a bounded device-side wait gave up             */
+} zmoe_status;
+
+typedef enum {
+  ZMOE_F32 = 0,
+  ZMOE_BF16 = 1
+} zmoe_dtype;
+
+/* Library version, as 10000 * major + 100 * minor + patch. */
+ZMOE_API int zmoe_version(void);
+
+/* Static text for a status code. */
+ZMOE_API const char* zmoe_status_string(int status);
+
+/* Message of the last failing call on this host thread ("" when none). */
+ZMOE_API const char* zmoe_last_error(void);
+
+/*
+ * Delay pattern, [DIGEST] item 1:  Y[b, t, j] = X[b, t - j, j]  when 0 <= t - j < T,
+ * and `pad` elsewhere.
+ *   X: int32 [B, T, N]  ->  Y: int32 [B, T + N - 1, N].
+ * B >= 0, T >= 0, 1 <= N <= 64.  Every id is copied bit-exactly.
+ */
+ZMOE_API zmoe_status zmoe_delay_shear(const int32_t* X, int32_t* Y, int B, int T, int N, int32_t pad,
+                             zmoe_stream_t stream);
+
+/*
+ * Inverse delay pattern, [DIGEST] item 1:  X_hat[b, t, j] = Y[b, t + j, j].
+ *   Y: int32 [B, Ty, N]  ->  X_hat: int32 [B, Ty - N + 1, N].   Requires Ty >= N - 1.
+ */
+ZMOE_API zmoe_status zmoe_delay_unshear(const int32_t* Y, int32_t* X, int B, int Ty, int N, zmoe_stream_t stream);
+
+/*
+ * Summed codebook embeddings followed by RMSNorm, [DIGEST] item 5 (RMSNorm as in
+ * "Root Mean Square Layer Normalization", [ABSTRACT] "Builds on"):
+ *   e[t] = sum_{j < N} tables[j, ids[t, j], :]              (fp32 sum)
+ *   out[t] = e[t] / sqrt(mean_c e[t, c]^2 + eps) * gamma
+ *   ids: int32 [T, N], each in [0, V) (V = 1025: ids 0..1023 plus the pad id 1024);
+ *   tables: [N, V, d] of `table_dtype`; gamma: f32 [d]; out: [T, d] of `out_dtype`.
+ *   d % 8 == 0.  An id outside [0, V) contributes nothing and counts a device error.
+ *   tables, out: 16-byte aligned.
+ */
+ZMOE_API zmoe_status zmoe_embed_sum_rmsnorm(const int32_t* ids, const void* tables, zmoe_dtype table_dtype,
+                                   const float* gamma, float eps, int T, int N, int V, int d,
+                                   void* out, zmoe_dtype out_dtype, zmoe_stream_t stream);
+
+/*
+ * RMSNorm of each row (the per-layer pre-norm of the decode stack):
+ *   out[t] = h[t] / sqrt(mean_c h[t, c]^2 + eps) * gamma
+ *   h: [T, d] of `in_dtype`; gamma: f32 [d]; out: [T, d] of `out_dtype`.  d % 8 == 0,
+ *   16-byte aligned h and out.
+ */
+ZMOE_API zmoe_status zmoe_rmsnorm(const void* h, zmoe_dtype in_dtype, const float* gamma, float eps, int T, int d,
+                         void* out, zmoe_dtype out_dtype, zmoe_stream_t stream);
+
+/*
+ * Router with a selection-only bias, [DIGEST] items 5-6, [ROUTING] section 2.1,
+ * [ABSTRACT] "Builds on" (Auxiliary-Loss-Free Load Balancing):
+ *   l = W_r x (fp32 accumulation);  q = l + logit_bias;  s = q + sel_bias;
+ *   expert_idx[t, :] = the k largest s, by descending s, ties -> lower expert index;
+ *   p = softmax(q) over all E;  k == 1: gates = p[sel];
+ *   k == 2: gates_i = p[sel_i] / (p[sel_0] + p[sel_1]).
+ *   margin[t] (optional) = s_(1) - s_(2) for k == 1, min(s_(1) - s_(2), s_(2) - s_(3))
+ *   for k == 2 (+inf when E == k).
+ *   x: [T, d], w_router: [E, d], both of `dtype`; logit_bias, sel_bias: f32 [E] or NULL
+ *   (= zeros); expert_idx: int32 [T, k]; gates: f32 [T, k]; margin: f32 [T] or NULL.
+ *   1 <= E <= 64, k in {1, 2}, k <= E, d % 8 == 0; x and w_router 16-byte aligned.
+ */
+ZMOE_API zmoe_status zmoe_route(const void* x, const void* w_router, zmoe_dtype dtype, const float* logit_bias,
+                       const float* sel_bias, int T, int d, int E, int k, int32_t* expert_idx, float* gates,
+                       float* margin, zmoe_stream_t stream);
+
+/* Bytes of workspace zmoe_permute needs for these sizes. */
+ZMOE_API size_t zmoe_permute_workspace_size(int T, int E, int k);
+
+/*
+ * Dispatch permutation (implied by sparse experts, [DIGEST] item 5):
+ *   counts[e]  = #{(t, i) : expert_idx[t, i] == e}            int32 [E]
+ *   offsets    = exclusive prefix sum of counts                int32 [E + 1]
+ *   rows ordered by expert, then by token (stable, deterministic):
+ *   perm[row] = t                                              int32 [T * k]
+ *   inv_perm[t, i] = row holding assignment (t, i)             int32 [T, k]
+ *   x_perm[row] = x[perm[row]]                                 [T * k, d] of `dtype`
+ * Bit-exact and deterministic.  An expert index outside [0, E) counts a device error;
+ * that assignment is dropped (its inv_perm entry is -1) and the rows after it in the
+ * same expert are unaffected.  d % 8 == 0; x, x_perm 16-byte aligned.
+ */
+ZMOE_API zmoe_status zmoe_permute(const int32_t* expert_idx, const void* x, zmoe_dtype dtype, int T, int d, int E, int k,
+                         int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* x_perm,
+                         void* workspace, size_t ws_bytes, zmoe_stream_t stream);
+
+/* Bytes of workspace zmoe_grouped_swiglu needs for these sizes. */
+ZMOE_API size_t zmoe_grouped_swiglu_workspace_size(int M_total, int E, int d, int f, zmoe_dtype dtype);
+
+/*
+ * Per-expert SwiGLU over the permuted rows ("GLU Variants Improve Transformer",
+ * [ABSTRACT] "Builds on"; SiLU per [ROUTING] section 2.1):
+ *   for each expert e and each row r in [offsets[e], offsets[e + 1]):
+ *     h[r]      = silu(W_gate[e] x_perm[r]) * (W_up[e] x_perm[r])     [f], stored in `dtype`
+ *     y_perm[r] = W_down[e] h[r]                                      [d], stored as f32
+ *   silu(z) = z / (1 + exp(-z)); contractions accumulate in fp32.  bf16 rounds h to
+ *   bf16 before the second contraction (it is the operand of that contraction); y_perm
+ *   leaves the fp32 accumulator unrounded.
+ *   x_perm: [M_total, d]; offsets: int32 [E + 1] on the DEVICE (read by the kernels,
+ *   never copied to the host); M_total = T * k is the host-side row bound and must be
+ *   >= offsets[E]; w_gate, w_up: [E, f, d]; w_down: [E, d, f]; h: [M_total, f] (caller
+ *   scratch that also exposes the hidden activations); y_perm: f32 [M_total, d].
+ *   bf16: d % 64 == 0, f % 64 == 0; f32: d % 4 == 0, f % 4 == 0.  16-byte aligned.
+ */
+ZMOE_API zmoe_status zmoe_grouped_swiglu(const void* x_perm, const int32_t* offsets, int M_total, const void* w_gate,
+                                const void* w_up, const void* w_down, zmoe_dtype dtype, int E, int d, int f,
+                                void* h, float* y_perm, void* workspace, size_t ws_bytes, zmoe_stream_t stream);
+
+/*
+ * Gate-weighted combine ([ROUTING] section 2.1: the output is the gate-weighted sum of
+ * the chosen experts), as a per-token gather in fixed slot order (deterministic):
+ *   y[t] = residual[t] + sum_{i < k} gates[t, i] * y_perm[inv_perm[t, i]]
+ *   y_perm: f32 [T * k, d]; inv_perm: int32 [T, k]; gates: f32 [T, k];
+ *   residual: f32 [T, d] or NULL (= zeros); y: f32 [T, d] (may alias residual).
+ *   An inv_perm entry outside [0, T * k) contributes nothing and counts a device error.
+ *   d % 4 == 0, 16-byte aligned y_perm, residual, y.
+ */
+ZMOE_API zmoe_status zmoe_combine(const float* y_perm, const int32_t* inv_perm, const float* gates, const float* residual,
+                         int T, int d, int k, float* y, zmoe_stream_t stream);
+
+/*
+ * Reads and clears the device error counter of the current device.  Synchronises
+ * `stream` first.  *count = number of data errors seen by kernels since the last read.
+ * Returns ZMOE_ERR_DEVICE_CHECK when *count > 0, ZMOE_OK otherwise.
+ */
+ZMOE_API zmoe_status zmoe_get_device_errors(zmoe_stream_t stream, uint32_t* count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZMOE_H */

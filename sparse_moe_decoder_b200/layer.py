@@ -1,0 +1,134 @@
+"""The MoE layer and the batch-1 decode stack, chained through libzmoe's C entry points.
+
+Buffers are allocated once (torch is used for device memory only); every step runs in
+libzmoe's kernels:
+
+    zmoe_route -> zmoe_permute -> zmoe_grouped_swiglu -> zmoe_combine
+
+ZONOS2 Technical Report digest, "method overview and architecture", item 5: 24 MoE layers
+of 16 experts with top-1 routing and top-2 in the last one, fed by the RMSNorm of the
+summed codebook embeddings.  Per-layer wiring of the stack (the pages leave it open):
+pre-norm residual, h <- h + MoE_l(RMSNorm_l(h)), with h kept in fp32 and the layer input
+rounded to the weights' dtype.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import List, Optional
+
+import torch
+
+from . import zmoe as Z
+
+
+@dataclass
+class MoEWeights:
+    """One layer's device weights.  Shapes: W_r [E, d], W_gate/W_up [E, f, d], W_down [E, d, f]."""
+
+    w_router: torch.Tensor
+    w_gate: torch.Tensor
+    w_up: torch.Tensor
+    w_down: torch.Tensor
+    sel_bias: Optional[torch.Tensor] = None     # f32 [E]
+    logit_bias: Optional[torch.Tensor] = None   # f32 [E]
+    gamma: Optional[torch.Tensor] = None        # f32 [d], pre-norm gain (stack only)
+    k: int = 1
+
+    @property
+    def E(self) -> int:
+        return self.w_router.shape[0]
+
+    @property
+    def d(self) -> int:
+        return self.w_router.shape[1]
+
+    @property
+    def f(self) -> int:
+        return self.w_gate.shape[1]
+
+    @property
+    def dtype(self) -> torch.dtype:
+        return self.w_router.dtype
+
+    @staticmethod
+    def from_host(L, device="cuda", dtype: Optional[torch.dtype] = None) -> "MoEWeights":
+        """From a ``moe_inputs.MoELayerInputs`` (float32 arrays, bf16-exact for bf16 layers)."""
+        dt = dtype or (torch.bfloat16 if L.dtype == "bf16" else torch.float32)
+
+        def dev(a, t=dt):
+            return None if a is None else torch.from_numpy(a).to(device=device, dtype=t).contiguous()
+
+        return MoEWeights(dev(L.w_router), dev(L.w_gate), dev(L.w_up), dev(L.w_down),
+                          dev(L.sel_bias, torch.float32), dev(L.logit_bias, torch.float32),
+                          dev(L.gamma, torch.float32), L.k)
+
+
+class MoELayerRunner:
+    """Preallocated buffers for T tokens through one MoE layer shape."""
+
+    def __init__(self, T: int, E: int, d: int, f: int, k: int, dtype: torch.dtype, device="cuda"):
+        self.T, self.E, self.d, self.f, self.k, self.dtype = T, E, d, f, k, dtype
+        dev = torch.device(device)
+        M = T * k
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        self.gates = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.margin = torch.empty((T,), dtype=torch.float32, device=dev)
+        self.perm_outs = dict(counts=torch.empty(E, dtype=torch.int32, device=dev),
+                              offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                              perm=torch.empty(M, dtype=torch.int32, device=dev),
+                              inv_perm=torch.empty((T, k), dtype=torch.int32, device=dev),
+                              x_perm=torch.empty((M, d), dtype=dtype, device=dev))
+        self.perm_ws = torch.empty(max(Z.zmoe_permute_workspace_size(T, E, k), 16), dtype=torch.uint8, device=dev)
+        self.h = torch.empty((M, f), dtype=dtype, device=dev)
+        self.y_perm = torch.empty((M, d), dtype=torch.float32, device=dev)
+        self.ffn_ws = torch.empty(max(Z.zmoe_grouped_swiglu_workspace_size(M, E, d, f, dtype), 16),
+                                  dtype=torch.uint8, device=dev)
+        self.y = torch.empty((T, d), dtype=torch.float32, device=dev)
+
+    def run(self, x: torch.Tensor, W: MoEWeights, residual: Optional[torch.Tensor] = None,
+            out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """y = residual + sum_i gate_i * FFN_{e_i}(x), f32 [T, d]."""
+        Z.zmoe_route(x, W.w_router, W.k, W.logit_bias, W.sel_bias, outs=(self.idx, self.gates, self.margin),
+                     stream=stream)
+        Z.zmoe_permute(self.idx, x, W.E, outs=self.perm_outs, workspace=self.perm_ws, stream=stream)
+        Z.zmoe_grouped_swiglu(self.perm_outs["x_perm"], self.perm_outs["offsets"], W.w_gate, W.w_up, W.w_down,
+                              h=self.h, y_perm=self.y_perm, workspace=self.ffn_ws, stream=stream)
+        return Z.zmoe_combine(self.y_perm, self.perm_outs["inv_perm"], self.gates, residual,
+                              out=self.y if out is None else out, stream=stream)
+
+
+class DecodeStack:
+    """Embedding sum + RMSNorm, then L pre-norm residual MoE layers, for T tokens per step."""
+
+    def __init__(self, tables: torch.Tensor, gamma0: torch.Tensor, layers: List[MoEWeights], eps: float = 1e-6,
+                 T: int = 1):
+        self.tables, self.gamma0, self.layers, self.eps, self.T = tables, gamma0, layers, eps, T
+        L0 = layers[0]
+        dev = tables.device
+        self.dtype = L0.dtype
+        self.runners = {k: MoELayerRunner(T, L0.E, L0.d, L0.f, k, L0.dtype, dev) for k in {L.k for L in layers}}
+        self.ids = torch.empty((T, tables.shape[0]), dtype=torch.int32, device=dev)
+        self.h = torch.empty((T, L0.d), dtype=torch.float32, device=dev)
+        self.x = torch.empty((T, L0.d), dtype=L0.dtype, device=dev)
+        self.record_inputs = False
+        self.layer_inputs: List[torch.Tensor] = []
+        self.layer_h: List[torch.Tensor] = []
+        self.layer_idx: List[torch.Tensor] = []
+
+    def step(self, ids: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """One decode step; returns the final fp32 residual stream h [T, d]."""
+        if ids is not None:
+            self.ids.copy_(ids)
+        Z.zmoe_embed_sum_rmsnorm(self.ids, self.tables, self.gamma0, self.eps, out=self.h, stream=stream)
+        if self.record_inputs:
+            self.layer_inputs, self.layer_h, self.layer_idx = [], [], []
+        for L in self.layers:
+            Z.zmoe_rmsnorm(self.h, L.gamma, self.eps, out=self.x, stream=stream)
+            if self.record_inputs:
+                self.layer_h.append(self.h.clone())
+                self.layer_inputs.append(self.x.clone())
+            R = self.runners[L.k]
+            R.run(self.x, L, residual=self.h, out=self.h, stream=stream)
+            if self.record_inputs:
+                self.layer_idx.append(R.idx.clone())
+        return self.h

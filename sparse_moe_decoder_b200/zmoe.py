@@ -1,0 +1,266 @@
+"""ctypes binding of libzmoe (argument marshalling only).
+
+Every ``zmoe_*`` function here takes torch CUDA tensors, checks shapes and dtypes,
+allocates outputs with torch (device memory is the only thing torch provides) and
+calls the C entry point of the same name on the current torch stream.  Every step
+of the computation runs in libzmoe's CUDA kernels; there is no CPU or PyTorch
+fallback: if the shared library is missing, loading fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzmoe.so")
+
+ZMOE_F32 = 0
+ZMOE_BF16 = 1
+
+STATUS_NAMES = {0: "ZMOE_OK", 1: "ZMOE_ERR_INVALID_ARG", 2: "ZMOE_ERR_UNSUPPORTED", 3: "ZMOE_ERR_CUDA",
+                4: "ZMOE_ERR_WORKSPACE_TOO_SMALL", 5: "ZMOE_ERR_DEVICE_CHECK", 6: "ZMOE_ERR_TIMEOUT"}
+
+# name -> (restype, argtypes)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_S = ctypes.c_size_t
+SIGNATURES = {
+    "zmoe_version": (_I, []),
+    "zmoe_status_string": (ctypes.c_char_p, [_I]),
+    "zmoe_last_error": (ctypes.c_char_p, []),
+    "zmoe_delay_shear": (_I, [_P, _P, _I, _I, _I, ctypes.c_int32, _P]),
+    "zmoe_delay_unshear": (_I, [_P, _P, _I, _I, _I, _P]),
+    "zmoe_embed_sum_rmsnorm": (_I, [_P, _P, _I, _P, _F, _I, _I, _I, _I, _P, _I, _P]),
+    "zmoe_rmsnorm": (_I, [_P, _I, _P, _F, _I, _I, _P, _I, _P]),
+    "zmoe_route": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "zmoe_permute_workspace_size": (_S, [_I, _I, _I]),
+    "zmoe_permute": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "zmoe_grouped_swiglu_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "zmoe_grouped_swiglu": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _S, _P]),
+    "zmoe_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "zmoe_get_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+}
+
+
+class ZmoeError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}" + (f" ({detail})" if detail else ""))
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libzmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libzmoe.so not found at {LIB_PATH}; build it with "
+                              "`python -m sparse_moe_decoder_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        detail = lib().zmoe_last_error().decode(errors="replace")
+        raise ZmoeError(status, where, detail)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return ZMOE_F32
+    if dt == torch.bfloat16:
+        return ZMOE_BF16
+    raise TypeError(f"libzmoe computes in float32 or bfloat16, got {dt}")
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+
+
+# ---------------------------------------------------------------------------------------------
+# the C-ABI calls
+# ---------------------------------------------------------------------------------------------
+
+def zmoe_version() -> int:
+    return lib().zmoe_version()
+
+
+def zmoe_delay_shear(X: torch.Tensor, pad: int = 1024, out: Optional[torch.Tensor] = None, stream=None):
+    """Y[b, t, j] = X[b, t - j, j] (pad outside), X int32 [B, T, N] or [T, N]."""
+    _need(X, "X", torch.int32)
+    squeeze = X.dim() == 2
+    X3 = X.unsqueeze(0) if squeeze else X
+    B, T, N = X3.shape
+    Y = out if out is not None else torch.empty((B, T + N - 1, N), dtype=torch.int32, device=X.device)
+    _check(lib().zmoe_delay_shear(_ptr(X3), _ptr(Y), B, T, N, int(pad), _stream(stream)), "zmoe_delay_shear")
+    return Y[0] if squeeze and out is None else Y
+
+
+def zmoe_delay_unshear(Y: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+    """X_hat[b, t, j] = Y[b, t + j, j], Y int32 [B, Ty, N] or [Ty, N]."""
+    _need(Y, "Y", torch.int32)
+    squeeze = Y.dim() == 2
+    Y3 = Y.unsqueeze(0) if squeeze else Y
+    B, Ty, N = Y3.shape
+    X = out if out is not None else torch.empty((B, max(Ty - N + 1, 0), N), dtype=torch.int32, device=Y.device)
+    _check(lib().zmoe_delay_unshear(_ptr(Y3), _ptr(X), B, Ty, N, _stream(stream)), "zmoe_delay_unshear")
+    return X[0] if squeeze and out is None else X
+
+
+def zmoe_embed_sum_rmsnorm(ids: torch.Tensor, tables: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
+                           out_dtype: Optional[torch.dtype] = None, out: Optional[torch.Tensor] = None, stream=None):
+    """RMSNorm(sum_j tables[j, ids[:, j]]) * gamma.  ids int32 [T, N], tables [N, V, d]."""
+    _need(ids, "ids", torch.int32, 2)
+    _need(tables, "tables", None, 3)
+    _need(gamma, "gamma", torch.float32, 1)
+    T, N = ids.shape
+    Nt, V, d = tables.shape
+    if Nt != N or gamma.shape[0] != d:
+        raise ValueError("ids / tables / gamma shapes disagree")
+    od = out_dtype or tables.dtype
+    o = out if out is not None else torch.empty((T, d), dtype=od, device=ids.device)
+    _check(lib().zmoe_embed_sum_rmsnorm(_ptr(ids), _ptr(tables), _dtype_code(tables.dtype), _ptr(gamma), float(eps),
+                                        T, N, V, d, _ptr(o), _dtype_code(o.dtype), _stream(stream)),
+           "zmoe_embed_sum_rmsnorm")
+    return o
+
+
+def zmoe_rmsnorm(h: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6, out_dtype: Optional[torch.dtype] = None,
+                 out: Optional[torch.Tensor] = None, stream=None):
+    _need(h, "h", None, 2)
+    _need(gamma, "gamma", torch.float32, 1)
+    T, d = h.shape
+    o = out if out is not None else torch.empty((T, d), dtype=out_dtype or h.dtype, device=h.device)
+    _check(lib().zmoe_rmsnorm(_ptr(h), _dtype_code(h.dtype), _ptr(gamma), float(eps), T, d, _ptr(o),
+                              _dtype_code(o.dtype), _stream(stream)), "zmoe_rmsnorm")
+    return o
+
+
+def zmoe_route(x: torch.Tensor, w_router: torch.Tensor, k: int, logit_bias: Optional[torch.Tensor] = None,
+               sel_bias: Optional[torch.Tensor] = None, margin: bool = True, outs=None, stream=None):
+    """Returns (expert_idx int32 [T, k], gates f32 [T, k], margin f32 [T] or None)."""
+    _need(x, "x", None, 2)
+    _need(w_router, "w_router", x.dtype, 2)
+    for t, n in ((logit_bias, "logit_bias"), (sel_bias, "sel_bias")):
+        if t is not None:
+            _need(t, n, torch.float32, 1)
+    T, d = x.shape
+    E = w_router.shape[0]
+    if outs is None:
+        idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+        g = torch.empty((T, k), dtype=torch.float32, device=x.device)
+        mg = torch.empty((T,), dtype=torch.float32, device=x.device) if margin else None
+    else:
+        idx, g, mg = outs
+    _check(lib().zmoe_route(_ptr(x), _ptr(w_router), _dtype_code(x.dtype), _ptr(logit_bias), _ptr(sel_bias), T, d, E,
+                            k, _ptr(idx), _ptr(g), _ptr(mg), _stream(stream)), "zmoe_route")
+    return idx, g, mg
+
+
+def zmoe_permute_workspace_size(T: int, E: int, k: int) -> int:
+    return int(lib().zmoe_permute_workspace_size(T, E, k))
+
+
+def zmoe_permute(expert_idx: torch.Tensor, x: torch.Tensor, E: int, outs: Optional[dict] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """counts, offsets, perm, inv_perm, x_perm of a [T, k] expert assignment."""
+    _need(expert_idx, "expert_idx", torch.int32, 2)
+    _need(x, "x", None, 2)
+    T, k = expert_idx.shape
+    d = x.shape[1]
+    dev = x.device
+    if outs is None:
+        outs = dict(counts=torch.empty(E, dtype=torch.int32, device=dev),
+                    offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                    perm=torch.empty(T * k, dtype=torch.int32, device=dev),
+                    inv_perm=torch.empty((T, k), dtype=torch.int32, device=dev),
+                    x_perm=torch.empty((T * k, d), dtype=x.dtype, device=dev))
+    ws_bytes = zmoe_permute_workspace_size(T, E, k)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    _check(lib().zmoe_permute(_ptr(expert_idx), _ptr(x), _dtype_code(x.dtype), T, d, E, k, _ptr(outs["counts"]),
+                              _ptr(outs["offsets"]), _ptr(outs["perm"]), _ptr(outs["inv_perm"]),
+                              _ptr(outs["x_perm"]), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "zmoe_permute")
+    return outs
+
+
+def zmoe_grouped_swiglu_workspace_size(M_total: int, E: int, d: int, f: int, dtype: torch.dtype) -> int:
+    return int(lib().zmoe_grouped_swiglu_workspace_size(M_total, E, d, f, _dtype_code(dtype)))
+
+
+def zmoe_grouped_swiglu(x_perm: torch.Tensor, offsets: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
+                        w_down: torch.Tensor, h: Optional[torch.Tensor] = None, y_perm: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None):
+    """Returns (h [M, f] in x's dtype, y_perm f32 [M, d])."""
+    _need(x_perm, "x_perm", None, 2)
+    _need(offsets, "offsets", torch.int32, 1)
+    for t, n in ((w_gate, "w_gate"), (w_up, "w_up"), (w_down, "w_down")):
+        _need(t, n, x_perm.dtype, 3)
+    M, d = x_perm.shape
+    E, f, _ = w_gate.shape
+    dev = x_perm.device
+    if h is None:
+        h = torch.empty((M, f), dtype=x_perm.dtype, device=dev)
+    if y_perm is None:
+        y_perm = torch.empty((M, d), dtype=torch.float32, device=dev)
+    ws_bytes = zmoe_grouped_swiglu_workspace_size(M, E, d, f, x_perm.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    _check(lib().zmoe_grouped_swiglu(_ptr(x_perm), _ptr(offsets), M, _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                     _dtype_code(x_perm.dtype), E, d, f, _ptr(h), _ptr(y_perm), _ptr(workspace),
+                                     workspace.numel(), _stream(stream)), "zmoe_grouped_swiglu")
+    return h, y_perm
+
+
+def zmoe_combine(y_perm: torch.Tensor, inv_perm: torch.Tensor, gates: torch.Tensor,
+                 residual: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, stream=None):
+    """y[t] = residual[t] + sum_i gates[t, i] * y_perm[inv_perm[t, i]], all f32."""
+    _need(y_perm, "y_perm", torch.float32, 2)
+    _need(inv_perm, "inv_perm", torch.int32, 2)
+    _need(gates, "gates", torch.float32, 2)
+    T, k = inv_perm.shape
+    d = y_perm.shape[1]
+    if residual is not None:
+        _need(residual, "residual", torch.float32, 2)
+    y = out if out is not None else torch.empty((T, d), dtype=torch.float32, device=y_perm.device)
+    _check(lib().zmoe_combine(_ptr(y_perm), _ptr(inv_perm), _ptr(gates), _ptr(residual), T, d, k, _ptr(y),
+                              _stream(stream)), "zmoe_combine")
+    return y
+
+
+def zmoe_get_device_errors(stream=None) -> int:
+    """Reads and clears the device error counter (synchronises the stream)."""
+    c = ctypes.c_uint32(0)
+    st = lib().zmoe_get_device_errors(_stream(stream), ctypes.byref(c))
+    if st not in (0, 5):
+        _check(st, "zmoe_get_device_errors")
+    return int(c.value)

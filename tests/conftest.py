@@ -16,3 +16,16 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+_BUILT = []
+
+
+@pytest.fixture(autouse=True)
+def _ensure_libzmoe_for_gpu_tests(request):
+    """GPU tests use the in-tree libzmoe.so; build it once (incrementally) if needed."""
+    if request.node.get_closest_marker("gpu") is not None and not _BUILT:
+        from sparse_moe_decoder_b200 import build as B
+        B.build()
+        _BUILT.append(True)
+    yield

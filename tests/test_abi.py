@@ -1,0 +1,89 @@
+"""The C-ABI library on the CPU: it loads, exports every symbol include/zmoe.h declares, and rejects
+bad arguments on the host (no compute call is made: nothing here needs a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_moe_decoder_b200 import build as B
+from sparse_moe_decoder_b200 import zmoe as Z
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "zmoe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return Z.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"ZMOE_API\s+[\w\s\*]+?\b(zmoe_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for n in ("zmoe_delay_shear", "zmoe_delay_unshear", "zmoe_embed_sum_rmsnorm", "zmoe_route", "zmoe_permute",
+              "zmoe_grouped_swiglu", "zmoe_combine"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in declared_functions():
+        assert hasattr(L, n), f"libzmoe.so does not export {n}"
+        assert n in Z.SIGNATURES, f"the binding has no signature for {n}"
+
+
+def test_status_strings_and_version(L):
+    assert L.zmoe_version() >= 100
+    assert L.zmoe_status_string(0) == b"ok"
+    assert L.zmoe_status_string(1) == b"invalid argument"
+    assert L.zmoe_status_string(99) == b"unknown status"
+
+
+NULL = None
+
+
+@pytest.mark.parametrize("call", [
+    lambda L: L.zmoe_delay_shear(NULL, NULL, 1, 4, 0, 1024, NULL),              # N = 0
+    lambda L: L.zmoe_delay_shear(NULL, NULL, 1, 4, 9, 1024, NULL),              # NULL pointers
+    lambda L: L.zmoe_delay_unshear(NULL, NULL, 1, 3, 9, NULL),                  # Ty < N - 1
+    lambda L: L.zmoe_embed_sum_rmsnorm(NULL, NULL, 1, NULL, 1e-6, 2, 9, 1025, 12, NULL, 1, NULL),  # d % 8
+    lambda L: L.zmoe_embed_sum_rmsnorm(NULL, NULL, 7, NULL, 1e-6, 2, 9, 1025, 16, NULL, 1, NULL),  # dtype
+    lambda L: L.zmoe_rmsnorm(NULL, 0, NULL, -1.0, 2, 16, NULL, 0, NULL),       # eps < 0
+    lambda L: L.zmoe_route(NULL, NULL, 1, NULL, NULL, 4, 64, 16, 3, NULL, NULL, NULL, NULL),   # k = 3
+    lambda L: L.zmoe_route(NULL, NULL, 1, NULL, NULL, 4, 64, 65, 1, NULL, NULL, NULL, NULL),   # E = 65
+    lambda L: L.zmoe_route(NULL, NULL, 1, NULL, NULL, 4, 64, 1, 2, NULL, NULL, NULL, NULL),    # k > E
+    lambda L: L.zmoe_route(NULL, NULL, 1, NULL, NULL, 4, 64, 16, 1, NULL, NULL, NULL, NULL),   # NULL
+    lambda L: L.zmoe_permute(NULL, NULL, 1, 4, 64, 16, 1, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL),
+    lambda L: L.zmoe_grouped_swiglu(NULL, NULL, 4, NULL, NULL, NULL, 1, 16, 64, 64, NULL, NULL, NULL, 0, NULL),
+    lambda L: L.zmoe_combine(NULL, NULL, NULL, NULL, 4, 64, 3, NULL, NULL),    # k = 3
+    lambda L: L.zmoe_combine(NULL, NULL, NULL, NULL, 4, 6, 1, NULL, NULL),     # d % 4
+])
+def test_bad_arguments_rejected_on_host(L, call):
+    assert call(L) == 1   # ZMOE_ERR_INVALID_ARG, nothing launched
+    assert len(L.zmoe_last_error()) > 0
+
+
+def test_unaligned_pointers_rejected(L):
+    # 16-byte alignment is checked on the host before any launch (pointer values are never dereferenced)
+    p = ctypes.c_void_p(0x1000 + 4)
+    q = ctypes.c_void_p(0x2000)
+    st = L.zmoe_route(p, q, 1, NULL, NULL, 4, 64, 16, 1, q, q, NULL, NULL)
+    assert st == 1
+    assert b"aligned" in L.zmoe_last_error()
+
+
+def test_empty_problems_are_no_ops(L):
+    # nothing to do -> OK without touching the device
+    assert L.zmoe_route(NULL, NULL, 1, NULL, NULL, 0, 64, 16, 1, NULL, NULL, NULL, NULL) == 0
+    assert L.zmoe_combine(NULL, NULL, NULL, NULL, 0, 64, 1, NULL, NULL) == 0
+    assert L.zmoe_delay_shear(NULL, NULL, 0, 5, 9, 1024, NULL) == 0
+
+
+def test_workspace_queries(L):
+    assert L.zmoe_permute_workspace_size(16384, 16, 2) >= (32768 // 256) * 16 * 4
+    assert L.zmoe_permute_workspace_size(-1, 16, 1) == 0
+    assert L.zmoe_grouped_swiglu_workspace_size(64, 16, 2048, 3072, 1) >= 0

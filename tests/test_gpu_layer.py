@@ -1,0 +1,86 @@
+"""The whole MoE layer (route -> permute -> grouped SwiGLU -> combine) through the C-ABI vs the oracle.
+
+Configurations 1 and 2 are compared on every token (configuration 2, T = 64, is the decode step the
+benchmark times, in the same launch configuration).  Configurations 3 and 4 (T = 16384) compare all
+routing decisions and a sample of output rows the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_inputs import make_config
+from sparse_moe_decoder_b200 import MoELayerRunner, MoEWeights
+from tests.gpu_util import MARGIN_EXEMPT, TOL, assert_close, host, rel_err, require_gpu, tdtype, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def run_layer(L):
+    dt = tdtype(L.dtype)
+    W = MoEWeights.from_host(L)
+    R = MoELayerRunner(L.T, L.E, L.d, L.f, L.k, dt)
+    y = R.run(to_dev(L.x, dt), W)
+    return R, host(y)
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_layer_every_token(cfg):
+    require_gpu()
+    L = make_config(cfg)
+    R, y = run_layer(L)
+    ref = oracle.moe_layer(L.x, L.w_router, L.w_gate, L.w_up, L.w_down, L.k, L.sel_bias, L.logit_bias)
+    idx = host(R.idx)
+    ok = ref["margin"] >= MARGIN_EXEMPT
+    assert np.array_equal(idx[ok], ref["expert_idx"][ok])
+    same = (idx == ref["expert_idx"]).all(1)
+    r = assert_close(y[same], ref["y"][same], L.dtype, f"config {cfg} y")
+    assert np.array_equal(host(R.perm_outs["counts"]), ref["counts"]) or not ok.all()
+    print(f"config {cfg}: y max err {r:.2e} x RMS; {int((~ok).sum())} low-margin tokens exempt")
+
+
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_layer_prefill_sampled(cfg):
+    require_gpu()
+    L = make_config(cfg)
+    R, y = run_layer(L)
+    sel, gates, margin, _ = oracle.route(L.x, L.w_router, L.k, L.sel_bias, L.logit_bias)
+    idx = host(R.idx)
+    ok = margin >= MARGIN_EXEMPT
+    assert np.array_equal(idx[ok], sel[ok]), "routing differs on a token with margin >= 1e-4"
+    counts = np.bincount(sel.ravel(), minlength=L.E)
+    print(f"config {cfg}: expert loads {counts.tolist()}, expert-0 share {counts[0] / counts.sum():.3f}, "
+          f"{int((~ok).sum())} low-margin tokens")
+    rng = np.random.default_rng(cfg)
+    sample = np.unique(np.concatenate([[0, L.T - 1], rng.integers(0, L.T, size=192)]))
+    sample = sample[(idx[sample] == sel[sample]).all(1)]
+    want = np.zeros((len(sample), L.d))
+    for n, t in enumerate(sample):
+        for i in range(L.k):
+            e = sel[t, i]
+            want[n] += gates[t, i] * oracle.swiglu_ffn(L.x[t:t + 1], L.w_gate[e], L.w_up[e], L.w_down[e])[0]
+    r = assert_close(y[sample], want, "bf16", f"config {cfg} sampled y")
+    print(f"config {cfg}: sampled y max err {r:.2e} x RMS over {len(sample)} tokens")
+
+
+def test_layer_token_permutation_invariance():
+    require_gpu()
+    L = make_config(2)
+    R, y = run_layer(L)
+    pi = np.random.default_rng(0).permutation(L.T)
+    L.x = L.x[pi]
+    R2, y2 = run_layer(L)
+    assert rel_err(y2, y[pi]) <= 1e-6
+    assert np.array_equal(host(R2.idx), host(R.idx)[pi])
+
+
+def test_layer_repeatable_bitwise():
+    require_gpu()
+    L = make_config(2)
+    dt = tdtype(L.dtype)
+    W = MoEWeights.from_host(L)
+    R = MoELayerRunner(L.T, L.E, L.d, L.f, L.k, dt)
+    x = to_dev(L.x, dt)
+    first = host(R.run(x, W)).copy()
+    for _ in range(3):
+        assert np.array_equal(host(R.run(x, W)), first)

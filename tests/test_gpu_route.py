@@ -1,0 +1,74 @@
+"""Router on the GPU vs the oracle: ids bit-exact (low-margin tokens exempt and counted), gates
+within the fp32 tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_inputs import make_config, make_moe_layer
+from sparse_moe_decoder_b200 import zmoe_route
+from tests.gpu_util import MARGIN_EXEMPT, TOL, host, rel_err, require_gpu, tdtype, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def check_route(L, label):
+    dt = tdtype(L.dtype)
+    x = to_dev(L.x, dt)
+    w = to_dev(L.w_router, dt)
+    lb = None if L.logit_bias is None else to_dev(L.logit_bias, torch.float32)
+    sb = to_dev(L.sel_bias, torch.float32)
+    idx, g, mg = zmoe_route(x, w, L.k, lb, sb)
+    sel, gates, margin, _ = oracle.route(L.x, L.w_router, L.k, L.sel_bias, L.logit_bias)
+    idx, g, mg = host(idx), host(g), host(mg)
+    ok = margin >= MARGIN_EXEMPT
+    exempt = int((~ok).sum())
+    assert np.array_equal(idx[ok], sel[ok]), f"{label}: expert ids differ on {(idx[ok] != sel[ok]).any(1).sum()} tokens"
+    # gates: fp32 results, compared on tokens with identical selection
+    same = (idx == sel).all(axis=1)
+    assert rel_err(g[same], gates[same]) <= TOL["f32"], f"{label}: gates"
+    fin = np.isfinite(margin) & same
+    assert np.allclose(mg[fin], margin[fin], rtol=1e-3, atol=1e-4), f"{label}: margin"
+    return exempt
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_route_configs(cfg):
+    require_gpu()
+    exempt = check_route(make_config(cfg), f"config {cfg}")
+    print(f"config {cfg}: {exempt} low-margin tokens exempt")
+
+
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_route_prefill_configs_full_size(cfg):
+    """Full T = 16384 routing (the oracle's router is cheap at this size)."""
+    require_gpu()
+    L = make_moe_layer(16384, 2048, 8, 16, 1 if cfg == 3 else 2, "bf16", seed=0,
+                       sel_bias_var=0.5 if cfg == 3 else 0.0, zipf_s=None if cfg == 3 else 1.2)
+    exempt = check_route(L, f"config {cfg}")
+    print(f"config {cfg}: {exempt} low-margin tokens exempt")
+
+
+@pytest.mark.parametrize("E,k", [(1, 1), (2, 2), (5, 2), (16, 1), (17, 2), (32, 1), (33, 2), (64, 2)])
+@pytest.mark.parametrize("T", [1, 7, 130])
+def test_route_edge_shapes(E, k, T):
+    require_gpu()
+    L = make_moe_layer(T, 264, 8, E, k, "bf16", seed=E * 7 + T, sel_bias_var=0.3, zipf_s=1.2)
+    check_route(L, f"E={E} k={k} T={T}")
+
+
+def test_route_exact_ties_lowest_index():
+    """Identical router rows give exactly tied scores: the lower expert index wins, gates split evenly."""
+    require_gpu()
+    E, d = 6, 64
+    rng = np.random.default_rng(1)
+    w = rng.standard_normal((E, d)).astype(np.float32)
+    w[4] = w[1]                      # experts 1 and 4 tie exactly for every token
+    w[3] = w[1]                      # and 3
+    x = rng.standard_normal((40, d)).astype(np.float32)
+    idx, g, _ = zmoe_route(to_dev(x, torch.float32), to_dev(w, torch.float32), 2)
+    sel, gates, _, _ = oracle.route(x, w, 2)
+    idx, g = host(idx), host(g)
+    assert ((sel == 1) | (sel == 3) | (sel == 4)).any(), "the tie must reach the top-2 somewhere"
+    assert np.array_equal(idx, sel)
+    assert np.allclose(g, gates, rtol=1e-5)

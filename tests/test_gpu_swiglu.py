@@ -1,0 +1,115 @@
+"""Grouped SwiGLU on the GPU vs the oracle.
+
+y_perm (fp32 result) is held to the parity bar: max |gpu - oracle| <= 2e-2 x RMS (bf16 weights)
+or 1e-4 x RMS (fp32).  h is the bf16 operand of the second contraction; besides fp32 accumulation
+its only error is its own rounding to bf16 (at most 2^-8 relative), which is what it is checked
+against.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_inputs import make_config, make_moe_layer, round_to_bf16
+from sparse_moe_decoder_b200 import zmoe_grouped_swiglu
+from tests.gpu_util import TOL, assert_close, host, rel_err, require_gpu, tdtype, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu(L, x_perm, offsets, M=None):
+    dt = tdtype(L.dtype)
+    M = x_perm.shape[0] if M is None else M
+    h, y = zmoe_grouped_swiglu(to_dev(x_perm[:M], dt) if M else torch.empty((0, L.d), dtype=dt, device="cuda"),
+                               to_dev(offsets, torch.int32), to_dev(L.w_gate, dt), to_dev(L.w_up, dt),
+                               to_dev(L.w_down, dt))
+    return host(h), host(y)
+
+
+def check_h(h_gpu, h_ref, kind):
+    if kind == "f32":
+        assert rel_err(h_gpu, h_ref) <= TOL["f32"]
+        return
+    bound = 2.0 ** -8 * np.abs(h_ref) + 1e-3 * np.sqrt(np.mean(h_ref ** 2))
+    assert np.all(np.abs(h_gpu - h_ref) <= bound), f"h: worst excess {np.max(np.abs(h_gpu - h_ref) - bound):.3e}"
+
+
+def routed(L):
+    sel, gates, margin, _ = oracle.route(L.x, L.w_router, L.k, L.sel_bias, L.logit_bias)
+    return oracle.permute(sel, L.E, L.x)
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_swiglu_configs(cfg):
+    require_gpu()
+    L = make_config(cfg)
+    p = routed(L)
+    h, y = run_gpu(L, p["x_perm"], p["offsets"])
+    y_ref, h_ref = oracle.grouped_swiglu(p["x_perm"], p["offsets"], L.w_gate, L.w_up, L.w_down)
+    r = assert_close(y, y_ref, L.dtype, f"config {cfg} y_perm")
+    check_h(h, h_ref, L.dtype)
+    print(f"config {cfg}: y_perm max err = {r:.2e} x RMS")
+
+
+def _offsets(counts):
+    return np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+
+
+@pytest.mark.parametrize("counts", [
+    [0, 5, 0, 1, 9, 0, 0, 33, 2, 0, 0, 0, 8, 0, 0, 1],       # empty experts, a 33-row expert (2 chunks)
+    [64] + [0] * 15,                                           # every row on one expert
+    [1] * 16,                                                  # one row each
+    [40, 90, 3, 0, 7, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 12],       # several token chunks
+])
+def test_swiglu_ragged_rows(counts):
+    require_gpu()
+    M = int(sum(counts))
+    L = make_moe_layer(M, 2048, 3072, 16, 1, "bf16", seed=M)
+    off = _offsets(counts)
+    h, y = run_gpu(L, L.x, off)
+    y_ref, h_ref = oracle.grouped_swiglu(L.x, off, L.w_gate, L.w_up, L.w_down)
+    assert_close(y, y_ref, "bf16", "ragged y_perm")
+    check_h(h, h_ref, "bf16")
+
+
+def test_swiglu_single_expert_equals_dense_ffn():
+    require_gpu()
+    L = make_moe_layer(48, 1024, 512, 1, 1, "bf16", seed=9)
+    off = np.array([0, 48], np.int32)
+    _, y = run_gpu(L, L.x, off)
+    want = oracle.swiglu_ffn(L.x, L.w_gate[0], L.w_up[0], L.w_down[0])
+    assert_close(y, want, "bf16", "dense FFN")
+
+
+def test_swiglu_rows_beyond_offsets_untouched():
+    """Rows past offsets[E] (M_total > rows) are neither read into results nor written."""
+    require_gpu()
+    L = make_moe_layer(40, 512, 256, 4, 1, "bf16", seed=4)
+    off = np.array([0, 10, 10, 25, 30], np.int32)       # 30 rows used of M_total = 40
+    dt = torch.bfloat16
+    ysent = torch.full((40, 512), 7.0, device="cuda")
+    h, y = zmoe_grouped_swiglu(to_dev(L.x, dt), to_dev(off, torch.int32), to_dev(L.w_gate, dt),
+                               to_dev(L.w_up, dt), to_dev(L.w_down, dt), y_perm=ysent)
+    y = host(y)
+    assert np.all(y[30:] == 7.0)
+    y_ref, _ = oracle.grouped_swiglu(L.x[:30], off, L.w_gate, L.w_up, L.w_down)
+    assert_close(y[:30], y_ref, "bf16", "y_perm")
+
+
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_swiglu_prefill_full_size_sampled(cfg):
+    """Full T = 16384 layer; the oracle checks a sample of rows from every expert."""
+    require_gpu()
+    L = make_config(cfg)
+    p = routed(L)
+    h, y = run_gpu(L, p["x_perm"], p["offsets"])
+    off = p["offsets"]
+    rng = np.random.default_rng(cfg)
+    for e in range(L.E):
+        a, b = int(off[e]), int(off[e + 1])
+        if b <= a:
+            continue
+        rows = np.unique(np.concatenate([[a, b - 1], rng.integers(a, b, size=min(24, b - a))]))
+        y_ref, h_ref = oracle.swiglu_ffn(p["x_perm"][rows], L.w_gate[e], L.w_up[e], L.w_down[e], return_hidden=True)
+        assert_close(y[rows], y_ref, "bf16", f"config {cfg} expert {e} y_perm")
+        check_h(h[rows], h_ref, "bf16")
