@@ -185,9 +185,11 @@ ZMOE_API zmoe_status zmoe_combine(const float* y_perm, const int32_t* inv_perm, 
                          int T, int d, int k, float* y, zmoe_stream_t stream);
 
 /*
- * Reads and clears the device error counter of the current device.  Synchronises
- * `stream` first.  *count = number of data errors seen by kernels since the last read.
- * Returns ZMOE_ERR_DEVICE_CHECK when *count > 0, ZMOE_OK otherwise.
+ * Reads and clears the device error counters of the current device.  Synchronises
+ * `stream` (and the device) first.  *count = data errors (ids or indices out of range)
+ * plus bounded device-side waits that gave up, since the last read.  Returns
+ * ZMOE_ERR_TIMEOUT when any wait gave up, else ZMOE_ERR_DEVICE_CHECK when *count > 0,
+ * else ZMOE_OK.
  */
 ZMOE_API zmoe_status zmoe_get_device_errors(zmoe_stream_t stream, uint32_t* count);
 

@@ -13,10 +13,13 @@ thread_local std::string g_last_error;
 // One error counter per device that loads this library.  Kernels receive its device
 // address as an argument; host code never dereferences it.
 __device__ unsigned int g_device_errors;
+// One timeout counter per device: kernels with bounded waits count here when a wait gives up.
+__device__ unsigned int g_device_timeouts;
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 unsigned int* g_counter_addr[kMaxDevices] = {};
+unsigned int* g_timeout_addr[kMaxDevices] = {};
 int g_sms[kMaxDevices] = {};
 int g_smem_optin[kMaxDevices] = {};
 
@@ -53,6 +56,21 @@ unsigned int* device_error_counter() {
     g_counter_addr[dev] = static_cast<unsigned int*>(p);
   }
   return g_counter_addr[dev];
+}
+
+unsigned int* device_timeout_counter() {
+  int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_timeout_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_timeouts) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_timeout_addr[dev] = static_cast<unsigned int*>(p);
+  }
+  return g_timeout_addr[dev];
 }
 
 int num_sms() {
@@ -109,17 +127,22 @@ const char* zmoe_last_error(void) { return zmoe::g_last_error.c_str(); }
 zmoe_status zmoe_get_device_errors(zmoe_stream_t stream, uint32_t* count) {
   if (!count) return zmoe::fail(ZMOE_ERR_INVALID_ARG, "zmoe_get_device_errors: count is NULL");
   *count = 0;
-  unsigned int* addr = zmoe::device_error_counter();
-  if (!addr) return zmoe::fail(ZMOE_ERR_CUDA, "zmoe_get_device_errors: no device error counter");
+  unsigned int* err = zmoe::device_error_counter();
+  unsigned int* tmo = zmoe::device_timeout_counter();
+  if (!err || !tmo) return zmoe::fail(ZMOE_ERR_CUDA, "zmoe_get_device_errors: no device counters");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  unsigned int host = 0;
-  cudaError_t e = cudaMemcpyAsync(&host, addr, sizeof(host), cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(addr, 0, sizeof(unsigned int), s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  unsigned int host[2] = {0, 0};
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&host[0], err, sizeof(unsigned int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(&host[1], tmo, sizeof(unsigned int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(err, 0, sizeof(unsigned int));
+  if (e == cudaSuccess) e = cudaMemset(tmo, 0, sizeof(unsigned int));
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return zmoe::fail(ZMOE_ERR_CUDA, std::string("zmoe_get_device_errors: ") + cudaGetErrorString(e));
-  *count = host;
+  *count = host[0] + host[1];
   zmoe::clear_error();
-  return host ? ZMOE_ERR_DEVICE_CHECK : ZMOE_OK;
+  if (host[1]) return zmoe::fail(ZMOE_ERR_TIMEOUT, "a bounded device-side wait gave up");
+  return host[0] ? ZMOE_ERR_DEVICE_CHECK : ZMOE_OK;
 }
 
 }  // extern "C"

@@ -261,6 +261,6 @@ def zmoe_get_device_errors(stream=None) -> int:
     """Reads and clears the device error counter (synchronises the stream)."""
     c = ctypes.c_uint32(0)
     st = lib().zmoe_get_device_errors(_stream(stream), ctypes.byref(c))
-    if st not in (0, 5):
+    if st not in (0, 5, 6):
         _check(st, "zmoe_get_device_errors")
     return int(c.value)

@@ -113,3 +113,23 @@ def test_swiglu_prefill_full_size_sampled(cfg):
         y_ref, h_ref = oracle.swiglu_ffn(p["x_perm"][rows], L.w_gate[e], L.w_up[e], L.w_down[e], return_hidden=True)
         assert_close(y[rows], y_ref, "bf16", f"config {cfg} expert {e} y_perm")
         check_h(h[rows], h_ref, "bf16")
+
+
+@pytest.mark.parametrize("E,d,f,counts", [
+    (1, 256, 128, [64]),                         # one m-tile, partially filled
+    (4, 256, 256, [300, 0, 129, 700]),           # ragged segments, an empty expert, tails of 44/1/60 rows
+    (2, 2048, 3072, [200, 57]),                  # full model dims: 32 / 48 k-blocks through the ring
+    (16, 512, 384, [0] * 15 + [1500]),           # everything on the last expert
+])
+def test_swiglu_tensor_core_path(E, d, f, counts):
+    """Row counts of >= 64 per expert on average take the tcgen05 GEMMs."""
+    require_gpu()
+    M = int(sum(counts))
+    assert M >= 64 * E
+    L = make_moe_layer(M, d, f, E, 1, "bf16", seed=M + d)
+    off = _offsets(counts)
+    h, y = run_gpu(L, L.x, off)
+    y_ref, h_ref = oracle.grouped_swiglu(L.x, off, L.w_gate, L.w_up, L.w_down)
+    check_h(h, h_ref, "bf16")
+    r = assert_close(y, y_ref, "bf16", "tcgen05 y_perm")
+    print(f"tcgen05 E={E} d={d} f={f}: y_perm max err {r:.2e} x RMS")
