@@ -46,6 +46,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle timing leg")
+    ap.add_argument("--weight-copies", type=int, default=0,
+                    help="device copies of the layer weights used in rotation (0: 4 for the decode step, else 1)")
     return ap.parse_args(argv)
 
 
@@ -266,7 +268,7 @@ def main(argv=None):
         L.x = round_to_bf16(rng.standard_normal(L.x.shape, dtype=np.float32))
     dt = torch.bfloat16
     W0 = MoEWeights.from_host(L)
-    n_copies = 4 if args.config == 2 else 1
+    n_copies = args.weight_copies if args.weight_copies > 0 else (4 if args.config == 2 else 1)
     Ws = [W0] + [MoEWeights(W0.w_router.clone(), W0.w_gate.clone(), W0.w_up.clone(), W0.w_down.clone(),
                             W0.sel_bias, W0.logit_bias, None, W0.k) for _ in range(n_copies - 1)]
     R = MoELayerRunner(L.T, L.E, L.d, L.f, L.k, dt)
@@ -355,7 +357,7 @@ def main(argv=None):
     touched = int((counts_all > 0).sum())
     M = int(counts_all.sum())
     weight_bytes = touched * 3 * L.f * L.d * bpe
-    act_bytes = M * L.d * bpe + 2 * M * L.f * bpe + M * L.d * 4   # x_perm in, h out + in, y_perm out
+    act_bytes = M * L.d * bpe + 2 * (M * 2 * L.f * bpe) + M * L.d * 4   # x_perm in, h pair out + in, y_perm out
     alg_bytes = weight_bytes + act_bytes
     flops = 2.0 * M * 3 * L.d * L.f
     if args.config == 2:
@@ -385,8 +387,8 @@ def main(argv=None):
             "config": {"workload": WORKLOADS[args.config], "T": L.T, "d_model": L.d, "d_ff": L.f, "E": L.E,
                        "k": L.k, "tokens_per_rank": L.T, "parallelism": f"dp{world} (replicated weights, no "
                        "data-path collective)",
-                       "l2": ("weights rotated over 4 device copies (2.4 GB > 126 MB L2)" if n_copies > 1
-                              else "inputs larger than L2 (weights 604 MB, activations >= 67 MB)"),
+                       "l2": (f"weights rotated over {n_copies} device copies ({n_copies * 0.604:.1f} GB > 126 MB L2)"
+                              if n_copies > 1 else "inputs larger than L2 (one layer's weights: 604 MB)"),
                        "experts_touched": experts_touched},
             "roofline": roof,
             "cpu_baseline": cpu,

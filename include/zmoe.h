@@ -157,16 +157,20 @@ ZMOE_API size_t zmoe_grouped_swiglu_workspace_size(int M_total, int E, int d, in
  * Per-expert SwiGLU over the permuted rows ("GLU Variants Improve Transformer",
  * [ABSTRACT] "Builds on"; SiLU per [ROUTING] section 2.1):
  *   for each expert e and each row r in [offsets[e], offsets[e + 1]):
- *     h[r]      = silu(W_gate[e] x_perm[r]) * (W_up[e] x_perm[r])     [f], stored in `dtype`
+ *     h[r]      = silu(W_gate[e] x_perm[r]) * (W_up[e] x_perm[r])     [f]
  *     y_perm[r] = W_down[e] h[r]                                      [d], stored as f32
- *   silu(z) = z / (1 + exp(-z)); contractions accumulate in fp32.  bf16 rounds h to
- *   bf16 before the second contraction (it is the operand of that contraction); y_perm
- *   leaves the fp32 accumulator unrounded.
+ *   silu(z) = z / (1 + exp(-z)); contractions accumulate in fp32.
+ *   bf16: h is kept as a pair of bf16 values, h_hi = bf16(h) and h_lo = bf16(h - h_hi),
+ *   stored side by side as h: bf16 [M_total, 2 f] (columns [0, f) = h_hi, [f, 2 f) = h_lo),
+ *   and y_perm = W_down h_hi + W_down h_lo: both tensor-core operands stay bf16 while h
+ *   carries ~16 significant bits into the second contraction.
+ *   f32: h is f32 [M_total, f].
  *   x_perm: [M_total, d]; offsets: int32 [E + 1] on the DEVICE (read by the kernels,
  *   never copied to the host); M_total = T * k is the host-side row bound and must be
- *   >= offsets[E]; w_gate, w_up: [E, f, d]; w_down: [E, d, f]; h: [M_total, f] (caller
- *   scratch that also exposes the hidden activations); y_perm: f32 [M_total, d].
- *   bf16: d % 64 == 0, f % 64 == 0; f32: d % 4 == 0, f % 4 == 0.  16-byte aligned.
+ *   >= offsets[E]; w_gate, w_up: [E, f, d]; w_down: [E, d, f]; h: caller scratch (above)
+ *   that also exposes the hidden activations; y_perm: f32 [M_total, d].  Rows at or past
+ *   offsets[E] are neither read into results nor written.
+ *   bf16: d % 256 == 0, f % 256 == 0; f32: d % 4 == 0, f % 4 == 0.  16-byte aligned.
  */
 ZMOE_API zmoe_status zmoe_grouped_swiglu(const void* x_perm, const int32_t* offsets, int M_total, const void* w_gate,
                                 const void* w_up, const void* w_down, zmoe_dtype dtype, int E, int d, int f,

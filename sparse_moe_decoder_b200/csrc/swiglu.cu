@@ -8,6 +8,8 @@
 //   f32  -> plain fp32 FMA kernels (no TF32 anywhere: one thread per output, float4 loads).
 //   bf16 -> rows per expert small (decode): weight-streaming kernels (swiglu_stream.cu);
 //           rows per expert large (prefill): tcgen05 / TMEM / TMA grouped GEMMs (swiglu_tc.cu).
+//           Both keep h as a bf16 pair h_hi + h_lo ([M, 2f]) so that the second contraction
+//           sees h to ~16 significant bits with bf16 tensor-core operands.
 #include "common.cuh"
 
 namespace zmoe {
@@ -20,6 +22,7 @@ zmoe_status grouped_swiglu_tc(const uint16_t* x_perm, const int32_t* offsets, in
                               float* y_perm, void* ws, size_t ws_bytes, cudaStream_t s);
 size_t grouped_swiglu_tc_workspace(int M_total, int E, int d, int f);
 bool grouped_swiglu_tc_supported(int d, int f);
+bool grouped_swiglu_stream_supported(int d, int f);
 
 namespace {
 
@@ -121,7 +124,7 @@ zmoe_status zmoe_grouped_swiglu(const void* x_perm, const int32_t* offsets, int 
                                                            static_cast<const float*>(w_down), y_perm);
     return check_launch("zmoe_grouped_swiglu (f32)");
   }
-  ZMOE_REQUIRE(d % 64 == 0 && f % 64 == 0, "zmoe_grouped_swiglu: bf16 needs d % 64 == 0 and f % 64 == 0");
+  ZMOE_REQUIRE(d % 256 == 0 && f % 256 == 0, "zmoe_grouped_swiglu: bf16 needs d % 256 == 0 and f % 256 == 0");
   const auto* xp = static_cast<const uint16_t*>(x_perm);
   const auto* wg = static_cast<const uint16_t*>(w_gate);
   const auto* wu = static_cast<const uint16_t*>(w_up);

@@ -1,29 +1,31 @@
 // Grouped SwiGLU for decode-size batches: weight streaming (HBM-bound).
 //
 // Per expert e (rows offsets[e]..offsets[e+1] of the permuted activations):
-//   h = silu(x W_gate[e]^T) * (x W_up[e]^T)      (bf16, the operand of the next contraction)
-//   y = h W_down[e]^T                              (fp32)
+//   h = silu(x W_gate[e]^T) * (x W_up[e]^T)       kept as a bf16 pair h ~= h_hi + h_lo
+//   y = h W_down[e]^T = h_hi W_down^T + h_lo W_down^T     (fp32)
 // ("GLU Variants Improve Transformer", ZONOS2 Technical Report "Builds on"; SiLU per the
 // telknet.cc article on ZONOS2, section 2.1.)
 //
 // With a handful of rows per expert the contraction has ~8 FLOP per weight byte: the time is
 // the time to stream every touched expert's weights from HBM once.  Design:
 //   * One persistent CTA per SM, 16 warps.  Work units are (expert, token chunk, 16 weight
-//     rows); each CTA takes a contiguous, equal share of the unit list (read on the device from
-//     `offsets`, so no host round trip), which keeps every SM's byte count within one unit.
-//   * A unit's K range is dealt in 64-wide chunks round-robin to the 16 warps; a warp loads its
-//     weight fragments straight from global memory with 16-byte streaming loads
-//     (L1::no_allocate, L2 evict-first) and keeps kDepth chunks in flight (~96 KB per SM).
+//     rows); each CTA takes a contiguous, equal share of the unit list (computed on the device
+//     from `offsets`, so no host round trip), which balances bytes per SM to within one unit.
+//   * A WARP owns a whole unit: it streams the unit's 16 weight rows over the full K with
+//     16-byte loads (L1::no_allocate, L2 evict-first) kept kDepth 64-wide chunks deep in
+//     registers, and finishes the unit alone -- no cross-warp reduction, no barrier per unit.
+//     The load cursor runs ahead across unit (and token-chunk) boundaries.
 //   * Swap-AB on the tensor cores: weight rows are the MMA's M = 16, tokens are N = 8
 //     (mma.sync m16n8k16, bf16 in, fp32 accumulate).  The physical k order inside a chunk is
 //     permuted identically for A and B so that each lane's 16-byte load lands directly in its
-//     A-fragment registers; the token rows (B) sit in shared memory with a 64-byte row pad
-//     that makes the 16-byte fragment reads bank-conflict free.
+//     A-fragment registers.  Only the token groups that hold rows are multiplied.
+//   * The CTA stages the current (expert, token chunk) rows in shared memory (64-byte row pad:
+//     conflict-free 16-byte fragment reads); it re-stages, between two CTA barriers, only when
+//     its unit range crosses into the next chunk (once or twice per CTA).
 //   * Gate/up units pair 8 gate rows (MMA rows 0..7) with the 8 matching up rows (rows 8..15),
 //     so each lane's accumulator holds gate and up of the same (feature, token): SiLU * up is
-//     applied in registers in the epilogue.  Down units are 16 rows of W_down.
-//   * The 16 warps' partial sums are added through shared memory (double-buffered, one CTA
-//     barrier per unit).
+//     applied in registers and h is stored as h_hi = bf16(h), h_lo = bf16(h - h_hi).  Down
+//     units are 16 rows of W_down; each A fragment is multiplied by the h_hi and h_lo rows.
 #include "common.cuh"
 
 namespace zmoe {
@@ -37,11 +39,11 @@ constexpr int kMaxE = 64;
 enum { kGateUp = 0, kDown = 1 };
 
 struct StreamArgs {
-  const uint16_t* a0;       // gate/up: W_gate [E, R, K];  down: W_down [E, R, K]
-  const uint16_t* a1;       // gate/up: W_up   [E, R, K];  down: unused
-  const uint16_t* x;        // gate/up: x_perm [M, K];     down: h [M, K]
+  const uint16_t* w0;       // gate/up: W_gate [E, R, K];  down: W_down [E, R, K]
+  const uint16_t* w1;       // gate/up: W_up   [E, R, K];  down: unused
+  const uint16_t* x;        // gate/up: x_perm [M, K];     down: h pair [M, 2K] (h_hi | h_lo)
   const int32_t* offsets;   // [E + 1], device
-  void* out;                // gate/up: h bf16 [M, R];     down: y_perm f32 [M, R]
+  void* out;                // gate/up: h pair bf16 [M, 2R]; down: y_perm f32 [M, R]
   int E, K, R, tokc;
 };
 
@@ -74,212 +76,222 @@ struct Frag {
   uint4 lo0, lo1, hi0, hi1;
 };
 
-// Position of a unit in the (expert, chunk, row block) grid, plus its row pointers.
-struct UnitPos {
-  int e, chunk, nb;
-  int row0, rows;               // first permuted row of the chunk, rows in it (<= tokc)
-  const uint16_t* lo;           // this lane's A row g at k = q*8
-  const uint16_t* hi;           // this lane's A row g + 8 at k = q*8
-};
+// The four MMAs of one chunk against one group of 8 token rows (b0: k = q*8.., b1: k = 32+q*8..).
+__device__ __forceinline__ void mma_chunk(float (&c)[4], const Frag& f, const uint4& b0, const uint4& b1) {
+  mma16816(c, f.lo0.x, f.hi0.x, f.lo0.y, f.hi0.y, b0.x, b0.y);
+  mma16816(c, f.lo0.z, f.hi0.z, f.lo0.w, f.hi0.w, b0.z, b0.w);
+  mma16816(c, f.lo1.x, f.hi1.x, f.lo1.y, f.hi1.y, b1.x, b1.y);
+  mma16816(c, f.lo1.z, f.hi1.z, f.lo1.w, f.hi1.w, b1.z, b1.w);
+}
 
+// Unit u -> segment (expert, token chunk) index u / nblk and row block u % nblk.
+__device__ __forceinline__ void seg_of(int s, const int* seg_start, const int* off, int E, int tokc, int& e,
+                                       int& row0, int& rows) {
+  e = 0;
+  while (e + 1 < E && seg_start[e + 1] <= s) ++e;
+  row0 = off[e] + (s - seg_start[e]) * tokc;
+  const int left = off[e + 1] - row0;
+  rows = left < tokc ? left : tokc;
+}
+
+// This lane's A row pointers (row g and row g + 8 of the unit, at k = q*8).
 template <int MODE>
-__device__ __forceinline__ UnitPos locate(long long u, const int* unit_start, const int* off, const StreamArgs& a,
-                                          int nblk, int lane) {
+__device__ __forceinline__ void unit_rows(const StreamArgs& a, int e, int nb, int lane, const uint16_t*& lo,
+                                          const uint16_t*& hi) {
   constexpr int FEAT = (MODE == kGateUp) ? 8 : 16;
-  UnitPos p;
-  int e = 0;
-  while (e + 1 < a.E && unit_start[e + 1] <= u) ++e;
-  const int local = static_cast<int>(u - unit_start[e]);
-  p.e = e;
-  p.chunk = local / nblk;
-  p.nb = local - p.chunk * nblk;
-  p.row0 = off[e] + p.chunk * a.tokc;
-  const int left = off[e + 1] - p.row0;
-  p.rows = left < a.tokc ? left : a.tokc;
   const int g = lane >> 2, q = lane & 3;
-  const size_t row = static_cast<size_t>(e) * a.R + static_cast<size_t>(p.nb) * FEAT + g;
-  p.lo = a.a0 + row * a.K + q * 8;
-  p.hi = (MODE == kGateUp) ? a.a1 + row * a.K + q * 8 : p.lo + static_cast<size_t>(8) * a.K;
-  return p;
+  const size_t row = static_cast<size_t>(e) * a.R + static_cast<size_t>(nb) * FEAT + g;
+  lo = a.w0 + row * a.K + q * 8;
+  hi = (MODE == kGateUp) ? a.w1 + row * a.K + q * 8 : lo + static_cast<size_t>(8) * a.K;
 }
 
 template <int MODE, int NG>
 __global__ void __launch_bounds__(kThreads, 1) stream_ffn_kernel(StreamArgs a) {
   constexpr int FEAT = (MODE == kGateUp) ? 8 : 16;
+  constexpr bool SPLIT = (MODE == kDown);   // the down contraction multiplies h_hi and h_lo
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  __shared__ int unit_start[kMaxE + 1];
+  __shared__ int seg_start[kMaxE + 1];
   __shared__ int off[kMaxE + 1];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, q = lane & 3;
   const int K = a.K;
-  const int srow = K + 32;                       // shared row stride (elements): conflict-free
-  const int nkc = K / 64;                        // 64-wide chunks per unit
-  const int per = (nkc + kWarps - 1) / kWarps;   // chunk slots per warp per unit
+  const int xld = SPLIT ? 2 * K : K;              // staged row length
+  const int srow = xld + 32;                      // shared row stride (elements): conflict-free
+  const int nkc = K / 64;                         // chunks per unit (a multiple of kDepth)
   const int nblk = a.R / FEAT;
   const int tokc = a.tokc;
-
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);                                     // [tokc][srow]
-  float4* red = reinterpret_cast<float4*>(smem_raw + static_cast<size_t>(tokc) * srow * 2);  // [2][16][NG][32]
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);   // [tokc][srow]
 
   if (tid <= a.E) off[tid] = a.offsets[tid];
   __syncthreads();
   if (tid == 0) {
     int acc = 0;
     for (int e = 0; e < a.E; ++e) {
-      unit_start[e] = acc;
-      const int m = off[e + 1] - off[e];
-      acc += ((m + tokc - 1) / tokc) * nblk;
+      seg_start[e] = acc;
+      acc += (off[e + 1] - off[e] + tokc - 1) / tokc;
     }
-    unit_start[a.E] = acc;
+    seg_start[a.E] = acc;
   }
   __syncthreads();
 
-  const long long U = unit_start[a.E];
-  const long long u_begin = U * blockIdx.x / gridDim.x;
-  const long long u_end = U * (blockIdx.x + 1) / gridDim.x;
-  const long long S = (u_end - u_begin) * per;   // chunk slots this warp walks through
-  if (S == 0) return;
+  // unit indices fit in int: (rows / 8 + E) segments x at most d / 8 row blocks
+  const int U = seg_start[a.E] * nblk;
+  const int u_begin = static_cast<int>(static_cast<long long>(U) * blockIdx.x / gridDim.x);
+  const int u_end = static_cast<int>(static_cast<long long>(U) * (blockIdx.x + 1) / gridDim.x);
+  if (u_begin >= u_end) return;
+  const int s_first = u_begin / nblk;
+  const int s_last = (u_end - 1) / nblk;
+
+  // This warp's units: in every segment s, lo(s) + warp, lo(s) + warp + 16, ... below hi(s).
+  auto first_in = [&](int s) -> int {
+    const int lo = max(s * nblk, u_begin);
+    const int hi = min((s + 1) * nblk, u_end);
+    return lo + warp < hi ? lo + warp : -1;
+  };
+  auto next_unit = [&](int u) -> int {
+    const int s = u / nblk;
+    const int hi = min((s + 1) * nblk, u_end);
+    if (u + kWarps < hi) return u + kWarps;
+    for (int s2 = s + 1; s2 <= s_last; ++s2) {
+      const int c = first_in(s2);
+      if (c >= 0) return c;
+    }
+    return -1;
+  };
 
   const uint64_t pol = evict_first_policy();
 
-  // load cursor (runs kDepth slots ahead of the compute cursor)
-  long long lu = u_begin;
-  int lj = 0;
-  UnitPos lp = locate<MODE>(lu, unit_start, off, a, nblk, lane);
-
+  // ---- load cursor: unit lu, chunk lc ----
+  int lu = -1;
+  for (int s = s_first; s <= s_last && lu < 0; ++s) lu = first_in(s);
+  int lc = 0;
+  const uint16_t* llo = nullptr;
+  const uint16_t* lhi = nullptr;
+  auto point_load_cursor = [&]() {
+    if (lu < 0) return;
+    int e, row0, rows;
+    seg_of(lu / nblk, seg_start, off, a.E, tokc, e, row0, rows);
+    unit_rows<MODE>(a, e, lu % nblk, lane, llo, lhi);
+  };
+  point_load_cursor();
   auto issue = [&](Frag& f) {
-    const int kc = warp + kWarps * lj;
-    if (lu < u_end && kc < nkc) {
-      const int kb = kc * 64;
-      f.lo0 = ldg_weights(lp.lo + kb, pol);
-      f.lo1 = ldg_weights(lp.lo + kb + 32, pol);
-      f.hi0 = ldg_weights(lp.hi + kb, pol);
-      f.hi1 = ldg_weights(lp.hi + kb + 32, pol);
-    }
-    if (++lj == per) {
-      lj = 0;
-      ++lu;
-      if (lu < u_end) lp = locate<MODE>(lu, unit_start, off, a, nblk, lane);
+    if (lu >= 0) {
+      const int kb = lc * 64;
+      f.lo0 = ldg_weights(llo + kb, pol);
+      f.lo1 = ldg_weights(llo + kb + 32, pol);
+      f.hi0 = ldg_weights(lhi + kb, pol);
+      f.hi1 = ldg_weights(lhi + kb + 32, pol);
+      if (++lc == nkc) {
+        lc = 0;
+        lu = next_unit(lu);
+        point_load_cursor();
+      }
     }
   };
-
   Frag buf[kDepth];
 #pragma unroll
   for (int r = 0; r < kDepth; ++r) issue(buf[r]);
 
-  // compute cursor
-  long long cu = u_begin;
-  int cj = 0;
-  UnitPos cp;
-  int tile_e = -1, tile_chunk = -1;
-  int parity = 0;
-  float acc[NG][4];
-#pragma unroll
-  for (int j = 0; j < NG; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  // ---- segments of this CTA ----
+  for (int s = s_first; s <= s_last; ++s) {
+    int e, row0, rows;
+    seg_of(s, seg_start, off, a.E, tokc, e, row0, rows);
+    const int ng = (rows + 7) >> 3;                 // token groups that hold rows
+    __syncthreads();                                // every warp is done with the previous rows
+    {
+      const int vpr = xld / 8;
+      const uint4* src = reinterpret_cast<const uint4*>(a.x);
+      for (int i = tid; i < ng * 8 * vpr; i += kThreads) {
+        const int rr = i / vpr, v = i - rr * vpr;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (rr < rows) val = src[static_cast<size_t>(row0 + rr) * vpr + v];
+        *reinterpret_cast<uint4*>(xs + static_cast<size_t>(rr) * srow + v * 8) = val;
+      }
+    }
+    __syncthreads();
 
-  for (long long s0 = 0; s0 < S; s0 += kDepth) {
+    for (int u = first_in(s); u >= 0 && u / nblk == s; u = next_unit(u)) {
+      const int nb = u % nblk;
+      float acc[NG][4];
 #pragma unroll
-    for (int r = 0; r < kDepth; ++r) {
-      if (s0 + r < S) {
-        if (cj == 0) {
-          cp = locate<MODE>(cu, unit_start, off, a, nblk, lane);
-          if (cp.e != tile_e || cp.chunk != tile_chunk) {
-            // Stage this chunk's token rows (zero-padded to tokc).  Every warp has passed the
-            // previous unit's barrier, so nobody still reads the old tile.
-            const int vpr = K / 8;
-            const uint4* src = reinterpret_cast<const uint4*>(a.x);
-            for (int i = tid; i < tokc * vpr; i += kThreads) {
-              const int rr = i / vpr, v = i - rr * vpr;
-              uint4 val = make_uint4(0u, 0u, 0u, 0u);
-              if (rr < cp.rows) val = src[static_cast<size_t>(cp.row0 + rr) * vpr + v];
-              *reinterpret_cast<uint4*>(xs + static_cast<size_t>(rr) * srow + v * 8) = val;
-            }
-            tile_e = cp.e;
-            tile_chunk = cp.chunk;
-            __syncthreads();
-          }
-        }
-        const int kc = warp + kWarps * cj;
-        if (kc < nkc) {
+      for (int j = 0; j < NG; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+
+      for (int c0 = 0; c0 < nkc; c0 += kDepth) {
+#pragma unroll
+        for (int r = 0; r < kDepth; ++r) {
           const Frag& f = buf[r];
-          const int kb = kc * 64;
+          const int kb = (c0 + r) * 64;
 #pragma unroll
           for (int j = 0; j < NG; ++j) {
-            const uint16_t* xr = xs + static_cast<size_t>(j * 8 + g) * srow + kb + q * 8;
-            const uint4 b0 = *reinterpret_cast<const uint4*>(xr);
-            const uint4 b1 = *reinterpret_cast<const uint4*>(xr + 32);
-            mma16816(acc[j], f.lo0.x, f.hi0.x, f.lo0.y, f.hi0.y, b0.x, b0.y);
-            mma16816(acc[j], f.lo0.z, f.hi0.z, f.lo0.w, f.hi0.w, b0.z, b0.w);
-            mma16816(acc[j], f.lo1.x, f.hi1.x, f.lo1.y, f.hi1.y, b1.x, b1.y);
-            mma16816(acc[j], f.lo1.z, f.hi1.z, f.lo1.w, f.hi1.w, b1.z, b1.w);
+            if (j < ng) {
+              const uint16_t* xr = xs + static_cast<size_t>(j * 8 + g) * srow + kb + q * 8;
+              const uint4 b0 = *reinterpret_cast<const uint4*>(xr);
+              const uint4 b1 = *reinterpret_cast<const uint4*>(xr + 32);
+              mma_chunk(acc[j], f, b0, b1);
+              if (SPLIT) {
+                const uint4 l0 = *reinterpret_cast<const uint4*>(xr + K);
+                const uint4 l1 = *reinterpret_cast<const uint4*>(xr + K + 32);
+                mma_chunk(acc[j], f, l0, l1);
+              }
+            }
           }
+          issue(buf[r]);                           // refill the slot: kDepth - 1 chunks stay in flight
         }
-        issue(buf[r]);
-        if (++cj == per) {
-          // end of unit: reduce the 16 warps' partial sums and write the outputs
-          float4* rb = red + static_cast<size_t>(parity) * kWarps * NG * 32;
+      }
+
+      // epilogue of the unit, straight from this warp's accumulators
 #pragma unroll
-          for (int j = 0; j < NG; ++j) {
-            rb[(warp * NG + j) * 32 + lane] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-            acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-          }
-          __syncthreads();
-          if (tid < NG * 32) {
-            const int j = tid >> 5;
-            float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) {
-              const float4 v = rb[(w * NG + j) * 32 + lane];
-              c.x += v.x;
-              c.y += v.y;
-              c.z += v.z;
-              c.w += v.w;
+      for (int j = 0; j < NG; ++j) {
+        if (j < ng) {
+          const int t0 = j * 8 + 2 * q, t1 = t0 + 1;
+          const int n = nb * FEAT + g;
+          if (MODE == kGateUp) {
+            uint16_t* h = static_cast<uint16_t*>(a.out);
+            const size_t ld = static_cast<size_t>(2) * a.R;
+            const float h0 = acc[j][0] / (1.f + expf(-acc[j][0])) * acc[j][2];
+            const float h1 = acc[j][1] / (1.f + expf(-acc[j][1])) * acc[j][3];
+            const uint16_t h0_hi = f32_to_bf16_bits(h0), h1_hi = f32_to_bf16_bits(h1);
+            if (t0 < rows) {
+              h[(row0 + t0) * ld + n] = h0_hi;
+              h[(row0 + t0) * ld + a.R + n] = f32_to_bf16_bits(h0 - bf16_to_f32(h0_hi));
             }
-            const int t0 = j * 8 + 2 * q, t1 = t0 + 1;
-            const int n = cp.nb * FEAT + g;
-            if (MODE == kGateUp) {
-              uint16_t* h = static_cast<uint16_t*>(a.out);
-              if (t0 < cp.rows) h[static_cast<size_t>(cp.row0 + t0) * a.R + n] = f32_to_bf16_bits(c.x / (1.f + expf(-c.x)) * c.z);
-              if (t1 < cp.rows) h[static_cast<size_t>(cp.row0 + t1) * a.R + n] = f32_to_bf16_bits(c.y / (1.f + expf(-c.y)) * c.w);
-            } else {
-              float* y = static_cast<float*>(a.out);
-              if (t0 < cp.rows) {
-                y[static_cast<size_t>(cp.row0 + t0) * a.R + n] = c.x;
-                y[static_cast<size_t>(cp.row0 + t0) * a.R + n + 8] = c.z;
-              }
-              if (t1 < cp.rows) {
-                y[static_cast<size_t>(cp.row0 + t1) * a.R + n] = c.y;
-                y[static_cast<size_t>(cp.row0 + t1) * a.R + n + 8] = c.w;
-              }
+            if (t1 < rows) {
+              h[(row0 + t1) * ld + n] = h1_hi;
+              h[(row0 + t1) * ld + a.R + n] = f32_to_bf16_bits(h1 - bf16_to_f32(h1_hi));
+            }
+          } else {
+            float* y = static_cast<float*>(a.out);
+            if (t0 < rows) {
+              y[static_cast<size_t>(row0 + t0) * a.R + n] = acc[j][0];
+              y[static_cast<size_t>(row0 + t0) * a.R + n + 8] = acc[j][2];
+            }
+            if (t1 < rows) {
+              y[static_cast<size_t>(row0 + t1) * a.R + n] = acc[j][1];
+              y[static_cast<size_t>(row0 + t1) * a.R + n + 8] = acc[j][3];
             }
           }
-          parity ^= 1;
-          cj = 0;
-          ++cu;
         }
       }
     }
   }
 }
 
-size_t stream_smem_bytes(int K, int tokc) {
-  const int ng = tokc / 8;
-  return static_cast<size_t>(tokc) * (K + 32) * 2 + static_cast<size_t>(2) * kWarps * ng * 32 * sizeof(float4);
-}
+size_t stream_smem_bytes(int xld, int tokc) { return static_cast<size_t>(tokc) * (xld + 32) * 2; }
 
-// Largest token chunk (multiple of 8, <= 32) whose tile fits the device's shared memory.
-int pick_tokc(int K) {
+// Largest token chunk (multiple of 8, <= 24: three token groups keep the kernel within 128
+// registers) whose staged rows fit the device's shared memory.
+int pick_tokc(int xld) {
   const size_t cap = static_cast<size_t>(max_smem_optin()) - 1024;   // static smem of the kernel
-  for (int tokc = 32; tokc >= 8; tokc -= 8)
-    if (stream_smem_bytes(K, tokc) <= cap) return tokc;
+  for (int tokc = 24; tokc >= 8; tokc -= 8)
+    if (stream_smem_bytes(xld, tokc) <= cap) return tokc;
   return 0;
 }
 
 template <int MODE, int NG>
 zmoe_status launch_stream_ng(const StreamArgs& a, cudaStream_t s) {
   auto kern = stream_ffn_kernel<MODE, NG>;
-  const size_t smem = stream_smem_bytes(a.K, a.tokc);
+  const size_t smem = stream_smem_bytes(MODE == kDown ? 2 * a.K : a.K, a.tokc);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return check_launch("grouped_swiglu (stream): shared memory attribute");
   kern<<<num_sms(), kThreads, smem, s>>>(a);
@@ -291,22 +303,25 @@ zmoe_status launch_stream(const StreamArgs& a, cudaStream_t s) {
   switch (a.tokc / 8) {
     case 1: return launch_stream_ng<MODE, 1>(a, s);
     case 2: return launch_stream_ng<MODE, 2>(a, s);
-    case 3: return launch_stream_ng<MODE, 3>(a, s);
-    default: return launch_stream_ng<MODE, 4>(a, s);
+    default: return launch_stream_ng<MODE, 3>(a, s);
   }
 }
 
 }  // namespace
 
-// bf16 grouped SwiGLU by weight streaming (any rows per expert; efficient for <= 32).
+bool grouped_swiglu_stream_supported(int d, int f) {
+  return d % (64 * kDepth) == 0 && f % (64 * kDepth) == 0 && pick_tokc(d) > 0 && pick_tokc(2 * f) > 0;
+}
+
+// bf16 grouped SwiGLU by weight streaming (any rows per expert; efficient up to one token chunk).
+// h: bf16 [M, 2f] (h_hi | h_lo); y_perm: f32 [M, d].
 zmoe_status grouped_swiglu_stream(const uint16_t* x_perm, const int32_t* offsets, const uint16_t* w_gate,
                                   const uint16_t* w_up, const uint16_t* w_down, int E, int d, int f, uint16_t* h,
                                   float* y_perm, cudaStream_t s) {
-  if (d % 64 != 0 || f % 64 != 0 || E > kMaxE)
-    return fail(ZMOE_ERR_UNSUPPORTED, "grouped_swiglu (stream): needs d % 64 == 0, f % 64 == 0, E <= 64");
+  if (!grouped_swiglu_stream_supported(d, f) || E > kMaxE)
+    return fail(ZMOE_ERR_UNSUPPORTED, "grouped_swiglu (stream): needs d % 256 == 0, f % 256 == 0, E <= 64");
   StreamArgs gu{w_gate, w_up, x_perm, offsets, h, E, d, f, pick_tokc(d)};
-  StreamArgs dn{w_down, nullptr, h, offsets, y_perm, E, f, d, pick_tokc(f)};
-  if (gu.tokc == 0 || dn.tokc == 0) return fail(ZMOE_ERR_UNSUPPORTED, "grouped_swiglu (stream): d or f too large");
+  StreamArgs dn{w_down, nullptr, h, offsets, y_perm, E, f, d, pick_tokc(2 * f)};
   zmoe_status st = launch_stream<kGateUp>(gu, s);
   if (st != ZMOE_OK) return st;
   return launch_stream<kDown>(dn, s);

@@ -2,8 +2,11 @@
 //
 // Per expert e over its rows of the permuted activations ("GLU Variants Improve Transformer",
 // ZONOS2 Technical Report "Builds on"; SiLU per the telknet.cc article on ZONOS2, section 2.1):
-//   gate/up GEMM:  [G | U] = X_e [W_gate,e ; W_up,e]^T,   h = silu(G) * U  -> bf16
-//   down GEMM:     y_perm  = h_e W_down,e^T                               -> fp32
+//   gate/up GEMM:  [G | U] = X_e [W_gate,e ; W_up,e]^T,   h = silu(G) * U
+//                  h is stored as a bf16 pair [h_hi | h_lo], h_hi = bf16(h), h_lo = bf16(h - h_hi)
+//   down GEMM:     y_perm  = [h_hi | h_lo]_e [W_down,e | W_down,e]^T   (K = 2f)  -> fp32
+// Carrying h to ~16 significant bits keeps the bf16 rounding of h out of the result (a single
+// bf16 h costs up to 3% of the output RMS on skewed gates); both MMA operands stay bf16.
 //
 // One persistent CTA per SM, 192 threads in three roles:
 //   warp 0      TMA producer: 2D tiled bulk-tensor loads (128-byte swizzle, no multicast) of a
@@ -49,7 +52,9 @@ enum { kGateUp = 0, kDown = 1 };
 struct TcParams {
   const int32_t* offsets;
   void* out;                 // gate/up: h bf16 [M, f]; down: y_perm f32 [M, d]
-  int E, K, out_ld;          // contraction length; row length of `out`
+  int E, K, out_ld;          // contraction length (A columns); row length of `out`
+  int lo_offset;             // gate/up: column of h_lo in `out` (= f)
+  int kb_wrap;               // B's k-block index is kb % kb_wrap (down: f / 64; gate/up: K / 64)
   int b_rows_per_expert;     // f (gate/up) or d (down)
   int n_tiles;               // n-tiles per m-tile
   unsigned int* timeouts;
@@ -266,13 +271,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(&C.full[s], STAGE_BYTES);
           unsigned char* sa = stages + s * STAGE_BYTES;
           unsigned char* sb = sa + A_BYTES;
+          const int kbb = (kb % p.kb_wrap) * BK;
           tma_load_2d(sa, &mapA, &C.full[s], kb * BK, arow);
           if (MODE == kGateUp) {
-            tma_load_2d(sb, &mapB0, &C.full[s], kb * BK, brow);
-            tma_load_2d(sb + B_HALF, &mapB1, &C.full[s], kb * BK, brow);
+            tma_load_2d(sb, &mapB0, &C.full[s], kbb, brow);
+            tma_load_2d(sb + B_HALF, &mapB1, &C.full[s], kbb, brow);
           } else {
-            tma_load_2d(sb, &mapB0, &C.full[s], kb * BK, brow);
-            tma_load_2d(sb + B_HALF, &mapB0, &C.full[s], kb * BK, brow + 128);
+            tma_load_2d(sb, &mapB0, &C.full[s], kbb, brow);
+            tma_load_2d(sb + B_HALF, &mapB0, &C.full[s], kbb, brow + 128);
           }
         }
         if (!ok) break;
@@ -348,17 +354,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(taddr + 128 + c * 32, u);
           tmem_wait_ld();
           if (valid) {
-            uint32_t packed[16];
+            uint32_t hi[16], lo[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
               const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-              packed[i] = pack_bf16x2(g0 / (1.f + expf(-g0)) * u0, g1 / (1.f + expf(-g1)) * u1);
+              const float h0 = g0 / (1.f + expf(-g0)) * u0, h1 = g1 / (1.f + expf(-g1)) * u1;
+              hi[i] = pack_bf16x2(h0, h1);
+              lo[i] = pack_bf16x2(h0 - __uint_as_float(hi[i] << 16), h1 - __uint_as_float(hi[i] & 0xFFFF0000u));
             }
             uint4* dst = reinterpret_cast<uint4*>(h + c * 32);
+            uint4* dlo = reinterpret_cast<uint4*>(h + p.lo_offset + c * 32);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            for (int j = 0; j < 4; ++j) {
+              dst[j] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
+              dlo[j] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
+            }
           }
         }
       } else {
@@ -465,14 +476,14 @@ zmoe_status grouped_swiglu_tc(const uint16_t* x_perm, const int32_t* offsets, in
     return fail(ZMOE_ERR_UNSUPPORTED, "grouped_swiglu (tcgen05): needs d % 256 == 0, f % 128 == 0, E <= 64");
   CUtensorMap mx, mg, mu, mh, md;
   if (!make_map(&mx, x_perm, d, M_total, BM) || !make_map(&mg, w_gate, d, static_cast<uint64_t>(E) * f, 128) ||
-      !make_map(&mu, w_up, d, static_cast<uint64_t>(E) * f, 128) || !make_map(&mh, h, f, M_total, BM) ||
+      !make_map(&mu, w_up, d, static_cast<uint64_t>(E) * f, 128) || !make_map(&mh, h, 2 * f, M_total, BM) ||
       !make_map(&md, w_down, f, static_cast<uint64_t>(E) * d, 128))
     return fail(ZMOE_ERR_CUDA, "grouped_swiglu (tcgen05): cuTensorMapEncodeTiled failed");
   unsigned int* tmo = device_timeout_counter();
-  TcParams gu{offsets, h, E, d, f, f, f / 128, tmo};
+  TcParams gu{offsets, h, E, d, 2 * f, f, d / BK, f, f / 128, tmo};
   zmoe_status st = launch_tc<kGateUp>(mx, mg, mu, gu, s);
   if (st != ZMOE_OK) return st;
-  TcParams dn{offsets, y_perm, E, f, d, d, d / 256, tmo};
+  TcParams dn{offsets, y_perm, E, 2 * f, d, 0, f / BK, d, d / 256, tmo};
   return launch_tc<kDown>(mh, md, md, dn, s);
 }
 

@@ -79,7 +79,7 @@ class MoELayerRunner:
                               inv_perm=torch.empty((T, k), dtype=torch.int32, device=dev),
                               x_perm=torch.empty((M, d), dtype=dtype, device=dev))
         self.perm_ws = torch.empty(max(Z.zmoe_permute_workspace_size(T, E, k), 16), dtype=torch.uint8, device=dev)
-        self.h = torch.empty((M, f), dtype=dtype, device=dev)
+        self.h = torch.empty((M, Z.hidden_cols(f, dtype)), dtype=dtype, device=dev)
         self.y_perm = torch.empty((M, d), dtype=torch.float32, device=dev)
         self.ffn_ws = torch.empty(max(Z.zmoe_grouped_swiglu_workspace_size(M, E, d, f, dtype), 16),
                                   dtype=torch.uint8, device=dev)

@@ -217,10 +217,16 @@ def zmoe_grouped_swiglu_workspace_size(M_total: int, E: int, d: int, f: int, dty
     return int(lib().zmoe_grouped_swiglu_workspace_size(M_total, E, d, f, _dtype_code(dtype)))
 
 
+def hidden_cols(f: int, dtype: torch.dtype) -> int:
+    """Columns of the h scratch of zmoe_grouped_swiglu: 2f (h_hi | h_lo) for bf16, f for f32."""
+    return 2 * f if dtype == torch.bfloat16 else f
+
+
 def zmoe_grouped_swiglu(x_perm: torch.Tensor, offsets: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
                         w_down: torch.Tensor, h: Optional[torch.Tensor] = None, y_perm: Optional[torch.Tensor] = None,
                         workspace: Optional[torch.Tensor] = None, stream=None):
-    """Returns (h [M, f] in x's dtype, y_perm f32 [M, d])."""
+    """Returns (h, y_perm f32 [M, d]).  h is bf16 [M, 2f] = [h_hi | h_lo] for bf16 inputs
+    (h ~= h_hi + h_lo), f32 [M, f] for f32 inputs."""
     _need(x_perm, "x_perm", None, 2)
     _need(offsets, "offsets", torch.int32, 1)
     for t, n in ((w_gate, "w_gate"), (w_up, "w_up"), (w_down, "w_down")):
@@ -229,7 +235,7 @@ def zmoe_grouped_swiglu(x_perm: torch.Tensor, offsets: torch.Tensor, w_gate: tor
     E, f, _ = w_gate.shape
     dev = x_perm.device
     if h is None:
-        h = torch.empty((M, f), dtype=x_perm.dtype, device=dev)
+        h = torch.empty((M, hidden_cols(f, x_perm.dtype)), dtype=x_perm.dtype, device=dev)
     if y_perm is None:
         y_perm = torch.empty((M, d), dtype=torch.float32, device=dev)
     ws_bytes = zmoe_grouped_swiglu_workspace_size(M, E, d, f, x_perm.dtype)

@@ -27,8 +27,9 @@ def check(idx, x, E, dt):
     for key in ("counts", "offsets", "perm", "inv_perm"):
         assert np.array_equal(host(out[key]), want[key]), key
     rows = int(want["offsets"][-1])
-    got_x = host(out["x_perm"])[:rows]
-    assert np.array_equal(got_x.view(np.uint32) if dt == torch.float32 else got_x, want["x_perm"][:rows])
+    got_x = np.ascontiguousarray(host(out["x_perm"])[:rows], np.float32)
+    want_x = np.ascontiguousarray(want["x_perm"][:rows], np.float32)
+    assert np.array_equal(got_x.view(np.uint32), want_x.view(np.uint32))      # bit-exact copy
     return out
 
 

@@ -1,9 +1,9 @@
 """Grouped SwiGLU on the GPU vs the oracle.
 
 y_perm (fp32 result) is held to the parity bar: max |gpu - oracle| <= 2e-2 x RMS (bf16 weights)
-or 1e-4 x RMS (fp32).  h is the bf16 operand of the second contraction; besides fp32 accumulation
-its only error is its own rounding to bf16 (at most 2^-8 relative), which is what it is checked
-against.
+or 1e-4 x RMS (fp32).  For bf16 the hidden activation comes back as the pair [h_hi | h_lo]; its
+sum carries h to ~16 significant bits, which is what it is checked against (2^-16 relative for
+the pair, plus fp32 accumulation).
 """
 import numpy as np
 import pytest
@@ -30,8 +30,14 @@ def check_h(h_gpu, h_ref, kind):
     if kind == "f32":
         assert rel_err(h_gpu, h_ref) <= TOL["f32"]
         return
-    bound = 2.0 ** -8 * np.abs(h_ref) + 1e-3 * np.sqrt(np.mean(h_ref ** 2))
-    assert np.all(np.abs(h_gpu - h_ref) <= bound), f"h: worst excess {np.max(np.abs(h_gpu - h_ref) - bound):.3e}"
+    f = h_ref.shape[1]
+    assert h_gpu.shape[1] == 2 * f
+    hi, lo = h_gpu[:, :f].astype(np.float64), h_gpu[:, f:].astype(np.float64)
+    assert np.all(np.abs(lo) <= 2.0 ** -8 * np.abs(hi) + 1e-30), "h_lo must be a remainder of h_hi"
+    rms = np.sqrt(np.mean(h_ref ** 2))
+    bound = (2.0 ** -16 + 4e-6) * np.abs(h_ref) + 1e-5 * rms
+    err = np.abs(hi + lo - h_ref)
+    assert np.all(err <= bound), f"h pair: worst excess {np.max(err - bound):.3e} (RMS {rms:.3e})"
 
 
 def routed(L):
@@ -116,7 +122,7 @@ def test_swiglu_prefill_full_size_sampled(cfg):
 
 
 @pytest.mark.parametrize("E,d,f,counts", [
-    (1, 256, 128, [64]),                         # one m-tile, partially filled
+    (1, 256, 256, [64]),                         # one m-tile, partially filled
     (4, 256, 256, [300, 0, 129, 700]),           # ragged segments, an empty expert, tails of 44/1/60 rows
     (2, 2048, 3072, [200, 57]),                  # full model dims: 32 / 48 k-blocks through the ring
     (16, 512, 384, [0] * 15 + [1500]),           # everything on the last expert
