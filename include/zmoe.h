@@ -150,6 +150,27 @@ ZMOE_API zmoe_status zmoe_permute(const int32_t* expert_idx, const void* x, zmoe
                          int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* x_perm,
                          void* workspace, size_t ws_bytes, zmoe_stream_t stream);
 
+/*
+ * zmoe_permute without any device allocation, for callers that cannot allocate: code
+ * whose device memory is wholly owned by a host framework's pool allocator (a cudaMalloc
+ * behind its back can fail for lack of memory, or stall the device while it waits),
+ * code that must not synchronise the device on its hot path, and code recording into a
+ * CUDA graph in a capture mode that forbids allocation.  The ZONOS2 pages have no
+ * counterpart: this is an interface convenience, not a step of the method.
+ *   Same arguments, outputs and results as zmoe_permute, without workspace/ws_bytes.
+ *   Its scratch (per-tile expert counts, 64 KB) is a static device array inside the
+ *   library, held by every GPU that loads it until the process exits.  Limit: T * k <=
+ *   65536; larger problems return ZMOE_ERR_INVALID_ARG with a message naming the limit.
+ *   The first call on a device looks up that array's device address (once per device,
+ *   with the device current) and caches it; make that first call before capturing a
+ *   stream into a CUDA graph.  All calls share the array: calls that overlap on the GPU
+ *   (different streams without ordering between them) race and give wrong results.  It
+ *   calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+ZMOE_API zmoe_status zmoe_permute_noalloc(const int32_t* expert_idx, const void* x, zmoe_dtype dtype, int T, int d,
+                                          int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
+                                          int32_t* inv_perm, void* x_perm, zmoe_stream_t stream);
+
 /* Bytes of workspace zmoe_grouped_swiglu needs for these sizes. */
 ZMOE_API size_t zmoe_grouped_swiglu_workspace_size(int M_total, int E, int d, int f, zmoe_dtype dtype);
 

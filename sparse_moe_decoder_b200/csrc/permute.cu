@@ -15,6 +15,9 @@
 // Small problems (T*k <= 1024) run as ONE CTA that does counting, prefix sums, positions and
 // the row copy.  Larger ones run count -> scan -> scatter over 256-assignment tiles, then a
 // grid-wide 16-byte row gather.
+#include <mutex>
+#include <string>
+
 #include "common.cuh"
 
 namespace zmoe {
@@ -243,3 +246,89 @@ zmoe_status zmoe_permute(const int32_t* expert_idx, const void* x, zmoe_dtype dt
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// zmoe_permute_noalloc: the same permutation for callers that cannot allocate device memory.
+//
+// The multi-CTA path keeps per-tile expert counts in scratch.  Here that scratch is a
+// file-scope device array, so the call allocates nothing: every GPU that loads this library
+// holds the array (64 KB) until the process exits.  In host code `g_noalloc_tile_counts` is
+// only a host-side stand-in for the symbol, never a device address; its device address is
+// fetched with cudaGetSymbolAddress once per device, with that device current, on the first
+// call made on that device, and cached.  Every call shares the array and it keeps the last
+// call's contents: the count pass writes every entry the later passes read, so nothing needs
+// clearing, but two calls that overlap on the GPU (different streams, no ordering) race on it.
+// ---------------------------------------------------------------------------------------------
+namespace zmoe {
+namespace {
+
+constexpr int kNoAllocMaxTiles = 256;   // 256 tiles x 256 assignments = 65536 assignments
+static __device__ __align__(256) int32_t g_noalloc_tile_counts[kNoAllocMaxTiles * kMaxE];
+
+std::mutex g_noalloc_mutex;
+int32_t* g_noalloc_addr[64] = {};
+
+// Device address of the static scratch on the current device (set up once per device).
+zmoe_status noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(ZMOE_ERR_CUDA, std::string("zmoe_permute_noalloc: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(ZMOE_ERR_UNSUPPORTED, "zmoe_permute_noalloc: device index >= 64");
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    int32_t* ptr = nullptr;
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_noalloc_tile_counts);
+    if (e != cudaSuccess || ptr == nullptr)
+      return fail(ZMOE_ERR_CUDA, std::string("zmoe_permute_noalloc: cudaGetSymbolAddress failed: ") +
+                                     cudaGetErrorString(e));
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return ZMOE_OK;
+}
+
+}  // namespace
+}  // namespace zmoe
+
+extern "C" zmoe_status zmoe_permute_noalloc(const int32_t* expert_idx, const void* x, zmoe_dtype dtype, int T, int d,
+                                            int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
+                                            int32_t* inv_perm, void* x_perm, zmoe_stream_t stream) {
+  using namespace zmoe;
+  ZMOE_REQUIRE(dtype_ok(dtype), "zmoe_permute_noalloc: bad dtype");
+  ZMOE_REQUIRE(T >= 0, "zmoe_permute_noalloc: T must be >= 0");
+  ZMOE_REQUIRE(E >= 1 && E <= kMaxE, "zmoe_permute_noalloc: E must be in [1, 64]");
+  ZMOE_REQUIRE(k == 1 || k == 2, "zmoe_permute_noalloc: k must be 1 or 2");
+  ZMOE_REQUIRE(d >= 8 && d % 8 == 0, "zmoe_permute_noalloc: d must be a positive multiple of 8");
+  ZMOE_REQUIRE(counts && offsets, "zmoe_permute_noalloc: counts/offsets NULL");
+  const long long n = static_cast<long long>(T) * k;
+  ZMOE_REQUIRE(n <= static_cast<long long>(kNoAllocMaxTiles) * kTile,
+               "zmoe_permute_noalloc: T * k exceeds the 65536 assignments its static scratch holds; "
+               "use zmoe_permute with a caller-provided workspace");
+  if (n > 0) {
+    ZMOE_REQUIRE(expert_idx && x && perm && inv_perm && x_perm, "zmoe_permute_noalloc: NULL pointer");
+    ZMOE_REQUIRE(aligned16(x) && aligned16(x_perm), "zmoe_permute_noalloc: x/x_perm not 16-byte aligned");
+  }
+  const int vecs = static_cast<int>(d * dtype_size(dtype) / 16);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int* err = device_error_counter();
+  clear_error();
+  if (n <= kSmallMax) {
+    permute_small_kernel<<<1, 1024, 0, s>>>(expert_idx, static_cast<const uint4*>(x), static_cast<int>(n), k, E, vecs,
+                                            counts, offsets, perm, inv_perm, static_cast<uint4*>(x_perm), err);
+    return check_launch("zmoe_permute_noalloc");
+  }
+  int32_t* tile_cnt = nullptr;
+  zmoe_status st = noalloc_scratch(&tile_cnt);
+  if (st != ZMOE_OK) return st;
+  const int tiles = tiles_for(n);
+  permute_count_kernel<<<tiles, kTile, 0, s>>>(expert_idx, static_cast<int>(n), E, tile_cnt, err);
+  permute_scan_kernel<<<1, 128, 0, s>>>(tile_cnt, tiles, E, counts, offsets);
+  permute_scatter_kernel<<<tiles, kTile, 0, s>>>(expert_idx, static_cast<int>(n), k, E, tile_cnt, perm, inv_perm);
+  const long long total_vecs = n * vecs;
+  long long grid = (total_vecs + 255) / 256;
+  const long long cap = static_cast<long long>(num_sms()) * 8;
+  if (grid > cap) grid = cap;
+  gather_rows_kernel<<<static_cast<int>(grid), 256, 0, s>>>(static_cast<const uint4*>(x), perm, offsets, E, vecs,
+                                                            static_cast<uint4*>(x_perm));
+  return check_launch("zmoe_permute_noalloc");
+}

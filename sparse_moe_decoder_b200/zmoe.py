@@ -39,6 +39,7 @@ SIGNATURES = {
     "zmoe_route": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P]),
     "zmoe_permute_workspace_size": (_S, [_I, _I, _I]),
     "zmoe_permute": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "zmoe_permute_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "zmoe_grouped_swiglu_workspace_size": (_S, [_I, _I, _I, _I, _I]),
     "zmoe_grouped_swiglu": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _S, _P]),
     "zmoe_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
