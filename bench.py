@@ -42,7 +42,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4])
+    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle timing leg")
@@ -68,6 +68,8 @@ WORKLOADS = {
        "bf16 weights/activations, fp32 accumulate",
     3: "prefill MoE layer: T=16384 (8 x 2048), d_model=2048, d_ff=3072, E=16, top-1, b~N(0,0.5), bf16",
     4: "final MoE layer: T=16384, d_model=2048, d_ff=3072, E=16, top-2, Zipf(1.2) logit skew, bf16",
+    5: "batch-1 decode stack: 9-codebook embedding sum + RMSNorm, 24 pre-norm MoE layers (d_model=2048, "
+       "d_ff=3072, E=16, top-1, top-2 in the last), attention omitted, bf16, one token per step",
 }
 
 
@@ -178,6 +180,8 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
+    if args.config == 5:
+        return run_reference_stack(args)
     from moe_inputs import make_config
     L = make_config(args.config)
 
@@ -239,10 +243,193 @@ def traffic_from_profiles(kernel_key: str):
         return None
 
 
+def run_reference_stack(args):
+    """The oracle stack (numpy float64) on a bounded number of tokens: experts are drawn on first use
+    and kept, so later tokens time the arithmetic, not the drawing."""
+    import oracle
+    from moe_inputs import StackSpec
+    spec = StackSpec()
+    cache = {}
+
+    def expert(l, e):
+        if (l, e) not in cache:
+            cache[(l, e)] = spec.expert(l, e)
+        return cache[(l, e)]
+
+    layers = []
+    for l in range(spec.n_layers):
+        wr, sb, gm = spec.layer_small(l)
+        layers.append(dict(w_router=wr, sel_bias=sb, gamma=gm, k=spec.k_of(l), experts=(lambda e, l=l: expert(l, e))))
+    tables, g0 = spec.tables(), spec.gamma0()
+    n = max(1, min(args.steps, 3))
+    codes = spec.codes(n + 1)
+    oracle.decode_stack_step(codes[n:n + 1], tables, g0, layers, spec.eps)      # warm-up: draws experts
+    t0 = time.perf_counter()
+    for i in range(n):
+        oracle.decode_stack_step(codes[i:i + 1], tables, g0, layers, spec.eps)
+    el = time.perf_counter() - t0
+    v = n / el
+    sample = (f"oracle.decode_stack_step (numpy float64), {n} token(s) through the 24-layer stack "
+              f"(experts drawn on first use, outside the timing where already drawn), {el:.1f} s")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": n, "warmup": 1, "ms_per_step": 1e3 * el / n, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOADS[5], "us_per_token": 1e6 * el / n, "batch": 1},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_stack(args):
+    """Configuration 5: tokens/s (= 1 / s per token) of the 24-layer batch-1 stack."""
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=torch.device("cuda", local_rank))
+    from moe_inputs import StackSpec, bf16_bits, stack_expert_bits
+    from sparse_moe_decoder_b200 import zmoe_get_device_errors
+    from sparse_moe_decoder_b200.layer import stack_from_bits
+
+    spec = StackSpec()
+    st = stack_from_bits(bf16_bits(spec.tables()), spec.gamma0(), spec.layer_small, stack_expert_bits(spec),
+                         spec.n_layers, spec.E, spec.d, spec.f, spec.k_of, spec.eps, T=1)
+    n = args.warmup + args.steps
+    codes = spec.codes(n + 1)
+    if rank > 0:
+        codes = np.random.default_rng(1000 + rank).integers(0, 1024, size=codes.shape).astype(np.int32)
+    codes_dev = torch.from_numpy(codes).cuda()
+    stream = torch.cuda.current_stream()
+
+    # touched experts of one step (the roofline's bytes)
+    st.record_inputs = True
+    st.step(codes_dev[n:n + 1])
+    torch.cuda.synchronize()
+    touched = sum(int(torch.unique(t).numel()) for t in st.layer_idx)
+    st.record_inputs = False
+    per_expert = 3 * spec.f * spec.d * 2
+    alg_bytes = touched * per_expert + spec.n_layers * spec.E * spec.d * 2 + spec.n_codebooks * spec.d * 2
+
+    graph = None
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for _ in range(2):
+                st.step()
+        stream.wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            st.step()
+        torch.cuda.synchronize()
+    except Exception as exc:   # capture not possible here: run the same calls eagerly
+        graph = None
+        print(f"# CUDA graph capture unavailable ({type(exc).__name__}: {exc}); timing eager launches",
+              file=sys.stderr)
+        torch.cuda.synchronize()
+
+    def step(i):
+        st.ids.copy_(codes_dev[i:i + 1])
+        if graph is not None:
+            graph.replay()
+        else:
+            st.step()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t[0])
+    ms_per_step = elapsed_ms / args.steps
+    value = world * args.steps / (elapsed_ms / 1e3)
+
+    # e2e: codes from pinned host memory each step, the final residual stream read back
+    codes_host = torch.from_numpy(codes).pin_memory()
+    h_host = torch.empty((1, spec.d), dtype=torch.float32).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        st.ids.copy_(codes_host[i:i + 1], non_blocking=True)
+        if graph is not None:
+            graph.replay()
+        else:
+            st.step()
+        h_host.copy_(st.h, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    dev_errors = zmoe_get_device_errors()
+    peaks = load_peaks()
+    achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        t0 = time.perf_counter()
+        layers = []
+        for l in range(spec.n_layers):
+            wr, sb, gm = spec.layer_small(l)
+            layers.append(dict(w_router=wr, sel_bias=sb, gamma=gm, k=spec.k_of(l),
+                               experts=(lambda e, l=l: spec.expert(l, e))))
+        oracle.decode_stack_step(codes[:1], spec.tables(), spec.gamma0(), layers, spec.eps)
+        el = time.perf_counter() - t0
+        cpu = {"value": 1.0 / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"oracle.decode_stack_step (numpy float64) on one token through all 24 layers, "
+                         f"drawing each touched expert's weights as it goes, {el:.1f} s"}
+    used_graph = graph is not None
+    graph = None          # release the graph before the process group goes away
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOADS[5], "us_per_token": ms_per_step * 1e3, "layers": spec.n_layers,
+                       "d_model": spec.d, "d_ff": spec.f, "E": spec.E, "batch": 1,
+                       "parallelism": f"dp{world} (replicated weights, no data-path collective)",
+                       "l2": "inputs larger than L2 (14.5 GB of weights; ~0.9 GB read per token)",
+                       "experts_touched_per_token": touched, "cuda_graph": used_graph},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "kernel": "whole decode step (embed + 24 x (rmsnorm, route, permute, swiglu, combine))",
+                         "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peaks["source"]},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": spec.n_codebooks * 4, "d2h_bytes_per_step": spec.d * 4},
+            "gpu_launches": (1 + spec.n_layers * 5) * args.steps,
+            "clocks": clk.summary(),
+            "device_errors": dev_errors,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.config == 5:
+        return run_stack(args)
 
     import torch
     import torch.distributed as dist

@@ -244,3 +244,29 @@ class StackSpec:
         """One fresh frame of (already delay-sheared) ids per decode step: int32 [steps, N]."""
         return self._rng(3, 0).integers(0, CODEBOOK_SIZE, size=(steps, self.n_codebooks),
                                         dtype=np.int64).astype(np.int32)
+
+
+# --------------------------------------------------------------------------------------------
+# Bulk generation of the stack's expert weights (bf16 bit patterns), in parallel worker processes.
+# --------------------------------------------------------------------------------------------
+
+def _expert_bits_job(args):
+    seed, layer, e, d, f = args
+    spec = StackSpec(seed=seed, d=d, f=f)
+    return layer, e, tuple(bf16_bits(w) for w in spec.expert(layer, e))
+
+
+def stack_expert_bits(spec: StackSpec, workers: Optional[int] = None):
+    """Yields (layer, expert, (W_gate, W_up, W_down) as uint16 bf16 bit arrays) for every expert of
+    the stack, drawn in worker processes (spawned, so it is safe after CUDA has been initialised)."""
+    import multiprocessing as mp
+    import os as _os
+    jobs = [(spec.seed, l, e, spec.d, spec.f) for l in range(spec.n_layers) for e in range(spec.E)]
+    n = workers or max(1, min(16, (_os.cpu_count() or 2) - 1))
+    if n == 1:
+        for j in jobs:
+            yield _expert_bits_job(j)
+        return
+    with mp.get_context("spawn").Pool(n) as pool:
+        for out in pool.imap(_expert_bits_job, jobs, chunksize=2):
+            yield out

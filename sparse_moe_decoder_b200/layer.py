@@ -132,3 +132,32 @@ class DecodeStack:
             if self.record_inputs:
                 self.layer_idx.append(R.idx.clone())
         return self.h
+
+
+def stack_from_bits(tables_bits, gamma0, layer_small, expert_bits, n_layers: int, E: int, d: int, f: int,
+                    k_of, eps: float = 1e-6, T: int = 1, device="cuda") -> DecodeStack:
+    """Builds a DecodeStack on the device from host arrays.
+
+    tables_bits: uint16 [N, V, d] bf16 bit patterns; gamma0: f32 [d]; layer_small(l) -> (W_r f32 [E, d]
+    bf16-exact, sel_bias f32 [E], gamma f32 [d]); expert_bits: iterable of (l, e, (wg, wu, wd) uint16
+    bit arrays); k_of(l) -> experts per token in layer l.
+    """
+    import numpy as np
+
+    def bits_to_dev(b):
+        return torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(device).view(torch.bfloat16)
+
+    layers = []
+    for l in range(n_layers):
+        wr, sb, gm = layer_small(l)
+        layers.append(MoEWeights(torch.from_numpy(wr).to(device=device, dtype=torch.bfloat16),
+                                 torch.empty((E, f, d), dtype=torch.bfloat16, device=device),
+                                 torch.empty((E, f, d), dtype=torch.bfloat16, device=device),
+                                 torch.empty((E, d, f), dtype=torch.bfloat16, device=device),
+                                 torch.from_numpy(sb).to(device), None, torch.from_numpy(gm).to(device), k_of(l)))
+    for l, e, (wg, wu, wd) in expert_bits:
+        layers[l].w_gate[e].copy_(bits_to_dev(wg))
+        layers[l].w_up[e].copy_(bits_to_dev(wu))
+        layers[l].w_down[e].copy_(bits_to_dev(wd))
+    tables = bits_to_dev(tables_bits)
+    return DecodeStack(tables, torch.from_numpy(gamma0).to(device), layers, eps, T)
