@@ -551,7 +551,7 @@ def main(argv=None):
         achieved = alg_bytes / (ffn_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_from_profiles("grouped_swiglu_cfg2"),
-                "kernel": "zmoe_grouped_swiglu (stream_ffn gate/up + down launches)",
+                "kernel": "zmoe_grouped_swiglu (dec_tc_kernel: gate/up and down in one launch)",
                 "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peaks["source"]}
     else:
         achieved = flops / (ffn_ms / 1e3) / 1e12

@@ -6,8 +6,8 @@
 //
 // Dispatch:
 //   f32  -> plain fp32 FMA kernels (no TF32 anywhere: one thread per output, float4 loads).
-//   bf16 -> rows per expert small (decode): one persistent weight-streaming launch
-//           (swiglu_decode.cu);
+//   bf16 -> rows per expert small (decode): one persistent stream-K launch on the tensor cores
+//           with weights as the MMA's M and tokens as its N (swiglu_dec_tc.cu);
 //           rows per expert large (prefill): tcgen05 / TMEM / TMA grouped GEMMs (swiglu_tc.cu).
 //           Both keep h as a bf16 pair h_hi + h_lo ([M, 2f]) so that the second contraction
 //           sees h to ~16 significant bits with bf16 tensor-core operands.
@@ -15,11 +15,11 @@
 
 namespace zmoe {
 
-zmoe_status grouped_swiglu_decode(const uint16_t* x_perm, const int32_t* offsets, int M_total, const uint16_t* w_gate,
+zmoe_status grouped_swiglu_dec_tc(const uint16_t* x_perm, const int32_t* offsets, int M_total, const uint16_t* w_gate,
                                   const uint16_t* w_up, const uint16_t* w_down, int E, int d, int f, uint16_t* h,
                                   float* y_perm, void* ws, cudaStream_t s);
-size_t grouped_swiglu_decode_workspace(int E);
-bool grouped_swiglu_decode_supported(int d, int f);
+size_t grouped_swiglu_dec_tc_workspace(int M_total, int E, int d, int f);
+bool grouped_swiglu_dec_tc_supported(int d, int f);
 zmoe_status grouped_swiglu_tc(const uint16_t* x_perm, const int32_t* offsets, int M_total, const uint16_t* w_gate,
                               const uint16_t* w_up, const uint16_t* w_down, int E, int d, int f, uint16_t* h,
                               float* y_perm, void* ws, size_t ws_bytes, cudaStream_t s);
@@ -94,7 +94,7 @@ size_t zmoe_grouped_swiglu_workspace_size(int M_total, int E, int d, int f, zmoe
   if (M_total < 0 || E < 1 || d < 1 || f < 1) return 0;
   if (dtype == ZMOE_BF16) {
     const size_t a = zmoe::grouped_swiglu_tc_workspace(M_total, E, d, f);
-    const size_t b = zmoe::grouped_swiglu_decode_workspace(E);
+    const size_t b = zmoe::grouped_swiglu_dec_tc_workspace(M_total, E, d, f);
     return a > b ? a : b;
   }
   return 0;
@@ -137,7 +137,7 @@ zmoe_status zmoe_grouped_swiglu(const void* x_perm, const int32_t* offsets, int 
   const auto* wd = static_cast<const uint16_t*>(w_down);
   auto* hh = static_cast<uint16_t*>(h);
   const bool tc_ok = grouped_swiglu_tc_supported(d, f);
-  const bool dec_ok = grouped_swiglu_decode_supported(d, f);
+  const bool dec_ok = grouped_swiglu_dec_tc_supported(d, f);
   if (tc_ok && (M_total >= kTcMinRowsPerExpert * E || !dec_ok)) {
     if (ws_bytes < grouped_swiglu_tc_workspace(M_total, E, d, f))
       return fail(ZMOE_ERR_WORKSPACE_TOO_SMALL,
@@ -145,10 +145,10 @@ zmoe_status zmoe_grouped_swiglu(const void* x_perm, const int32_t* offsets, int 
     return grouped_swiglu_tc(xp, offsets, M_total, wg, wu, wd, E, d, f, hh, y_perm, workspace, ws_bytes, s);
   }
   if (!dec_ok) return fail(ZMOE_ERR_UNSUPPORTED, "zmoe_grouped_swiglu: no bf16 kernel for this d, f");
-  if (!workspace || ws_bytes < grouped_swiglu_decode_workspace(E))
+  if (!workspace || ws_bytes < grouped_swiglu_dec_tc_workspace(M_total, E, d, f))
     return fail(ZMOE_ERR_WORKSPACE_TOO_SMALL,
                 "zmoe_grouped_swiglu: workspace smaller than zmoe_grouped_swiglu_workspace_size()");
-  return grouped_swiglu_decode(xp, offsets, M_total, wg, wu, wd, E, d, f, hh, y_perm, workspace, s);
+  return grouped_swiglu_dec_tc(xp, offsets, M_total, wg, wu, wd, E, d, f, hh, y_perm, workspace, s);
 }
 
 }  // extern "C"

@@ -394,6 +394,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // The producer and MMA roles run on lane 0 alone: the other lanes wait here for it, so that every
+  // warp meets the CTA barrier (and warp 1 the TMEM release) converged.
+  __syncwarp();
   __syncthreads();
   if (warp == 0 && lane == 0 && *abort_flag) {
     // After an abort, loads the MMA warp never consumed may still be landing in the ring.  The
