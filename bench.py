@@ -408,12 +408,13 @@ def run_stack(args):
                        "experts_touched_per_token": touched, "cuda_graph": used_graph},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                         "kernel": "whole decode step (embed + 24 x (rmsnorm, route, permute, swiglu, combine))",
+                         "kernel": "whole decode step (embed + 24 x moe_layer_kernel: pre-norm, router, dispatch, "
+                                   "SwiGLU and combine in one launch per layer)",
                          "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peaks["source"]},
             "cpu_baseline": cpu,
             "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": spec.n_codebooks * 4, "d2h_bytes_per_step": spec.d * 4},
-            "gpu_launches": (1 + spec.n_layers * 5) * args.steps,
+            "gpu_launches": (1 + spec.n_layers) * args.steps,
             "clocks": clk.summary(),
             "device_errors": dev_errors,
         }
@@ -465,10 +466,13 @@ def main(argv=None):
     def step(i):
         return R.run(x, Ws[i % n_copies])
 
+    # decode sizes: the whole layer is one zmoe_moe_layer call (one cooperative launch); prefill sizes
+    # time the four entry points separately, with events around the grouped SwiGLU
+    fused = L.T * L.k < 64 * L.E
     for i in range(args.warmup):
-        step(i)
+        step(i) if fused else R.run_steps(x, Ws[i % n_copies])
     torch.cuda.synchronize()
-    counts = R.perm_outs["counts"].cpu().numpy()
+    counts = np.bincount(R.idx.cpu().numpy().ravel(), minlength=L.E)
     experts_touched = int((counts > 0).sum())
 
     # timed region: K steps, per-step events around the grouped-SwiGLU call (dominant kernels)
@@ -482,6 +486,11 @@ def main(argv=None):
         ev0.record(stream)
         for i in range(args.steps):
             W = Ws[i % n_copies]
+            if fused:
+                ev_ffn[i][0].record(stream)
+                R.run(x, W)
+                ev_ffn[i][1].record(stream)
+                continue
             Z.zmoe_route(x, W.w_router, W.k, W.logit_bias, W.sel_bias, outs=(R.idx, R.gates, R.margin))
             Z.zmoe_permute(R.idx, x, W.E, outs=R.perm_outs, workspace=R.perm_ws)
             ev_ffn[i][0].record(stream)
@@ -505,7 +514,7 @@ def main(argv=None):
 
     # launches of libzmoe kernels per step
     n_assign = L.T * L.k
-    launches_per_step = 1 + (1 if n_assign <= 1024 else 4) + 2 + 1
+    launches_per_step = 1 if fused else 1 + (1 if n_assign <= 1024 else 4) + 2 + 1
 
     # e2e: the same steps through the public API from pinned host memory, result read back
     x_host = torch.from_numpy(L.x).to(dt).pin_memory()
@@ -540,18 +549,22 @@ def main(argv=None):
     # roofline of the dominant kernels (the grouped-SwiGLU launches: gate/up then down)
     peaks = load_peaks()
     bpe = 2
-    counts_all = R.perm_outs["counts"].cpu().numpy()
+    counts_all = counts
     touched = int((counts_all > 0).sum())
     M = int(counts_all.sum())
     weight_bytes = touched * 3 * L.f * L.d * bpe
     act_bytes = M * L.d * bpe + 2 * (M * 2 * L.f * bpe) + M * L.d * 4   # x_perm in, h pair out + in, y_perm out
+    if fused:
+        # the launch also reads x and W_r, writes and re-reads x_perm, and writes y
+        act_bytes += L.T * L.d * bpe + L.E * L.d * bpe + M * L.d * bpe + L.T * L.d * 4
     alg_bytes = weight_bytes + act_bytes
     flops = 2.0 * M * 3 * L.d * L.f
     if args.config == 2:
         achieved = alg_bytes / (ffn_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_from_profiles("grouped_swiglu_cfg2"),
-                "kernel": "zmoe_grouped_swiglu (dec_tc_kernel: gate/up and down in one launch)",
+                "kernel": ("moe_layer_kernel: router, dispatch, SwiGLU and combine in one launch" if fused else
+                           "zmoe_grouped_swiglu (dec_tc_kernel)"),
                 "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peaks["source"]}
     else:
         achieved = flops / (ffn_ms / 1e3) / 1e12

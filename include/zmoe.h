@@ -209,6 +209,38 @@ ZMOE_API zmoe_status zmoe_grouped_swiglu(const void* x_perm, const int32_t* offs
 ZMOE_API zmoe_status zmoe_combine(const float* y_perm, const int32_t* inv_perm, const float* gates, const float* residual,
                          int T, int d, int k, float* y, zmoe_stream_t stream);
 
+/* Bytes of workspace zmoe_moe_layer needs for these sizes (0 for T == 0 or bad arguments). */
+ZMOE_API size_t zmoe_moe_layer_workspace_size(int T, int d, int f, int E, int k, zmoe_dtype dtype);
+
+/*
+ * One sparse MoE layer, optionally with its pre-norm ([DIGEST] items 5-6: RMSNorm, sparse
+ * MoE FFN with top-1 routing and top-2 in the last layer; [ROUTING] section 2.1: router,
+ * gate-weighted sum of the chosen experts' SwiGLU outputs):
+ *   gamma != NULL:  x = RMSNorm(h) * gamma = h / sqrt(mean_c h^2 + eps) * gamma, rounded to
+ *                   `dtype` (the decode stack's pre-norm residual block); `x` is not read.
+ *   gamma == NULL:  x is the layer input.
+ *   y[t] = h[t] + sum_{i < k} gates[t, i] * FFN_{expert_idx[t, i]}(x[t])   (h == NULL: no residual)
+ * with the router, dispatch, SwiGLU and combine of zmoe_route, zmoe_permute,
+ * zmoe_grouped_swiglu and zmoe_combine (same conventions, same results up to fp32 summation
+ * order).  Decode sizes (bf16, T * k < 64 E, T * k <= 1024, d and f multiples of 256) run as
+ * one cooperative launch; other sizes run those entry points in order.
+ *   x: [T, d] of `dtype` (or NULL with gamma); h: f32 [T, d] or NULL (required with gamma);
+ *   gamma: f32 [d] or NULL; w_router [E, d], w_gate, w_up [E, f, d], w_down [E, d, f] of
+ *   `dtype`; logit_bias, sel_bias: f32 [E] or NULL.
+ *   Outputs: y: f32 [T, d] (may alias h); expert_idx int32 [T, k], gates f32 [T, k],
+ *   margin f32 [T] (as zmoe_route) and x_norm [T, d] of `dtype` (the routed input, with
+ *   gamma only) are optional (NULL: kept in the workspace).
+ *   workspace: zmoe_moe_layer_workspace_size() bytes, 256-byte aligned; it also holds the
+ *   intermediates (x_perm, the hidden activations, y_perm).  1 <= E <= 64, k in {1, 2},
+ *   k <= E, d % 8 == 0, f % 8 == 0 (bf16: multiples of 256); 16-byte aligned pointers.
+ */
+ZMOE_API zmoe_status zmoe_moe_layer(const void* x, const float* h, const float* gamma, float eps,
+                                    const void* w_router, const float* logit_bias, const float* sel_bias,
+                                    const void* w_gate, const void* w_up, const void* w_down, zmoe_dtype dtype,
+                                    int T, int d, int f, int E, int k, float* y, int32_t* expert_idx,
+                                    float* gates, float* margin, void* x_norm, void* workspace, size_t ws_bytes,
+                                    zmoe_stream_t stream);
+
 /*
  * Reads and clears the device error counters of the current device.  Synchronises
  * `stream` (and the device) first.  *count = data errors (ids or indices out of range)

@@ -1,0 +1,1199 @@
+// Decode-size MoE on the tensor cores: the grouped SwiGLU as one swap-AB stream-K launch, and the
+// whole MoE layer (pre-norm, router, dispatch, SwiGLU, combine) as one cooperative launch.
+//
+// Per expert e over its rows of the permuted activations ("GLU Variants Improve Transformer",
+// ZONOS2 Technical Report "Builds on"; SiLU per the telknet.cc article on ZONOS2, section 2.1):
+//   phase A (gate/up): h = silu(x W_gate[e]^T) * (x W_up[e]^T), stored as the bf16 pair
+//                      h_hi = bf16(h), h_lo = bf16(h - h_hi)
+//   phase B (down):    y_perm = h_hi W_down[e]^T + h_lo W_down[e]^T          (fp32)
+//
+// With a few rows per expert the work is streaming the touched experts' weights from HBM once.
+// Design of the SwiGLU part:
+//   * Swap-AB on tcgen05: 128 weight rows are the MMA's M, a block of up to 16 token rows is its N
+//     (kind::f16, bf16 in, fp32 accumulate in TMEM).  A unit is (expert, 128-row weight block, token
+//     block); its k-range is cut into 256-wide stages (a 64 KB weight box + an 8/16 KB token box).
+//   * Stream-K: every CTA (one per SM, cooperative launch: all resident) takes an equal,
+//     contiguous range of the stage list of each phase, so bytes per SM balance to within one
+//     stage whatever the expert loads are (down to a single expert at batch 1).  A unit wholly
+//     inside a CTA's range is finished in TMEM; a unit cut by a range edge leaves fp32 partial
+//     sums in a per-CTA slot and the last CTA to arrive adds the partials in CTA order
+//     (deterministic) and finishes it.  Each CTA runs its (at most two) cut units first, so the
+//     cross-CTA hand-offs overlap the whole units that follow.
+//   * Roles: warp 0 loads weight boxes and warp 6 token boxes (x, or the h pair) with TMA into a
+//     2-stage ring (160 KB; a 64 KB box is the size at which one SM's TMA reaches full HBM rate),
+//     each completing on its own mbarrier, so weight loads never wait for h; warp 1 allocates TMEM
+//     and issues the MMAs from one thread (tcgen05.commit frees a stage when its MMAs are done);
+//     warps 2..5 read the accumulators with tcgen05.ld and run the epilogues.
+//   * Phase-A units of expert e release-increment ready[e]; the token producer acquires ready[e]
+//     before loading h rows of expert e (cross-proxy fence before the TMA).
+//   * Every wait is bounded (time limit): on expiry the CTA counts a device timeout, aborts,
+//     drains its own copies and MMAs, frees its TMEM and returns.
+//
+// The fused layer adds, before the SwiGLU, in the same launch:
+//   0a  per token (CTA c takes tokens c, c + C, ...): optional RMSNorm of the fp32 residual stream
+//       ("Root Mean Square Layer Normalization", ZONOS2 Technical Report "Builds on"), the router
+//       logits, top-k selection on logits + selection bias and the softmax gates (ZONOS2 digest,
+//       items 5-6; "Auxiliary-Loss-Free Load Balancing" for the selection-only bias);
+//   0b  after a grid barrier, every CTA recomputes the dispatch permutation from all T * k choices
+//       (a few hundred integers: cheaper than another barrier) and gathers its share of x_perm;
+//   and, after a second barrier, fuses the gate-weighted combine into the down projection's
+//   epilogue: y[t] = residual[t] + sum_i gate[t, i] * y_perm[row(t, i)], formed in slot order (for
+//   k = 2 by the later of the token's two units, from both rows, so the sum is deterministic).
+#include "sm100_ptx.cuh"
+
+namespace zmoe {
+
+unsigned int* device_timeout_counter();
+
+namespace {
+
+using namespace ptx;
+
+constexpr int BM = 128;                       // weight rows per unit (MMA M)
+constexpr int NT = 16;                        // token rows per block (MMA N)
+constexpr int KS = 256;                       // k per stage
+constexpr int CH = KS / 64;                   // 64-wide chunks per stage
+constexpr int STAGES = 2;
+constexpr int W_BYTES = BM * KS * 2;          // 64 KB
+constexpr int X_BYTES = NT * KS * 2;          // 8 KB  x slice
+constexpr int HP_BYTES = NT * KS * 2 * 2;     // 16 KB h_hi + h_lo slice
+constexpr int STAGE_BYTES = W_BYTES + HP_BYTES;
+constexpr int kThreads = 224;                 // 7 warps
+constexpr int kWarps = kThreads / 32;
+constexpr int kWarpTok = 6;
+constexpr uint32_t TMEM_COLS = 64;            // 2 accumulator buffers x (gate 16 | up 16)
+constexpr int kMaxE = 64;
+constexpr int kMaxCtas = 256;
+constexpr int kMaxAssign = 1024;              // T * k of the fused layer
+constexpr unsigned long long kTimeoutNs = 2000000000ull;
+constexpr uint32_t kIdesc = idesc_bf16_f32(BM, NT);
+// fused layer, phase 0 scratch in the (then idle) ring: ids, ranks, the routed row (f32), the raw
+// token row, gamma, and the router matrix when it fits
+constexpr int kRingBytes = STAGES * STAGE_BYTES;
+constexpr int kScratch0 = 2 * kMaxAssign * 4;
+
+struct DecArgs {
+  const int32_t* offsets;   // [E + 1] (grouped-SwiGLU entry; the fused layer forms its own)
+  uint16_t* h;              // [M, 2f] h_hi | h_lo
+  float* y;                 // [M, d]  y_perm
+  unsigned int* ready;      // [E]    finished phase-A units per expert
+  unsigned int* cnt_a;      // [ua]   arrivals per cut phase-A unit
+  unsigned int* cnt_b;      // [ub]
+  float* part_a;            // [C][2 slots][2 mats][NT][BM] partial sums of cut phase-A units
+  float* part_b;            // [C][2 slots][NT][BM]
+  unsigned int* timeouts;
+  unsigned int* errors;
+  int E, d, f, M_total;
+  int ua_cap, ub_cap;       // units the counter arrays hold
+  // combine fused into the phase-B epilogue (fused layer only)
+  int fuse, k;
+  const float* gates;       // [T, k]
+  const float* residual;    // [T, d] or null
+  float* out;               // [T, d] (may alias residual)
+  unsigned int* comb_cnt;   // [T, d / BM] units of each token's row block done (k = 2)
+};
+
+struct LayerArgs {
+  const uint16_t* x_in;     // [T, d] layer input (without gamma)
+  const float* h_in;        // [T, d] fp32 residual stream, input of the pre-norm (with gamma)
+  const float* gamma;       // [d] or null
+  float eps;
+  const uint16_t* w_r;      // [E, d]
+  const float* logit_bias;  // [E] or null
+  const float* sel_bias;    // [E] or null
+  int T;
+  uint16_t* x_norm;         // [T, d] the layer input as routed (written when gamma is given)
+  int32_t* expert_idx;      // [T, k]
+  float* gates;             // [T, k]
+  float* margin;            // [T] or null
+  int32_t* counts;          // [E]
+  int32_t* offsets;         // [E + 1]
+  int32_t* perm;            // [T * k]
+  int32_t* inv_perm;        // [T, k]
+  uint16_t* x_perm;         // [T * k, d]
+  unsigned int* gbar;       // grid barrier arrivals
+};
+
+struct __align__(16) Ctrl {
+  uint64_t full_w[STAGES];
+  uint64_t full_t[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint64_t rbar[2];          // fused layer: router matrix (+ gamma), token row
+  uint32_t tmem_base;
+  int abort;
+  int bad;
+  int last_flag;
+  int last_tok[NT];
+  int off[kMaxE + 1];
+  int ustart[2][kMaxE + 1];  // first unit of each expert, per phase
+  int rlo[2][kMaxCtas + 1];  // first stage of each CTA's range, per phase
+  // fused layer
+  int rowsrc[kMaxAssign];    // permuted row -> token
+  int invp[kMaxAssign];      // assignment (t, i) -> permuted row
+  int wcnt[kWarps][kMaxE];
+  int run[kMaxE];
+  float red[kWarps + 1];
+  float wpart[kWarps][16];
+  float logit[kMaxE];
+};
+
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + sizeof(Ctrl);
+
+// ------------------------------------------------------------------------------------------
+// work geometry (every role walks the same sequence)
+// ------------------------------------------------------------------------------------------
+struct Unit {
+  int e, rb, row0, rows;    // expert, weight block, first permuted row, rows in the token block
+};
+
+__device__ __forceinline__ Unit unit_of(const Ctrl& C, int ph, int E, int u) {
+  const int* us = C.ustart[ph];
+  int e = 0;
+  while (e + 1 < E && us[e + 1] <= u) ++e;
+  const int ntb = (C.off[e + 1] - C.off[e] + NT - 1) / NT;
+  const int local = u - us[e];
+  Unit U;
+  U.e = e;
+  U.rb = local / ntb;
+  const int tb = local - U.rb * ntb;
+  U.row0 = C.off[e] + tb * NT;
+  const int left = C.off[e + 1] - U.row0;
+  U.rows = left < NT ? left : NT;
+  return U;
+}
+
+// A CTA's stage range [sb, se) as segments (one unit each): the cut first and last units, then the
+// whole units in order.
+struct Plan {
+  int sb, se, S, uf, ul, pf, pl, w0, n;
+};
+
+struct Seg {
+  int u, j0, j1;
+};
+
+__device__ __forceinline__ Plan make_plan(int sb, int se, int S) {
+  Plan P{sb, se, S, 0, 0, 0, 0, 0, 0};
+  if (se <= sb) return P;
+  P.uf = sb / S;
+  P.ul = (se - 1) / S;
+  if (P.uf == P.ul) {
+    P.n = 1;
+    return P;
+  }
+  P.pf = (sb % S) != 0;
+  P.pl = (se % S) != 0;
+  P.w0 = P.pf ? P.uf + 1 : P.uf;
+  const int w1 = P.pl ? P.ul - 1 : P.ul;
+  P.n = P.pf + P.pl + (w1 - P.w0 + 1);
+  return P;
+}
+
+__device__ __forceinline__ Seg seg_at(const Plan& P, int i) {
+  if (P.uf == P.ul) return Seg{P.uf, P.sb - P.uf * P.S, P.se - P.uf * P.S};
+  if (P.pf) {
+    if (i == 0) return Seg{P.uf, P.sb - P.uf * P.S, P.S};
+    --i;
+  }
+  if (P.pl) {
+    if (i == 0) return Seg{P.ul, 0, P.se - P.ul * P.S};
+    --i;
+  }
+  return Seg{P.w0 + i, 0, P.S};
+}
+
+// The CTA whose range holds stage s (the largest c with rlo[c] <= s; its range is not empty).
+__device__ __forceinline__ int cta_of(const int* rlo, int nC, int s) {
+  int lo = 0, hi = nC - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (rlo[mid] <= s) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void set_abort(Ctrl& C, unsigned int* counter) {
+  if (atomicExch(&C.abort, 1) == 0 && counter) atomicAdd(counter, 1u);
+}
+
+// Named barrier 1 joins the four epilogue warps.
+__device__ __forceinline__ void epi_bar() { bar_sync(1, 128); }
+
+// Waits until the latest armed phase of each slot of `bars` has completed (bounded).
+__device__ __forceinline__ void drain_ring(uint64_t* bars, int armed) {
+  for (int sl = 0; sl < STAGES; ++sl) {
+    const int last = armed - 1 - (((armed - 1 - sl) % STAGES) + STAGES) % STAGES;
+    if (last < 0) continue;
+    const uint64_t t1 = globaltimer();
+    while (!mbar_try_wait(&bars[sl], static_cast<uint32_t>((last / STAGES) & 1)) && globaltimer() - t1 < kTimeoutNs) {
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// shared setup: barriers and TMEM; unit and range tables from C.off
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void init_ctrl(Ctrl& C) {
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&C.full_w[s], 1);
+      mbar_init(&C.full_t[s], 1);
+      mbar_init(&C.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&C.tfull[b], 1);
+      mbar_init(&C.tempty[b], 4);
+    }
+    mbar_init(&C.drain, 1);
+    mbar_init(&C.rbar[0], 1);
+    mbar_init(&C.rbar[1], 1);
+    C.abort = 0;
+    C.bad = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if ((threadIdx.x >> 5) == 1) tmem_alloc(&C.tmem_base, TMEM_COLS);
+}
+
+// Needs C.off; ends with a CTA barrier.  Sets C.bad when the offsets are not a monotone split of
+// [0, M_total) or need more units than the counters hold.
+__device__ __forceinline__ void build_tables(Ctrl& C, const DecArgs& p, const int* S) {
+  const int E = p.E, nC = gridDim.x;
+  if (threadIdx.x == 0) {
+    int bad = C.off[0] != 0 || C.off[E] > p.M_total;
+    int a = 0, b = 0;
+    for (int e = 0; e < E; ++e) {
+      bad |= C.off[e + 1] < C.off[e];
+      const int ntb = bad ? 0 : (C.off[e + 1] - C.off[e] + NT - 1) / NT;
+      C.ustart[0][e] = a;
+      C.ustart[1][e] = b;
+      a += ntb * (p.f / BM);
+      b += ntb * (p.d / BM);
+    }
+    C.ustart[0][E] = a;
+    C.ustart[1][E] = b;
+    bad |= a > p.ua_cap || b > p.ub_cap;
+    if (bad) {
+      C.bad = 1;
+      if (blockIdx.x == 0) record_device_error(p.errors);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i <= nC; i += blockDim.x) {
+    C.rlo[0][i] = static_cast<int>(static_cast<long long>(C.ustart[0][E]) * S[0] * i / nC);
+    C.rlo[1][i] = static_cast<int>(static_cast<long long>(C.ustart[1][E]) * S[1] * i / nC);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+// ------------------------------------------------------------------------------------------
+// the SwiGLU roles (both kernels)
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensorMap* mWu, const CUtensorMap* mWd,
+                                          const CUtensorMap* mX, const CUtensorMap* mH, const DecArgs& p, Ctrl& C,
+                                          unsigned char* base, uint32_t tmem, const int* S) {
+  volatile int* abort_flag = &C.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = p.E;
+  const int nC = gridDim.x, cta = blockIdx.x;
+
+  if (warp == 0 || warp == kWarpTok) {
+    // ============================ producers: weights (warp 0), tokens (warp 6) ============================
+    if (lane == 0) {
+      const bool wt = warp == 0;
+      uint64_t* full = wt ? C.full_w : C.full_t;
+      int q = 0;            // stages armed on `full`
+      bool ok = true;
+      int ready_e = -1;     // last expert whose phase-A units were all seen complete
+      if (!wt) asm volatile("fence.proxy.async.global;" ::: "memory");   // x_perm may come from this launch
+      for (int ph = 0; ph < 2 && ok; ++ph) {
+        const Plan P = make_plan(C.rlo[ph][cta], C.rlo[ph][cta + 1], S[ph]);
+        for (int i = 0; i < P.n && ok; ++i) {
+          const Seg g = seg_at(P, i);
+          const Unit U = unit_of(C, ph, E, g.u);
+          for (int j = g.j0; j < g.j1; ++j) {
+            const int slot = q % STAGES;
+            if (!mbar_wait(&C.empty[slot], static_cast<uint32_t>((q / STAGES) & 1) ^ 1u, abort_flag, kTimeoutNs)) {
+              ok = false;
+              break;
+            }
+            unsigned char* dst = base + slot * STAGE_BYTES;
+            if (wt) {
+              mbar_expect_tx(&full[slot], W_BYTES);
+              if (ph == 0)
+                tma_load_3d(dst, (j & 1) ? mWu : mWg, &full[slot], 0, U.e * p.f + U.rb * BM, (j >> 1) * CH);
+              else
+                tma_load_3d(dst, mWd, &full[slot], 0, U.e * p.d + U.rb * BM, j * CH);
+            } else if (ph == 0) {
+              mbar_expect_tx(&full[slot], X_BYTES);
+              tma_load_3d(dst + W_BYTES, mX, &full[slot], 0, U.row0, (j >> 1) * CH);
+            } else {
+              if (U.e != ready_e) {
+                // every phase-A unit of expert e must have stored its h rows
+                const unsigned int target = static_cast<unsigned int>(C.ustart[0][U.e + 1] - C.ustart[0][U.e]);
+                const uint64_t t0 = globaltimer();
+                for (uint32_t it = 0; ld_acquire(p.ready + U.e) < target; ++it) {
+                  if ((it & 15) == 15 && (*abort_flag || globaltimer() - t0 > kTimeoutNs)) {
+                    ok = false;
+                    break;
+                  }
+                }
+                if (!ok) break;
+                ready_e = U.e;
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+              }
+              mbar_expect_tx(&full[slot], HP_BYTES);
+              tma_load_4d(dst + W_BYTES, mH, &full[slot], 0, U.row0, 0, j * CH);
+            }
+            ++q;
+          }
+        }
+      }
+      if (!ok) set_abort(C, p.timeouts);
+      if (*abort_flag) drain_ring(full, q);   // no copy may land after the CTA has gone
+    }
+  } else if (warp == 1) {
+    // ===================================== MMA issuer =====================================
+    if (lane == 0) {
+      int q = 0;     // stages consumed
+      int seg = 0;   // segments (accumulator uses)
+      bool ok = true;
+      for (int ph = 0; ph < 2 && ok; ++ph) {
+        const Plan P = make_plan(C.rlo[ph][cta], C.rlo[ph][cta + 1], S[ph]);
+        for (int i = 0; i < P.n && ok; ++i) {
+          const Seg g = seg_at(P, i);
+          const int b = seg & 1;
+          if (!mbar_wait(&C.tempty[b], static_cast<uint32_t>((seg >> 1) & 1) ^ 1u, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int j = g.j0; j < g.j1; ++j, ++q) {
+            const int slot = q % STAGES;
+            const uint32_t par = static_cast<uint32_t>((q / STAGES) & 1);
+            if (!mbar_wait(&C.full_w[slot], par, abort_flag, kTimeoutNs) ||
+                !mbar_wait(&C.full_t[slot], par, abort_flag, kTimeoutNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(base + slot * STAGE_BYTES);
+            const uint32_t sb = sa + W_BYTES;
+            if (ph == 0) {
+              // gate and up stages alternate: the first stage of each matrix in the segment is one of
+              // the first two, and its first MMA overwrites that accumulator
+              const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * 32 + (j & 1) * 16);
+              const bool fresh = j - g.j0 < 2;
+#pragma unroll
+              for (int c = 0; c < CH; ++c)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  umma_bf16(d_tmem, sw128_desc(sa + c * (BM * 128) + kk * 32), sw128_desc(sb + c * (NT * 128) + kk * 32),
+                            kIdesc, (fresh && c == 0 && kk == 0) ? 0u : 1u);
+            } else {
+              // h_hi and h_lo slices of chunk c sit at 2c and 2c + 1 (2 KB each)
+              const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * 32);
+              const bool fresh = j == g.j0;
+#pragma unroll
+              for (int c = 0; c < CH; ++c)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t ad = sw128_desc(sa + c * (BM * 128) + kk * 32);
+                  umma_bf16(d_tmem, ad, sw128_desc(sb + (2 * c) * (NT * 128) + kk * 32), kIdesc,
+                            (fresh && c == 0 && kk == 0) ? 0u : 1u);
+                  umma_bf16(d_tmem, ad, sw128_desc(sb + (2 * c + 1) * (NT * 128) + kk * 32), kIdesc, 1u);
+                }
+            }
+            umma_commit(&C.empty[slot]);
+          }
+          if (!ok) break;
+          umma_commit(&C.tfull[b]);
+          ++seg;
+        }
+      }
+      if (!ok) set_abort(C, p.timeouts);
+      // every MMA this thread issued completes before the drain barrier flips
+      umma_commit(&C.drain);
+      const uint64_t t1 = globaltimer();
+      while (!mbar_try_wait(&C.drain, 0) && globaltimer() - t1 < kTimeoutNs) {
+      }
+    }
+  } else {
+    // ===================================== epilogue (warps 2..5) =====================================
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;                 // accumulator row = TMEM lane
+    const int et = threadIdx.x - 64;                     // 0..127 in the epilogue group
+    int seg = 0;
+    bool ok = true;
+    for (int ph = 0; ph < 2 && ok; ++ph) {
+      const Plan P = make_plan(C.rlo[ph][cta], C.rlo[ph][cta + 1], S[ph]);
+      const int* rlo = C.rlo[ph];
+      for (int i = 0; i < P.n; ++i) {
+        const Seg sg = seg_at(P, i);
+        const int b = seg & 1;
+        // all four warps take the same branch (a warp alone at a named barrier would never leave it)
+        ok = bar_and(1, 128, mbar_wait(&C.tfull[b], static_cast<uint32_t>((seg >> 1) & 1), abort_flag, kTimeoutNs));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * 32);
+        float g[NT], v[NT];
+        {
+          uint32_t r0[16], r1[16];
+          tmem_ld16(taddr, r0);
+          if (ph == 0) tmem_ld16(taddr + 16, r1);
+          tmem_wait_ld();
+          // a segment without gate (up) stages left that accumulator untouched: it contributes 0
+          const bool has_g = ph == 1 || sg.j0 < sg.j1 - 1 || (sg.j0 & 1) == 0;
+          const bool has_u = ph == 0 && (sg.j0 < sg.j1 - 1 || (sg.j0 & 1) == 1);
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            g[t] = has_g ? __uint_as_float(r0[t]) : 0.f;
+            v[t] = has_u ? __uint_as_float(r1[t]) : 0.f;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&C.tempty[b]);
+        ++seg;
+
+        const Unit U = unit_of(C, ph, E, sg.u);
+        if (!(sg.j0 == 0 && sg.j1 == P.S)) {
+          // leave this CTA's partial sums, then let the last contributor finish the unit
+          const size_t part_elems = static_cast<size_t>(ph == 0 ? 2 : 1) * NT * BM;
+          float* const part = ph == 0 ? p.part_a : p.part_b;
+          {
+            float* pp = part + (static_cast<size_t>(cta) * 2 + (rlo[cta] / P.S == sg.u ? 0 : 1)) * part_elems;
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+              if (t < U.rows) {
+                pp[t * BM + row] = g[t];
+                if (ph == 0) pp[NT * BM + t * BM + row] = v[t];
+              }
+          }
+          const int c_first = cta_of(rlo, nC, sg.u * P.S);
+          const int c_last = cta_of(rlo, nC, (sg.u + 1) * P.S - 1);
+          int ncontrib = 0;
+          for (int c2 = c_first; c2 <= c_last; ++c2) ncontrib += rlo[c2 + 1] > rlo[c2];
+          epi_bar();
+          if (et == 0) {
+            unsigned int* cnt = (ph ? p.cnt_b : p.cnt_a) + sg.u;
+            C.last_flag = (atom_acq_rel_add(cnt, 1u) == static_cast<unsigned int>(ncontrib - 1)) ? 1 : 0;
+          }
+          epi_bar();
+          if (!C.last_flag) continue;
+          // sum the contributions in CTA order, two contributors' loads in flight at a time
+#pragma unroll
+          for (int t = 0; t < NT; ++t) g[t] = v[t] = 0.f;
+          for (int c2 = c_first; c2 <= c_last; c2 += 2) {
+            float ga[2][NT], va[2][NT];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int c3 = c2 + k;
+              const bool live = c3 <= c_last && rlo[c3 + 1] > rlo[c3];
+              const float* pp =
+                  part + (static_cast<size_t>(live ? c3 : cta) * 2 + (live && rlo[c3] / P.S == sg.u ? 0 : 1)) * part_elems;
+#pragma unroll
+              for (int t = 0; t < NT; ++t) {
+                const bool in = live && t < U.rows;
+                ga[k][t] = in ? __ldcg(pp + t * BM + row) : 0.f;
+                va[k][t] = (in && ph == 0) ? __ldcg(pp + NT * BM + t * BM + row) : 0.f;
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+#pragma unroll
+              for (int t = 0; t < NT; ++t) {
+                g[t] += ga[k][t];
+                v[t] += va[k][t];
+              }
+          }
+        }
+        // the unit's final epilogue
+        const int n = U.rb * BM + row;
+        if (ph == 0) {
+          const size_t ld = static_cast<size_t>(2) * p.f;
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            if (t < U.rows) {
+              const float hv = g[t] / (1.f + expf(-g[t])) * v[t];
+              const uint16_t hi = f32_to_bf16_bits(hv);
+              uint16_t* hr = p.h + static_cast<size_t>(U.row0 + t) * ld;
+              hr[n] = hi;
+              hr[p.f + n] = f32_to_bf16_bits(hv - bf16_to_f32(hi));
+            }
+          }
+          epi_bar();
+          if (et == 0) red_release_add(p.ready + U.e, 1u);
+        } else {
+#pragma unroll
+          for (int t = 0; t < NT; ++t)
+            if (t < U.rows) p.y[static_cast<size_t>(U.row0 + t) * p.d + n] = g[t];
+          if (p.fuse) {
+            if (p.k == 1) {
+              // one row per token: y = residual + gate * y_perm, written here
+#pragma unroll
+              for (int t = 0; t < NT; ++t)
+                if (t < U.rows) {
+                  const int tok = C.rowsrc[U.row0 + t];
+                  const size_t o = static_cast<size_t>(tok) * p.d + n;
+                  float acc = fmaf(__ldcg(p.gates + tok), g[t], 0.f);
+                  if (p.residual) acc += p.residual[o];
+                  p.out[o] = acc;
+                }
+            } else {
+              // two rows per token, in different units: the later of the two forms the sum from both
+              // rows in slot order, so the result does not depend on which unit finished first
+              epi_bar();
+              if (et < U.rows) {
+                const int tok = C.rowsrc[U.row0 + et];
+                const int want = (C.invp[2 * tok] >= 0) + (C.invp[2 * tok + 1] >= 0);
+                const unsigned int old = atom_acq_rel_add(p.comb_cnt + static_cast<size_t>(tok) * (p.d / BM) + U.rb, 1u);
+                C.last_tok[et] = old == static_cast<unsigned int>(want - 1);
+              }
+              epi_bar();
+#pragma unroll
+              for (int t = 0; t < NT; ++t)
+                if (t < U.rows && C.last_tok[t]) {
+                  const int tok = C.rowsrc[U.row0 + t];
+                  const size_t o = static_cast<size_t>(tok) * p.d + n;
+                  float acc = 0.f;
+#pragma unroll
+                  for (int s = 0; s < 2; ++s) {
+                    const int r = C.invp[2 * tok + s];
+                    if (r >= 0) acc = fmaf(__ldcg(p.gates + 2 * tok + s), __ldcg(p.y + static_cast<size_t>(r) * p.d + n), acc);
+                  }
+                  if (p.residual) acc += p.residual[o];
+                  p.out[o] = acc;
+                }
+            }
+          }
+        }
+      }
+    }
+    if (!ok) set_abort(C, p.timeouts);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// kernel 1: the grouped SwiGLU (offsets from the caller)
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, 1)
+    dec_tc_kernel(const __grid_constant__ CUtensorMap mapWg, const __grid_constant__ CUtensorMap mapWu,
+                  const __grid_constant__ CUtensorMap mapWd, const __grid_constant__ CUtensorMap mapX,
+                  const __grid_constant__ CUtensorMap mapH, DecArgs p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  Ctrl& C = *reinterpret_cast<Ctrl*>(base + STAGES * STAGE_BYTES);
+  const int S[2] = {2 * (p.d / KS), p.f / KS};   // stages per unit; phase A alternates gate / up along k
+  init_ctrl(C);
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) C.off[i] = p.offsets[i];
+  __syncthreads();
+  build_tables(C, p, S);
+  const uint32_t tmem = C.tmem_base;
+  if (!C.bad) ffn_roles(&mapWg, &mapWu, &mapWd, &mapX, &mapH, p, C, base, tmem, S);
+  // The producer and MMA roles run on lane 0 alone: the other lanes wait here for it, so that every
+  // warp meets the CTA barrier (and warp 1 the TMEM release) converged.
+  __syncwarp();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// kernel 2: the fused MoE layer
+// ------------------------------------------------------------------------------------------
+
+// Grid-wide barrier over a counter zeroed before the launch: arrival `round` waits for
+// round * gridDim.x arrivals (bounded; on expiry the CTA aborts).  False after an abort.
+__device__ __forceinline__ bool grid_barrier(unsigned int* ctr, unsigned int round, Ctrl& C, unsigned int* timeouts) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    red_release_add(ctr, 1u);
+    const unsigned int target = round * gridDim.x;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 0; ld_acquire(ctr) < target; ++it) {
+      if ((it & 15) == 15 && globaltimer() - t0 > kTimeoutNs) {
+        set_abort(C, timeouts);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  return *reinterpret_cast<volatile int*>(&C.abort) == 0;
+}
+
+__device__ __forceinline__ float block_sum(float v, Ctrl& C) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) C.red[warp] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int w = 0; w < kWarps; ++w) s += C.red[w];
+    C.red[kWarps] = s;
+  }
+  __syncthreads();
+  return C.red[kWarps];
+}
+
+// Larger score first, then lower expert index.
+__device__ __forceinline__ bool better(float s, int e, float s2, int e2) { return s > s2 || (s == s2 && e < e2); }
+
+__device__ __forceinline__ void warp_argmax(float& s, int& e) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float so = __shfl_xor_sync(0xffffffffu, s, o);
+    const int eo = __shfl_xor_sync(0xffffffffu, e, o);
+    if (better(so, eo, s, e)) {
+      s = so;
+      e = eo;
+    }
+  }
+}
+
+// Phase 0a scratch in the ring (byte offsets; all multiples of 16).
+struct RouteSmem {
+  float* xs;           // [d]    the routed row, f32 values of the bf16 layer input
+  unsigned char* raw;  // [4 d]  the token row as loaded (f32 h or bf16 x)
+  float* gam;          // [d]
+  uint16_t* wr;        // [E, d] the router matrix, or null when it does not fit (read from global)
+};
+
+__device__ __forceinline__ RouteSmem route_smem(unsigned char* base, int d, int E) {
+  RouteSmem R;
+  R.xs = reinterpret_cast<float*>(base + kScratch0);
+  R.raw = base + kScratch0 + 4 * d;
+  R.gam = reinterpret_cast<float*>(base + kScratch0 + 8 * d);
+  const size_t w_off = static_cast<size_t>(kScratch0) + 12 * static_cast<size_t>(d);
+  R.wr = (w_off + static_cast<size_t>(E) * d * 2 <= static_cast<size_t>(kRingBytes))
+             ? reinterpret_cast<uint16_t*>(base + w_off)
+             : nullptr;
+  return R;
+}
+
+// Bulk copy of `bytes` (multiple of 16) in pieces of at most 32 KB onto one mbarrier phase.
+__device__ __forceinline__ void bulk_load_split(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  for (uint32_t o = 0; o < bytes; o += 32768u) {
+    const uint32_t n = bytes - o < 32768u ? bytes - o : 32768u;
+    bulk_load(static_cast<unsigned char*>(dst) + o, static_cast<const unsigned char*>(src) + o, n, bar);
+  }
+}
+
+// Phase 0a for the `it`-th token t of this CTA (whole CTA): the routed input row (RMSNorm'd from
+// h_in when gamma is given, rounded to bf16 like the layer input it stands for), its E logits, the
+// top-k and the gates.  Thread 0 has the router matrix and gamma in flight on rbar[0] (first token)
+// and loads the token row onto rbar[1].  False when a wait gave up.
+__device__ __forceinline__ bool route_token(const LayerArgs& L, const DecArgs& p, Ctrl& C, const RouteSmem& R, int t,
+                                            int it) {
+  const int d = p.d, E = p.E, k = p.k;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &C.abort;
+  if (threadIdx.x == 0) {
+    // generic reads of the previous row are done (barrier at the end of the last token)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    const uint32_t bytes = static_cast<uint32_t>(d) * (L.gamma ? 4u : 2u);
+    mbar_expect_tx(&C.rbar[1], bytes);
+    bulk_load_split(R.raw, L.gamma ? static_cast<const void*>(L.h_in + static_cast<size_t>(t) * d)
+                                   : static_cast<const void*>(L.x_in + static_cast<size_t>(t) * d),
+                    bytes, &C.rbar[1]);
+  }
+  bool ok = mbar_wait(&C.rbar[1], static_cast<uint32_t>(it & 1), abort_flag, kTimeoutNs);
+  if (it == 0 && (L.gamma || R.wr)) ok = ok && mbar_wait(&C.rbar[0], 0, abort_flag, kTimeoutNs);
+  if (!__syncthreads_and(ok)) {
+    if (threadIdx.x == 0) set_abort(C, p.timeouts);
+    return false;
+  }
+  if (L.gamma) {
+    const float* hr = reinterpret_cast<const float*>(R.raw);
+    float ss = 0.f;
+    for (int v = threadIdx.x; v < d / 4; v += kThreads) {
+      const float4 a = reinterpret_cast<const float4*>(hr)[v];
+      ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+    }
+    ss = block_sum(ss, C);
+    const float inv = rsqrtf(ss / static_cast<float>(d) + L.eps);
+    for (int v = threadIdx.x; v < d / 8; v += kThreads) {
+      uint16_t b[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        b[i] = f32_to_bf16_bits(hr[8 * v + i] * inv * R.gam[8 * v + i]);
+        R.xs[8 * v + i] = bf16_to_f32(b[i]);
+      }
+      uint4 pk;
+      pk.x = b[0] | (static_cast<uint32_t>(b[1]) << 16);
+      pk.y = b[2] | (static_cast<uint32_t>(b[3]) << 16);
+      pk.z = b[4] | (static_cast<uint32_t>(b[5]) << 16);
+      pk.w = b[6] | (static_cast<uint32_t>(b[7]) << 16);
+      reinterpret_cast<uint4*>(L.x_norm + static_cast<size_t>(t) * d)[v] = pk;
+    }
+  } else {
+    for (int v = threadIdx.x; v < d / 8; v += kThreads)
+      unpack_bf16x8(reinterpret_cast<const uint4*>(R.raw)[v], R.xs + 8 * v);
+  }
+  __syncthreads();
+  // logits, fp32 accumulation: thread i owns the 8-wide slices i, i + 224, ... of the row and
+  // accumulates all experts on them, then the partial sums are reduced over each warp and across
+  // the warps
+  for (int e0 = 0; e0 < E; e0 += 16) {
+    float acc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+    for (int v = threadIdx.x; v < d / 8; v += kThreads) {
+      float xv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) xv[i] = R.xs[8 * v + i];
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (e0 + j < E) {
+          const uint4 w = R.wr ? reinterpret_cast<const uint4*>(R.wr + static_cast<size_t>(e0 + j) * d)[v]
+                               : __ldg(reinterpret_cast<const uint4*>(L.w_r + static_cast<size_t>(e0 + j) * d) + v);
+          float wf[8];
+          unpack_bf16x8(w, wf);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[j] = fmaf(wf[i], xv[i], acc[j]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) C.wpart[warp][j] = acc[j];
+    }
+    __syncthreads();
+    if (threadIdx.x < 16 && e0 + threadIdx.x < E) {
+      float sum = 0.f;
+      for (int w = 0; w < kWarps; ++w) sum += C.wpart[w][threadIdx.x];
+      C.logit[e0 + threadIdx.x] = sum;
+    }
+    __syncthreads();
+  }
+  if (warp == 0) {
+    const float NEG = -INFINITY;
+    float q[2], s[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int e = lane + 32 * h;
+      const bool ok = e < E;
+      q[h] = ok ? C.logit[e] + (L.logit_bias ? L.logit_bias[e] : 0.f) : NEG;
+      s[h] = ok ? q[h] + (L.sel_bias ? L.sel_bias[e] : 0.f) : NEG;
+    }
+    // ranks 1..3 of s (rank 3 only for the top-2 margin)
+    int sel[3] = {0x7fffffff, 0x7fffffff, 0x7fffffff};
+    float sv[3] = {NEG, NEG, NEG};
+    for (int r = 0; r < (k == 2 ? 3 : 2); ++r) {
+      float bs = NEG;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int e = lane + 32 * h;
+        bool taken = e >= E;
+        for (int r2 = 0; r2 < r; ++r2) taken |= sel[r2] == e;
+        if (!taken && better(s[h], e, bs, be)) {
+          bs = s[h];
+          be = e;
+        }
+      }
+      warp_argmax(bs, be);
+      sel[r] = be;
+      sv[r] = bs;
+    }
+    // softmax over q
+    float m = fmaxf(q[0], q[1]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float z = (lane < E ? expf(q[0] - m) : 0.f) + (lane + 32 < E ? expf(q[1] - m) : 0.f);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane == 0) {
+      const float q1 = C.logit[sel[0]] + (L.logit_bias ? L.logit_bias[sel[0]] : 0.f);
+      if (k == 1) {
+        L.expert_idx[t] = sel[0];
+        L.gates[t] = expf(q1 - m) / z;
+        if (L.margin) L.margin[t] = (E > 1) ? sv[0] - sv[1] : INFINITY;
+      } else {
+        const float q2 = C.logit[sel[1]] + (L.logit_bias ? L.logit_bias[sel[1]] : 0.f);
+        const float z1 = expf(q1 - m), z2 = expf(q2 - m);
+        const float inv = 1.f / (z1 + z2);
+        L.expert_idx[2 * t] = sel[0];
+        L.expert_idx[2 * t + 1] = sel[1];
+        L.gates[2 * t] = z1 * inv;
+        L.gates[2 * t + 1] = z2 * inv;
+        if (L.margin) L.margin[t] = (E > 2) ? fminf(sv[0] - sv[1], sv[1] - sv[2]) : sv[0] - sv[1];
+      }
+    }
+  }
+  __syncthreads();
+  return true;
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Phase 0b (every CTA, redundantly): counts, offsets and the stable (expert, token) order of all
+// T * k assignments into C.off / C.rowsrc / C.invp; CTA 0 publishes them; each CTA gathers its
+// share of x_perm.  ids and per-assignment ranks use the (idle) ring as scratch.
+__device__ __forceinline__ void permute_all(const LayerArgs& L, const DecArgs& p, Ctrl& C, int* ids, int* rel) {
+  const int n = L.T * p.k, E = p.E;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int a = threadIdx.x; a < n; a += kThreads) {
+    int e = __ldcg(L.expert_idx + a);
+    if (e < 0 || e >= E) {
+      if (blockIdx.x == 0) record_device_error(p.errors);
+      e = -1;
+    }
+    ids[a] = e;
+  }
+  if (threadIdx.x < E) C.run[threadIdx.x] = 0;
+  __syncthreads();
+  for (int b0 = 0; b0 < n; b0 += kThreads) {
+    for (int i = threadIdx.x; i < kWarps * kMaxE; i += kThreads) (&C.wcnt[0][0])[i] = 0;
+    __syncthreads();
+    const int a = b0 + threadIdx.x;
+    const int e = a < n ? ids[a] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lanemask_lt());
+    if (e >= 0 && rank == 0) C.wcnt[warp][e] = __popc(peers);
+    __syncthreads();
+    if (threadIdx.x < E) {
+      int r = C.run[threadIdx.x];
+      for (int w = 0; w < kWarps; ++w) {
+        const int c = C.wcnt[w][threadIdx.x];
+        C.wcnt[w][threadIdx.x] = r;
+        r += c;
+      }
+      C.run[threadIdx.x] = r;
+    }
+    __syncthreads();
+    if (e >= 0) rel[a] = C.wcnt[warp][e] + rank;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    C.off[0] = 0;
+    for (int e = 0; e < E; ++e) C.off[e + 1] = C.off[e] + C.run[e];
+  }
+  __syncthreads();
+  for (int a = threadIdx.x; a < n; a += kThreads) {
+    const int e = ids[a];
+    if (e >= 0) {
+      const int pos = C.off[e] + rel[a];
+      C.invp[a] = pos;
+      C.rowsrc[pos] = a / p.k;
+    } else {
+      C.invp[a] = -1;
+    }
+  }
+  __syncthreads();
+  const int rows = C.off[E];
+  if (blockIdx.x == 0) {
+    for (int i = threadIdx.x; i < E; i += kThreads) L.counts[i] = C.run[i];
+    for (int i = threadIdx.x; i <= E; i += kThreads) L.offsets[i] = C.off[i];
+    for (int i = threadIdx.x; i < rows; i += kThreads) L.perm[i] = C.rowsrc[i];
+    for (int i = threadIdx.x; i < n; i += kThreads) L.inv_perm[i] = C.invp[i];
+  }
+  // x_perm rows, one warp per row, spread over the grid
+  const uint16_t* xsrc = L.gamma ? L.x_norm : L.x_in;
+  const int vecs = p.d / 8;
+  for (int r = blockIdx.x * kWarps + warp; r < rows; r += gridDim.x * kWarps) {
+    const uint4* s = reinterpret_cast<const uint4*>(xsrc + static_cast<size_t>(C.rowsrc[r]) * p.d);
+    uint4* dst = reinterpret_cast<uint4*>(L.x_perm + static_cast<size_t>(r) * p.d);
+    for (int v0 = 0; v0 < vecs; v0 += 32 * 8) {
+      uint4 buf[8];   // eight loads in flight per lane
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (v0 + j * 32 + lane < vecs) buf[j] = __ldcg(s + v0 + j * 32 + lane);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (v0 + j * 32 + lane < vecs) dst[v0 + j * 32 + lane] = buf[j];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    moe_layer_kernel(const __grid_constant__ CUtensorMap mapWg, const __grid_constant__ CUtensorMap mapWu,
+                     const __grid_constant__ CUtensorMap mapWd, const __grid_constant__ CUtensorMap mapX,
+                     const __grid_constant__ CUtensorMap mapH, DecArgs p, LayerArgs L) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  Ctrl& C = *reinterpret_cast<Ctrl*>(base + STAGES * STAGE_BYTES);
+  const int S[2] = {2 * (p.d / KS), p.f / KS};
+  init_ctrl(C);
+  __syncthreads();
+  // the ring is idle until the SwiGLU roles start: phase 0 keeps its scratch there
+  int* ids = reinterpret_cast<int*>(base);
+  int* rel = ids + kMaxAssign;
+  const RouteSmem R = route_smem(base, p.d, p.E);
+  const uint32_t wb = R.wr ? static_cast<uint32_t>(p.E) * p.d * 2u : 0u;
+  const uint32_t gb = L.gamma ? static_cast<uint32_t>(p.d) * 4u : 0u;
+  const bool armed0 = static_cast<int>(blockIdx.x) < L.T && wb + gb > 0;
+  if (threadIdx.x == 0 && armed0) {
+    // the router matrix (when it fits) and gamma, once per CTA, with the TMA engine: one SM's plain
+    // loads keep too few bytes in flight to fetch 64 KB quickly
+    mbar_expect_tx(&C.rbar[0], wb + gb);
+    if (wb) bulk_load_split(R.wr, L.w_r, wb, &C.rbar[0]);
+    if (gb) bulk_load_split(R.gam, L.gamma, gb, &C.rbar[0]);
+  }
+  bool ok = true;
+  int nrow = 0;   // token rows loaded onto rbar[1]
+  for (int t = blockIdx.x; t < L.T && ok; t += gridDim.x) ok = route_token(L, p, C, R, t, nrow++);
+  if (!ok && threadIdx.x == 0) {
+    // bulk copies that may still be landing in the ring must finish before the CTA moves on
+    const uint64_t t1 = globaltimer();
+    while (((armed0 && !mbar_try_wait(&C.rbar[0], 0)) ||
+            (nrow > 0 && !mbar_try_wait(&C.rbar[1], static_cast<uint32_t>((nrow - 1) & 1)))) &&
+           globaltimer() - t1 < kTimeoutNs) {
+    }
+  }
+  if (grid_barrier(L.gbar, 1, C, p.timeouts)) {
+    permute_all(L, p, C, ids, rel);
+    // generic-proxy writes to the ring are ordered before the TMA writes that will reuse it
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (grid_barrier(L.gbar, 2, C, p.timeouts)) {
+      build_tables(C, p, S);
+      if (!C.bad) ffn_roles(&mapWg, &mapWu, &mapWd, &mapX, &mapH, p, C, base, C.tmem_base, S);
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == 1) {
+    tc_fence_after();
+    tmem_dealloc(C.tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------
+
+// Upper bound of the token blocks over all experts (the exact count depends on device offsets).
+int ntb_bound(int M_total, int E) { return (M_total + NT - 1) / NT + E; }
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+struct Layout {
+  size_t ready, cnt_a, cnt_b, comb, gbar, counters_end;   // counters (one memset)
+  size_t part_a, part_b;
+  size_t total;
+  int ua, ub;
+};
+
+// Counters first (zeroed per call), then the per-CTA partial slots.
+Layout ffn_layout(int M_total, int E, int d, int f, int T_comb) {
+  Layout Lo{};
+  Lo.ua = ntb_bound(M_total, E) * (f / BM);
+  Lo.ub = ntb_bound(M_total, E) * (d / BM);
+  size_t o = 0;
+  Lo.ready = o;
+  o += static_cast<size_t>(E) * 4;
+  Lo.cnt_a = o;
+  o += static_cast<size_t>(Lo.ua) * 4;
+  Lo.cnt_b = o;
+  o += static_cast<size_t>(Lo.ub) * 4;
+  Lo.comb = o;
+  o += static_cast<size_t>(T_comb) * (d / BM) * 4;
+  Lo.gbar = o;
+  o += 4;
+  Lo.counters_end = align256(o);
+  Lo.part_a = Lo.counters_end;
+  Lo.part_b = Lo.part_a + static_cast<size_t>(num_sms()) * 2 * 2 * NT * BM * 4;
+  Lo.total = Lo.part_b + static_cast<size_t>(num_sms()) * 2 * NT * BM * 4;
+  return Lo;
+}
+
+struct Maps {
+  CUtensorMap g, u, dn, x, h;
+};
+
+bool encode_maps(Maps* m, const uint16_t* x_perm, int M_total, const uint16_t* w_gate, const uint16_t* w_up,
+                 const uint16_t* w_down, int E, int d, int f, const uint16_t* h) {
+  // weights viewed as [K/64 chunks][rows][64]: a box of 128 rows x 4 chunks lands as
+  // [chunk][row][128 B], the K-major 128-byte-swizzle layout the MMA descriptors describe
+  const cuuint64_t dg[3] = {64, static_cast<cuuint64_t>(E) * f, static_cast<cuuint64_t>(d) / 64};
+  const cuuint64_t sg[2] = {static_cast<cuuint64_t>(d) * 2, 128};
+  const cuuint32_t bw[3] = {64, BM, CH};
+  const cuuint64_t dd[3] = {64, static_cast<cuuint64_t>(E) * d, static_cast<cuuint64_t>(f) / 64};
+  const cuuint64_t sd[2] = {static_cast<cuuint64_t>(f) * 2, 128};
+  // token slices: x rows [chunk][16 rows][128 B]; h pair rows [chunk][hi | lo][16 rows][128 B]
+  const cuuint64_t dx[3] = {64, static_cast<cuuint64_t>(M_total), static_cast<cuuint64_t>(d) / 64};
+  const cuuint64_t sx[2] = {static_cast<cuuint64_t>(d) * 2, 128};
+  const cuuint32_t bx[3] = {64, NT, CH};
+  const cuuint64_t dh[4] = {64, static_cast<cuuint64_t>(M_total), 2, static_cast<cuuint64_t>(f) / 64};
+  const cuuint64_t shh[3] = {static_cast<cuuint64_t>(f) * 4, static_cast<cuuint64_t>(f) * 2, 128};
+  const cuuint32_t bh[4] = {64, NT, 2, CH};
+  return encode_bf16_map(&m->g, w_gate, 3, dg, sg, bw) && encode_bf16_map(&m->u, w_up, 3, dg, sg, bw) &&
+         encode_bf16_map(&m->dn, w_down, 3, dd, sd, bw) && encode_bf16_map(&m->x, x_perm, 3, dx, sx, bx) &&
+         encode_bf16_map(&m->h, h, 4, dh, shh, bh);
+}
+
+template <typename K, typename... Args>
+zmoe_status launch_coop(K kernel, const char* what, cudaStream_t s, Args... args) {
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes)) !=
+      cudaSuccess)
+    return check_launch(what);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms()));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: CTAs wait on one another
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) return fail(ZMOE_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return check_launch(what);
+}
+
+DecArgs dec_args(const Layout& Lo, void* ws, const int32_t* offsets, uint16_t* h, float* y_perm, int E, int d, int f,
+                 int M_total) {
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  DecArgs a{};
+  a.offsets = offsets;
+  a.h = h;
+  a.y = y_perm;
+  a.ready = reinterpret_cast<unsigned int*>(w + Lo.ready);
+  a.cnt_a = reinterpret_cast<unsigned int*>(w + Lo.cnt_a);
+  a.cnt_b = reinterpret_cast<unsigned int*>(w + Lo.cnt_b);
+  a.part_a = reinterpret_cast<float*>(w + Lo.part_a);
+  a.part_b = reinterpret_cast<float*>(w + Lo.part_b);
+  a.timeouts = device_timeout_counter();
+  a.errors = device_error_counter();
+  a.E = E;
+  a.d = d;
+  a.f = f;
+  a.M_total = M_total;
+  a.ua_cap = Lo.ua;
+  a.ub_cap = Lo.ub;
+  return a;
+}
+
+}  // namespace
+
+bool grouped_swiglu_dec_tc_supported(int d, int f) {
+  return d % KS == 0 && f % KS == 0 && num_sms() <= kMaxCtas && kSmemBytes <= static_cast<size_t>(max_smem_optin());
+}
+
+size_t grouped_swiglu_dec_tc_workspace(int M_total, int E, int d, int f) {
+  return ffn_layout(M_total, E, d, f, 0).total;
+}
+
+// h: bf16 [M, 2f] (h_hi | h_lo); y_perm: f32 [M, d]; ws: grouped_swiglu_dec_tc_workspace() bytes.
+zmoe_status grouped_swiglu_dec_tc(const uint16_t* x_perm, const int32_t* offsets, int M_total, const uint16_t* w_gate,
+                                  const uint16_t* w_up, const uint16_t* w_down, int E, int d, int f, uint16_t* h,
+                                  float* y_perm, void* ws, cudaStream_t s) {
+  if (!grouped_swiglu_dec_tc_supported(d, f) || E > kMaxE)
+    return fail(ZMOE_ERR_UNSUPPORTED, "grouped_swiglu (decode): needs d % 256 == 0, f % 256 == 0, E <= 64");
+  Maps m;
+  if (!encode_maps(&m, x_perm, M_total, w_gate, w_up, w_down, E, d, f, h))
+    return fail(ZMOE_ERR_CUDA, "grouped_swiglu (decode): cuTensorMapEncodeTiled failed");
+  const Layout Lo = ffn_layout(M_total, E, d, f, 0);
+  if (cudaMemsetAsync(ws, 0, Lo.counters_end, s) != cudaSuccess)
+    return check_launch("grouped_swiglu (decode): clearing the counters");
+  const DecArgs args = dec_args(Lo, ws, offsets, h, y_perm, E, d, f, M_total);
+  return launch_coop(dec_tc_kernel, "grouped_swiglu (decode)", s, m.g, m.u, m.dn, m.x, m.h, args);
+}
+
+// ------------------------------------------------------------------------------------------
+// the fused layer: workspace carve-up and launch
+// ------------------------------------------------------------------------------------------
+bool moe_layer_fused_supported(int T, int E, int d, int f, int k) {
+  return grouped_swiglu_dec_tc_supported(d, f) && E <= kMaxE && T >= 1 && static_cast<long long>(T) * k <= kMaxAssign &&
+         static_cast<long long>(kScratch0) + 12LL * d <= kRingBytes;
+}
+
+struct LayerWs {
+  Layout ffn;
+  size_t x_norm, x_perm, h, y_perm, idx, gates, margin, counts, offsets, perm, inv_perm, total;
+};
+
+LayerWs layer_ws(int T, int E, int d, int f, int k) {
+  LayerWs W{};
+  const int n = T * k;
+  W.ffn = ffn_layout(n, E, d, f, T);
+  size_t o = align256(W.ffn.total);
+  auto take = [&o](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  W.x_norm = take(static_cast<size_t>(T) * d * 2);
+  W.x_perm = take(static_cast<size_t>(n) * d * 2);
+  W.h = take(static_cast<size_t>(n) * 2 * f * 2);
+  W.y_perm = take(static_cast<size_t>(n) * d * 4);
+  W.idx = take(static_cast<size_t>(n) * 4);
+  W.gates = take(static_cast<size_t>(n) * 4);
+  W.margin = take(static_cast<size_t>(T) * 4);
+  W.counts = take(static_cast<size_t>(E) * 4);
+  W.offsets = take(static_cast<size_t>(E + 1) * 4);
+  W.perm = take(static_cast<size_t>(n) * 4);
+  W.inv_perm = take(static_cast<size_t>(n) * 4);
+  W.total = o;
+  return W;
+}
+
+size_t moe_layer_fused_workspace(int T, int E, int d, int f, int k) { return layer_ws(T, E, d, f, k).total; }
+
+zmoe_status moe_layer_fused(const uint16_t* x, const float* h_in, const float* gamma, float eps, const uint16_t* w_r,
+                            const float* logit_bias, const float* sel_bias, const uint16_t* w_gate,
+                            const uint16_t* w_up, const uint16_t* w_down, int T, int d, int f, int E, int k, float* y,
+                            int32_t* expert_idx, float* gates, float* margin, uint16_t* x_norm_out, void* ws,
+                            cudaStream_t s) {
+  const LayerWs W = layer_ws(T, E, d, f, k);
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  const int n = T * k;
+  uint16_t* xn = x_norm_out ? x_norm_out : reinterpret_cast<uint16_t*>(w + W.x_norm);
+  uint16_t* xp = reinterpret_cast<uint16_t*>(w + W.x_perm);
+  uint16_t* hh = reinterpret_cast<uint16_t*>(w + W.h);
+  float* yp = reinterpret_cast<float*>(w + W.y_perm);
+  Maps m;
+  if (!encode_maps(&m, xp, n, w_gate, w_up, w_down, E, d, f, hh))
+    return fail(ZMOE_ERR_CUDA, "zmoe_moe_layer: cuTensorMapEncodeTiled failed");
+  if (cudaMemsetAsync(ws, 0, W.ffn.counters_end, s) != cudaSuccess)
+    return check_launch("zmoe_moe_layer: clearing the counters");
+  DecArgs a = dec_args(W.ffn, ws, nullptr, hh, yp, E, d, f, n);
+  LayerArgs L{};
+  L.x_in = x;
+  L.h_in = h_in;
+  L.gamma = gamma;
+  L.eps = eps;
+  L.w_r = w_r;
+  L.logit_bias = logit_bias;
+  L.sel_bias = sel_bias;
+  L.T = T;
+  L.x_norm = xn;
+  L.expert_idx = expert_idx ? expert_idx : reinterpret_cast<int32_t*>(w + W.idx);
+  L.gates = gates ? gates : reinterpret_cast<float*>(w + W.gates);
+  L.margin = margin;
+  L.counts = reinterpret_cast<int32_t*>(w + W.counts);
+  L.offsets = reinterpret_cast<int32_t*>(w + W.offsets);
+  L.perm = reinterpret_cast<int32_t*>(w + W.perm);
+  L.inv_perm = reinterpret_cast<int32_t*>(w + W.inv_perm);
+  L.x_perm = xp;
+  L.gbar = reinterpret_cast<unsigned int*>(w + W.ffn.gbar);
+  a.fuse = 1;
+  a.k = k;
+  a.gates = L.gates;
+  a.residual = h_in;
+  a.out = y;
+  a.comb_cnt = reinterpret_cast<unsigned int*>(w + W.ffn.comb);
+  return launch_coop(moe_layer_kernel, "zmoe_moe_layer (fused decode)", s, m.g, m.u, m.dn, m.x, m.h, a, L);
+}
+
+}  // namespace zmoe

@@ -1,7 +1,8 @@
 """The MoE layer and the batch-1 decode stack, chained through libzmoe's C entry points.
 
 Buffers are allocated once (torch is used for device memory only); every step runs in
-libzmoe's kernels:
+libzmoe's kernels.  A layer is one call of ``zmoe_moe_layer`` (one cooperative launch at
+decode sizes); ``MoELayerRunner.run_steps`` chains the separate entry points instead:
 
     zmoe_route -> zmoe_permute -> zmoe_grouped_swiglu -> zmoe_combine
 
@@ -84,10 +85,26 @@ class MoELayerRunner:
         self.ffn_ws = torch.empty(max(Z.zmoe_grouped_swiglu_workspace_size(M, E, d, f, dtype), 16),
                                   dtype=torch.uint8, device=dev)
         self.y = torch.empty((T, d), dtype=torch.float32, device=dev)
+        self.layer_ws = torch.empty(max(Z.zmoe_moe_layer_workspace_size(T, d, f, E, k, dtype), 16), dtype=torch.uint8,
+                                    device=dev)
 
-    def run(self, x: torch.Tensor, W: MoEWeights, residual: Optional[torch.Tensor] = None,
-            out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-        """y = residual + sum_i gate_i * FFN_{e_i}(x), f32 [T, d]."""
+    def run(self, x: Optional[torch.Tensor], W: MoEWeights, residual: Optional[torch.Tensor] = None,
+            out: Optional[torch.Tensor] = None, stream=None, gamma: Optional[torch.Tensor] = None, eps: float = 1e-6,
+            x_norm: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """y = residual + sum_i gate_i * FFN_{e_i}(x), f32 [T, d], in one zmoe_moe_layer call.
+
+        With ``gamma`` the layer input is RMSNorm(residual) * gamma (written to ``x_norm`` if given)."""
+        outs = dict(expert_idx=self.idx, gates=self.gates, margin=self.margin)
+        if x_norm is not None:
+            outs["x_norm"] = x_norm
+        return Z.zmoe_moe_layer(W.w_router, W.w_gate, W.w_up, W.w_down, W.k, x=x, h=residual, gamma=gamma, eps=eps,
+                                logit_bias=W.logit_bias, sel_bias=W.sel_bias,
+                                out=self.y if out is None else out, outs=outs, workspace=self.layer_ws,
+                                stream=stream)
+
+    def run_steps(self, x: torch.Tensor, W: MoEWeights, residual: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """The same layer through the four separate entry points (intermediates kept in this runner)."""
         Z.zmoe_route(x, W.w_router, W.k, W.logit_bias, W.sel_bias, outs=(self.idx, self.gates, self.margin),
                      stream=stream)
         Z.zmoe_permute(self.idx, x, W.E, outs=self.perm_outs, workspace=self.perm_ws, stream=stream)
@@ -123,13 +140,14 @@ class DecodeStack:
         if self.record_inputs:
             self.layer_inputs, self.layer_h, self.layer_idx = [], [], []
         for L in self.layers:
-            Z.zmoe_rmsnorm(self.h, L.gamma, self.eps, out=self.x, stream=stream)
+            R = self.runners[L.k]
             if self.record_inputs:
                 self.layer_h.append(self.h.clone())
-                self.layer_inputs.append(self.x.clone())
-            R = self.runners[L.k]
-            R.run(self.x, L, residual=self.h, out=self.h, stream=stream)
+            # h <- h + MoE(RMSNorm(h) * gamma): one zmoe_moe_layer call, in place
+            R.run(None, L, residual=self.h, out=self.h, stream=stream, gamma=L.gamma, eps=self.eps,
+                  x_norm=self.x if self.record_inputs else None)
             if self.record_inputs:
+                self.layer_inputs.append(self.x.clone())
                 self.layer_idx.append(R.idx.clone())
         return self.h
 

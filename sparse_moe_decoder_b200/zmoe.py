@@ -43,6 +43,9 @@ SIGNATURES = {
     "zmoe_grouped_swiglu_workspace_size": (_S, [_I, _I, _I, _I, _I]),
     "zmoe_grouped_swiglu": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _S, _P]),
     "zmoe_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "zmoe_moe_layer_workspace_size": (_S, [_I, _I, _I, _I, _I, _I]),
+    "zmoe_moe_layer": (_I, [_P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                            _P, _S, _P]),
     "zmoe_get_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
 }
 
@@ -261,6 +264,44 @@ def zmoe_combine(y_perm: torch.Tensor, inv_perm: torch.Tensor, gates: torch.Tens
     y = out if out is not None else torch.empty((T, d), dtype=torch.float32, device=y_perm.device)
     _check(lib().zmoe_combine(_ptr(y_perm), _ptr(inv_perm), _ptr(gates), _ptr(residual), T, d, k, _ptr(y),
                               _stream(stream)), "zmoe_combine")
+    return y
+
+
+def zmoe_moe_layer_workspace_size(T: int, d: int, f: int, E: int, k: int, dtype: torch.dtype) -> int:
+    return int(lib().zmoe_moe_layer_workspace_size(T, d, f, E, k, _dtype_code(dtype)))
+
+
+def zmoe_moe_layer(w_router: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor, k: int,
+                   x: Optional[torch.Tensor] = None, h: Optional[torch.Tensor] = None,
+                   gamma: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                   logit_bias: Optional[torch.Tensor] = None, sel_bias: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None, outs: Optional[dict] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y = h + MoE(x), or with gamma y = h + MoE(RMSNorm(h) * gamma); f32 [T, d].
+
+    ``outs`` may hold preallocated ``expert_idx`` int32 [T, k], ``gates`` f32 [T, k], ``margin`` f32 [T]
+    and ``x_norm`` [T, d] tensors to receive those intermediates.
+    """
+    src = h if gamma is not None else x
+    if src is None:
+        raise ValueError("zmoe_moe_layer: needs x, or h with gamma")
+    T, d = src.shape
+    E, f = w_gate.shape[0], w_gate.shape[1]
+    dt = w_router.dtype
+    if x is not None:
+        _need(x, "x", dt, 2)
+    if h is not None:
+        _need(h, "h", torch.float32, 2)
+    outs = outs or {}
+    y = out if out is not None else torch.empty((T, d), dtype=torch.float32, device=src.device)
+    ws_bytes = zmoe_moe_layer_workspace_size(T, d, f, E, k, dt)
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=src.device)
+    _check(lib().zmoe_moe_layer(_ptr(x), _ptr(h), _ptr(gamma), float(eps), _ptr(w_router), _ptr(logit_bias),
+                                _ptr(sel_bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _dtype_code(dt), T, d, f, E,
+                                k, _ptr(y), _ptr(outs.get("expert_idx")), _ptr(outs.get("gates")),
+                                _ptr(outs.get("margin")), _ptr(outs.get("x_norm")), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream)), "zmoe_moe_layer")
     return y
 
 

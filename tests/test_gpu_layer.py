@@ -1,4 +1,5 @@
-"""The whole MoE layer (route -> permute -> grouped SwiGLU -> combine) through the C-ABI vs the oracle.
+"""The whole MoE layer through the C-ABI vs the oracle: zmoe_moe_layer (one call) and the four separate
+entry points (route -> permute -> grouped SwiGLU -> combine).
 
 Configurations 1 and 2 are compared on every token (configuration 2, T = 64, is the decode step the
 benchmark times, in the same launch configuration).  Configurations 3 and 4 (T = 16384) compare all
@@ -16,26 +17,28 @@ from tests.gpu_util import MARGIN_EXEMPT, TOL, assert_close, host, rel_err, requ
 pytestmark = pytest.mark.gpu
 
 
-def run_layer(L):
+def run_layer(L, steps=False):
     dt = tdtype(L.dtype)
     W = MoEWeights.from_host(L)
     R = MoELayerRunner(L.T, L.E, L.d, L.f, L.k, dt)
-    y = R.run(to_dev(L.x, dt), W)
+    y = (R.run_steps if steps else R.run)(to_dev(L.x, dt), W)
     return R, host(y)
 
 
 @pytest.mark.parametrize("cfg", [1, 2])
-def test_layer_every_token(cfg):
+@pytest.mark.parametrize("steps", [False, True], ids=["one_call", "separate_calls"])
+def test_layer_every_token(cfg, steps):
     require_gpu()
     L = make_config(cfg)
-    R, y = run_layer(L)
+    R, y = run_layer(L, steps)
     ref = oracle.moe_layer(L.x, L.w_router, L.w_gate, L.w_up, L.w_down, L.k, L.sel_bias, L.logit_bias)
     idx = host(R.idx)
     ok = ref["margin"] >= MARGIN_EXEMPT
     assert np.array_equal(idx[ok], ref["expert_idx"][ok])
     same = (idx == ref["expert_idx"]).all(1)
     r = assert_close(y[same], ref["y"][same], L.dtype, f"config {cfg} y")
-    assert np.array_equal(host(R.perm_outs["counts"]), ref["counts"]) or not ok.all()
+    counts = host(R.perm_outs["counts"]) if steps else np.bincount(idx.ravel(), minlength=L.E)
+    assert np.array_equal(counts, ref["counts"]) or not ok.all()
     print(f"config {cfg}: y max err {r:.2e} x RMS; {int((~ok).sum())} low-margin tokens exempt")
 
 
