@@ -11,7 +11,8 @@
 // Design of the SwiGLU part:
 //   * Swap-AB on tcgen05: 128 weight rows are the MMA's M, a block of up to 16 token rows is its N
 //     (kind::f16, bf16 in, fp32 accumulate in TMEM).  A unit is (expert, 128-row weight block, token
-//     block); its k-range is cut into 256-wide stages (a 64 KB weight box + an 8/16 KB token box).
+//     block); its k-range is cut into 128-wide stages (a 32 KB weight box + a 4 KB x slice or an
+//     8 KB h-pair slice).
 //   * Stream-K: every CTA (one per SM, cooperative launch: all resident) takes an equal,
 //     contiguous range of the stage list of each phase, so bytes per SM balance to within one
 //     stage whatever the expert loads are (down to a single expert at batch 1).  A unit wholly
@@ -20,7 +21,8 @@
 //     (deterministic) and finishes it.  Each CTA runs its (at most two) cut units first, so the
 //     cross-CTA hand-offs overlap the whole units that follow.
 //   * Roles: warp 0 loads weight boxes and warp 6 token boxes (x, or the h pair) with TMA into a
-//     2-stage ring (160 KB; a 64 KB box is the size at which one SM's TMA reaches full HBM rate),
+//     5-stage ring (200 KB: 160 KB of weights in flight per SM; boxes of 32 KB or more keep one
+//     SM's TMA near full HBM rate; 5 x 32 KB measured 2% faster than 2 x 64 KB on the decode step),
 //     each completing on its own mbarrier, so weight loads never wait for h; warp 1 allocates TMEM
 //     and issues the MMAs from one thread (tcgen05.commit frees a stage when its MMAs are done);
 //     warps 2..5 read the accumulators with tcgen05.ld and run the epilogues.
@@ -51,12 +53,12 @@ using namespace ptx;
 
 constexpr int BM = 128;                       // weight rows per unit (MMA M)
 constexpr int NT = 16;                        // token rows per block (MMA N)
-constexpr int KS = 256;                       // k per stage
+constexpr int KS = 128;                       // k per stage
 constexpr int CH = KS / 64;                   // 64-wide chunks per stage
-constexpr int STAGES = 2;
-constexpr int W_BYTES = BM * KS * 2;          // 64 KB
-constexpr int X_BYTES = NT * KS * 2;          // 8 KB  x slice
-constexpr int HP_BYTES = NT * KS * 2 * 2;     // 16 KB h_hi + h_lo slice
+constexpr int STAGES = 5;
+constexpr int W_BYTES = BM * KS * 2;          // 32 KB
+constexpr int X_BYTES = NT * KS * 2;          // 4 KB  x slice
+constexpr int HP_BYTES = NT * KS * 2 * 2;     // 8 KB  h_hi + h_lo slice
 constexpr int STAGE_BYTES = W_BYTES + HP_BYTES;
 constexpr int kThreads = 224;                 // 7 warps
 constexpr int kWarps = kThreads / 32;
@@ -70,6 +72,7 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(BM, NT);
 // fused layer, phase 0 scratch in the (then idle) ring: ids, ranks, the routed row (f32), the raw
 // token row, gamma, and the router matrix when it fits
 constexpr int kRingBytes = STAGES * STAGE_BYTES;
+
 constexpr int kScratch0 = 2 * kMaxAssign * 4;
 
 struct DecArgs {
@@ -91,6 +94,9 @@ struct DecArgs {
   const float* residual;    // [T, d] or null
   float* out;               // [T, d] (may alias residual)
   unsigned int* comb_cnt;   // [T, d / BM] units of each token's row block done (k = 2)
+  // fused layer: x_perm is complete once this counter reaches x_target (grid-wide arrivals)
+  const unsigned int* x_ready;
+  unsigned int x_target;
 };
 
 struct LayerArgs {
@@ -111,7 +117,9 @@ struct LayerArgs {
   int32_t* perm;            // [T * k]
   int32_t* inv_perm;        // [T, k]
   uint16_t* x_perm;         // [T * k, d]
+  float* logits;            // [T, E] router logits, exchanged through the grid barrier
   unsigned int* gbar;       // grid barrier arrivals
+  int G, EG;                // phase-0 items: (token, expert group); EG experts per group
 };
 
 struct __align__(16) Ctrl {
@@ -133,14 +141,17 @@ struct __align__(16) Ctrl {
   // fused layer
   int rowsrc[kMaxAssign];    // permuted row -> token
   int invp[kMaxAssign];      // assignment (t, i) -> permuted row
+  float gsm[kMaxAssign];     // gate of assignment (t, i)
   int wcnt[kWarps][kMaxE];
   int run[kMaxE];
   float red[kWarps + 1];
   float wpart[kWarps][16];
-  float logit[kMaxE];
+  float lbias[kMaxE];        // logit_bias (0 when absent)
+  float sbias[kMaxE];        // selection bias (0 when absent)
 };
 
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + sizeof(Ctrl);
+static_assert(kSmemBytes <= 227 * 1024, "ring + control block exceed the 227 KB a B200 CTA may use");
 
 // ------------------------------------------------------------------------------------------
 // work geometry (every role walks the same sequence)
@@ -311,7 +322,17 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
       int q = 0;            // stages armed on `full`
       bool ok = true;
       int ready_e = -1;     // last expert whose phase-A units were all seen complete
-      if (!wt) asm volatile("fence.proxy.async.global;" ::: "memory");   // x_perm may come from this launch
+      if (!wt && p.x_ready) {
+        // x_perm is written in this launch by every CTA: wait for all of them (weights need not)
+        const uint64_t t0 = globaltimer();
+        for (uint32_t it = 0; ld_acquire(p.x_ready) < p.x_target; ++it) {
+          if ((it & 15) == 15 && (*abort_flag || globaltimer() - t0 > kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+        }
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
       for (int ph = 0; ph < 2 && ok; ++ph) {
         const Plan P = make_plan(C.rlo[ph][cta], C.rlo[ph][cta + 1], S[ph]);
         for (int i = 0; i < P.n && ok; ++i) {
@@ -319,7 +340,8 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
           const Unit U = unit_of(C, ph, E, g.u);
           for (int j = g.j0; j < g.j1; ++j) {
             const int slot = q % STAGES;
-            if (!mbar_wait(&C.empty[slot], static_cast<uint32_t>((q / STAGES) & 1) ^ 1u, abort_flag, kTimeoutNs)) {
+            const uint32_t epar = static_cast<uint32_t>((q / STAGES) & 1) ^ 1u;
+            if (!mbar_wait(&C.empty[slot], epar, abort_flag, kTimeoutNs)) {
               ok = false;
               break;
             }
@@ -542,7 +564,7 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
                 if (t < U.rows) {
                   const int tok = C.rowsrc[U.row0 + t];
                   const size_t o = static_cast<size_t>(tok) * p.d + n;
-                  float acc = fmaf(__ldcg(p.gates + tok), g[t], 0.f);
+                  float acc = fmaf(C.gsm[tok], g[t], 0.f);
                   if (p.residual) acc += p.residual[o];
                   p.out[o] = acc;
                 }
@@ -566,7 +588,7 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
 #pragma unroll
                   for (int s = 0; s < 2; ++s) {
                     const int r = C.invp[2 * tok + s];
-                    if (r >= 0) acc = fmaf(__ldcg(p.gates + 2 * tok + s), __ldcg(p.y + static_cast<size_t>(r) * p.d + n), acc);
+                    if (r >= 0) acc = fmaf(C.gsm[2 * tok + s], __ldcg(p.y + static_cast<size_t>(r) * p.d + n), acc);
                   }
                   if (p.residual) acc += p.residual[o];
                   p.out[o] = acc;
@@ -663,19 +685,19 @@ __device__ __forceinline__ void warp_argmax(float& s, int& e) {
 
 // Phase 0a scratch in the ring (byte offsets; all multiples of 16).
 struct RouteSmem {
-  float* xs;           // [d]    the routed row, f32 values of the bf16 layer input
-  unsigned char* raw;  // [4 d]  the token row as loaded (f32 h or bf16 x)
+  float* xs;           // [d]     the routed row, f32 values of the bf16 layer input
+  unsigned char* raw;  // [4 d]   the token row as loaded (f32 h or bf16 x)
   float* gam;          // [d]
-  uint16_t* wr;        // [E, d] the router matrix, or null when it does not fit (read from global)
+  uint16_t* wr;        // [EG, d] this CTA's router rows, or null when they do not fit (read from global)
 };
 
-__device__ __forceinline__ RouteSmem route_smem(unsigned char* base, int d, int E) {
+__device__ __forceinline__ RouteSmem route_smem(unsigned char* base, int d, int EG) {
   RouteSmem R;
   R.xs = reinterpret_cast<float*>(base + kScratch0);
   R.raw = base + kScratch0 + 4 * d;
   R.gam = reinterpret_cast<float*>(base + kScratch0 + 8 * d);
   const size_t w_off = static_cast<size_t>(kScratch0) + 12 * static_cast<size_t>(d);
-  R.wr = (w_off + static_cast<size_t>(E) * d * 2 <= static_cast<size_t>(kRingBytes))
+  R.wr = (w_off + static_cast<size_t>(EG) * d * 2 <= static_cast<size_t>(kRingBytes))
              ? reinterpret_cast<uint16_t*>(base + w_off)
              : nullptr;
   return R;
@@ -689,17 +711,20 @@ __device__ __forceinline__ void bulk_load_split(void* dst, const void* src, uint
   }
 }
 
-// Phase 0a for the `it`-th token t of this CTA (whole CTA): the routed input row (RMSNorm'd from
-// h_in when gamma is given, rounded to bf16 like the layer input it stands for), its E logits, the
-// top-k and the gates.  Thread 0 has the router matrix and gamma in flight on rbar[0] (first token)
-// and loads the token row onto rbar[1].  False when a wait gave up.
-__device__ __forceinline__ bool route_token(const LayerArgs& L, const DecArgs& p, Ctrl& C, const RouteSmem& R, int t,
-                                            int it) {
-  const int d = p.d, E = p.E, k = p.k;
+// Phase 0a item `it` of this CTA: token t, expert group g (experts [g EG, g EG + ne)).  The routed
+// input row (RMSNorm'd from h_in when gamma is given, rounded to bf16 like the layer input it stands
+// for; group 0 publishes it as x_norm) and its logits for the group's experts, published to
+// L.logits.  Thread 0 has this CTA's router rows and gamma in flight on rbar[0] and loads the token
+// row onto rbar[1].  False when a wait gave up.
+__device__ __forceinline__ bool route_item(const LayerArgs& L, const DecArgs& p, Ctrl& C, const RouteSmem& R, int t,
+                                           int g, int it) {
+  const int d = p.d, E = p.E;
+  const int e0 = g * L.EG;
+  const int ne = (E - e0) < L.EG ? (E - e0) : L.EG;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &C.abort;
   if (threadIdx.x == 0) {
-    // generic reads of the previous row are done (barrier at the end of the last token)
+    // generic reads of the previous row are done (barrier at the end of the last item)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     const uint32_t bytes = static_cast<uint32_t>(d) * (L.gamma ? 4u : 2u);
     mbar_expect_tx(&C.rbar[1], bytes);
@@ -729,12 +754,14 @@ __device__ __forceinline__ bool route_token(const LayerArgs& L, const DecArgs& p
         b[i] = f32_to_bf16_bits(hr[8 * v + i] * inv * R.gam[8 * v + i]);
         R.xs[8 * v + i] = bf16_to_f32(b[i]);
       }
-      uint4 pk;
-      pk.x = b[0] | (static_cast<uint32_t>(b[1]) << 16);
-      pk.y = b[2] | (static_cast<uint32_t>(b[3]) << 16);
-      pk.z = b[4] | (static_cast<uint32_t>(b[5]) << 16);
-      pk.w = b[6] | (static_cast<uint32_t>(b[7]) << 16);
-      reinterpret_cast<uint4*>(L.x_norm + static_cast<size_t>(t) * d)[v] = pk;
+      if (g == 0) {
+        uint4 pk;
+        pk.x = b[0] | (static_cast<uint32_t>(b[1]) << 16);
+        pk.y = b[2] | (static_cast<uint32_t>(b[3]) << 16);
+        pk.z = b[4] | (static_cast<uint32_t>(b[5]) << 16);
+        pk.w = b[6] | (static_cast<uint32_t>(b[7]) << 16);
+        reinterpret_cast<uint4*>(L.x_norm + static_cast<size_t>(t) * d)[v] = pk;
+      }
     }
   } else {
     for (int v = threadIdx.x; v < d / 8; v += kThreads)
@@ -742,9 +769,9 @@ __device__ __forceinline__ bool route_token(const LayerArgs& L, const DecArgs& p
   }
   __syncthreads();
   // logits, fp32 accumulation: thread i owns the 8-wide slices i, i + 224, ... of the row and
-  // accumulates all experts on them, then the partial sums are reduced over each warp and across
-  // the warps
-  for (int e0 = 0; e0 < E; e0 += 16) {
+  // accumulates up to 16 experts on them, then the partial sums are reduced over each warp and
+  // across the warps
+  for (int j0 = 0; j0 < ne; j0 += 16) {
     float acc[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) acc[j] = 0.f;
@@ -754,9 +781,9 @@ __device__ __forceinline__ bool route_token(const LayerArgs& L, const DecArgs& p
       for (int i = 0; i < 8; ++i) xv[i] = R.xs[8 * v + i];
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        if (e0 + j < E) {
-          const uint4 w = R.wr ? reinterpret_cast<const uint4*>(R.wr + static_cast<size_t>(e0 + j) * d)[v]
-                               : __ldg(reinterpret_cast<const uint4*>(L.w_r + static_cast<size_t>(e0 + j) * d) + v);
+        if (j0 + j < ne) {
+          const uint4 w = R.wr ? reinterpret_cast<const uint4*>(R.wr + static_cast<size_t>(j0 + j) * d)[v]
+                               : __ldg(reinterpret_cast<const uint4*>(L.w_r + static_cast<size_t>(e0 + j0 + j) * d) + v);
           float wf[8];
           unpack_bf16x8(w, wf);
 #pragma unroll
@@ -773,70 +800,90 @@ __device__ __forceinline__ bool route_token(const LayerArgs& L, const DecArgs& p
       for (int j = 0; j < 16; ++j) C.wpart[warp][j] = acc[j];
     }
     __syncthreads();
-    if (threadIdx.x < 16 && e0 + threadIdx.x < E) {
+    if (threadIdx.x < 16 && j0 + threadIdx.x < ne) {
       float sum = 0.f;
       for (int w = 0; w < kWarps; ++w) sum += C.wpart[w][threadIdx.x];
-      C.logit[e0 + threadIdx.x] = sum;
+      L.logits[static_cast<size_t>(t) * E + e0 + j0 + threadIdx.x] = sum;
     }
     __syncthreads();
   }
-  if (warp == 0) {
-    const float NEG = -INFINITY;
-    float q[2], s[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int e = lane + 32 * h;
-      const bool ok = e < E;
-      q[h] = ok ? C.logit[e] + (L.logit_bias ? L.logit_bias[e] : 0.f) : NEG;
-      s[h] = ok ? q[h] + (L.sel_bias ? L.sel_bias[e] : 0.f) : NEG;
-    }
-    // ranks 1..3 of s (rank 3 only for the top-2 margin)
-    int sel[3] = {0x7fffffff, 0x7fffffff, 0x7fffffff};
-    float sv[3] = {NEG, NEG, NEG};
-    for (int r = 0; r < (k == 2 ? 3 : 2); ++r) {
-      float bs = NEG;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int e = lane + 32 * h;
-        bool taken = e >= E;
-        for (int r2 = 0; r2 < r; ++r2) taken |= sel[r2] == e;
-        if (!taken && better(s[h], e, bs, be)) {
-          bs = s[h];
-          be = e;
-        }
+  return true;
+}
+
+// Phase 0b (every CTA, one thread per token): top-k of s = q + sel_bias (ties -> lower index) and
+// the softmax gates of q = logit + logit_bias, from the published logits.  Writes the choices to
+// ids (shared, [T k]) and the gates to C.gsm; CTA 0 also publishes expert_idx, gates and margin.
+__device__ __forceinline__ void select_all(const LayerArgs& L, const DecArgs& p, Ctrl& C, int* ids, float* scratch,
+                                           size_t scratch_bytes) {
+  const int E = p.E, k = p.k;
+  const float NEG = -INFINITY;
+  // all logits at once (one coalesced pass) when they fit in the scratch, so that the per-token
+  // loops below read shared memory instead of issuing dependent global loads
+  const size_t nl = static_cast<size_t>(L.T) * E;
+  const float* lbase = L.logits;
+  if (nl * 4 <= scratch_bytes) {
+    for (size_t i = threadIdx.x; i < nl; i += kThreads) scratch[i] = __ldcg(L.logits + i);
+    lbase = scratch;
+  }
+  for (int e = threadIdx.x; e < E; e += kThreads) {
+    C.lbias[e] = L.logit_bias ? L.logit_bias[e] : 0.f;
+    C.sbias[e] = L.sel_bias ? L.sel_bias[e] : 0.f;
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < L.T; t += kThreads) {
+    const float* lg = lbase + static_cast<size_t>(t) * E;
+    float s1 = NEG, s2 = NEG, s3 = NEG, q1 = NEG, q2 = NEG, m = NEG;
+    int e1 = -1, e2 = -1;
+    for (int e = 0; e < E; ++e) {
+      const float q = lg[e] + C.lbias[e];
+      const float sc = q + C.sbias[e];
+      m = fmaxf(m, q);
+      // strict ">" keeps the lower index on ties (experts arrive in increasing order)
+      if (e1 < 0 || sc > s1) {
+        s3 = s2;
+        s2 = s1;
+        e2 = e1;
+        q2 = q1;
+        s1 = sc;
+        e1 = e;
+        q1 = q;
+      } else if (e2 < 0 || sc > s2) {
+        s3 = s2;
+        s2 = sc;
+        e2 = e;
+        q2 = q;
+      } else if (sc > s3) {
+        s3 = sc;
       }
-      warp_argmax(bs, be);
-      sel[r] = be;
-      sv[r] = bs;
     }
-    // softmax over q
-    float m = fmaxf(q[0], q[1]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float z = (lane < E ? expf(q[0] - m) : 0.f) + (lane + 32 < E ? expf(q[1] - m) : 0.f);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (lane == 0) {
-      const float q1 = C.logit[sel[0]] + (L.logit_bias ? L.logit_bias[sel[0]] : 0.f);
-      if (k == 1) {
-        L.expert_idx[t] = sel[0];
-        L.gates[t] = expf(q1 - m) / z;
-        if (L.margin) L.margin[t] = (E > 1) ? sv[0] - sv[1] : INFINITY;
-      } else {
-        const float q2 = C.logit[sel[1]] + (L.logit_bias ? L.logit_bias[sel[1]] : 0.f);
-        const float z1 = expf(q1 - m), z2 = expf(q2 - m);
-        const float inv = 1.f / (z1 + z2);
-        L.expert_idx[2 * t] = sel[0];
-        L.expert_idx[2 * t + 1] = sel[1];
+    float z = 0.f;
+    for (int e = 0; e < E; ++e) z += expf(lg[e] + C.lbias[e] - m);
+    if (k == 1) {
+      const float gt = expf(q1 - m) / z;
+      ids[t] = e1;
+      C.gsm[t] = gt;
+      if (blockIdx.x == 0) {
+        L.expert_idx[t] = e1;
+        L.gates[t] = gt;
+        if (L.margin) L.margin[t] = (E > 1) ? s1 - s2 : INFINITY;
+      }
+    } else {
+      const float z1 = expf(q1 - m), z2 = expf(q2 - m);
+      const float inv = 1.f / (z1 + z2);
+      ids[2 * t] = e1;
+      ids[2 * t + 1] = e2;
+      C.gsm[2 * t] = z1 * inv;
+      C.gsm[2 * t + 1] = z2 * inv;
+      if (blockIdx.x == 0) {
+        L.expert_idx[2 * t] = e1;
+        L.expert_idx[2 * t + 1] = e2;
         L.gates[2 * t] = z1 * inv;
         L.gates[2 * t + 1] = z2 * inv;
-        if (L.margin) L.margin[t] = (E > 2) ? fminf(sv[0] - sv[1], sv[1] - sv[2]) : sv[0] - sv[1];
+        if (L.margin) L.margin[t] = (E > 2) ? fminf(s1 - s2, s2 - s3) : s1 - s2;
       }
     }
   }
   __syncthreads();
-  return true;
 }
 
 __device__ __forceinline__ unsigned lanemask_lt() {
@@ -845,20 +892,12 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
-// Phase 0b (every CTA, redundantly): counts, offsets and the stable (expert, token) order of all
-// T * k assignments into C.off / C.rowsrc / C.invp; CTA 0 publishes them; each CTA gathers its
-// share of x_perm.  ids and per-assignment ranks use the (idle) ring as scratch.
+// Phase 0b, after select_all (every CTA, redundantly): counts, offsets and the stable (expert, token)
+// order of all T * k assignments in ids into C.off / C.rowsrc / C.invp; CTA 0 publishes them; each
+// CTA gathers its share of x_perm.  ids and per-assignment ranks use the (idle) ring as scratch.
 __device__ __forceinline__ void permute_all(const LayerArgs& L, const DecArgs& p, Ctrl& C, int* ids, int* rel) {
   const int n = L.T * p.k, E = p.E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int a = threadIdx.x; a < n; a += kThreads) {
-    int e = __ldcg(L.expert_idx + a);
-    if (e < 0 || e >= E) {
-      if (blockIdx.x == 0) record_device_error(p.errors);
-      e = -1;
-    }
-    ids[a] = e;
-  }
   if (threadIdx.x < E) C.run[threadIdx.x] = 0;
   __syncthreads();
   for (int b0 = 0; b0 < n; b0 += kThreads) {
@@ -938,20 +977,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the ring is idle until the SwiGLU roles start: phase 0 keeps its scratch there
   int* ids = reinterpret_cast<int*>(base);
   int* rel = ids + kMaxAssign;
-  const RouteSmem R = route_smem(base, p.d, p.E);
-  const uint32_t wb = R.wr ? static_cast<uint32_t>(p.E) * p.d * 2u : 0u;
+  const RouteSmem R = route_smem(base, p.d, L.EG);
+  // this CTA's items (t, g) = (i / G, i % G) for i = blockIdx.x, blockIdx.x + C, ...; with G > 1
+  // there is at most one item per CTA, so the router rows of one group serve all of them
+  const int g0 = static_cast<int>(blockIdx.x) % L.G;
+  const int ne0 = (p.E - g0 * L.EG) < L.EG ? (p.E - g0 * L.EG) : L.EG;
+  const uint32_t wb = R.wr ? static_cast<uint32_t>(ne0) * p.d * 2u : 0u;
   const uint32_t gb = L.gamma ? static_cast<uint32_t>(p.d) * 4u : 0u;
-  const bool armed0 = static_cast<int>(blockIdx.x) < L.T && wb + gb > 0;
+  const bool armed0 = static_cast<int>(blockIdx.x) < L.T * L.G && wb + gb > 0;
   if (threadIdx.x == 0 && armed0) {
-    // the router matrix (when it fits) and gamma, once per CTA, with the TMA engine: one SM's plain
-    // loads keep too few bytes in flight to fetch 64 KB quickly
+    // the router rows (when they fit) and gamma, once per CTA, with the TMA engine: one SM's plain
+    // loads keep too few bytes in flight to fetch tens of KB quickly
     mbar_expect_tx(&C.rbar[0], wb + gb);
-    if (wb) bulk_load_split(R.wr, L.w_r, wb, &C.rbar[0]);
+    if (wb) bulk_load_split(R.wr, L.w_r + static_cast<size_t>(g0) * L.EG * p.d, wb, &C.rbar[0]);
     if (gb) bulk_load_split(R.gam, L.gamma, gb, &C.rbar[0]);
   }
   bool ok = true;
   int nrow = 0;   // token rows loaded onto rbar[1]
-  for (int t = blockIdx.x; t < L.T && ok; t += gridDim.x) ok = route_token(L, p, C, R, t, nrow++);
+  for (int i = blockIdx.x; i < L.T * L.G && ok; i += gridDim.x) ok = route_item(L, p, C, R, i / L.G, i % L.G, nrow++);
   if (!ok && threadIdx.x == 0) {
     // bulk copies that may still be landing in the ring must finish before the CTA moves on
     const uint64_t t1 = globaltimer();
@@ -961,13 +1004,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (grid_barrier(L.gbar, 1, C, p.timeouts)) {
+    select_all(L, p, C, ids, reinterpret_cast<float*>(base + kScratch0), kRingBytes - kScratch0);
     permute_all(L, p, C, ids, rel);
     // generic-proxy writes to the ring are ordered before the TMA writes that will reuse it
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    if (grid_barrier(L.gbar, 2, C, p.timeouts)) {
-      build_tables(C, p, S);
-      if (!C.bad) ffn_roles(&mapWg, &mapWu, &mapWd, &mapX, &mapH, p, C, base, C.tmem_base, S);
-    }
+    build_tables(C, p, S);   // ends with a CTA barrier: this CTA's x_perm rows are written
+    // second grid arrival: x_perm complete here.  Only the token producer waits for all CTAs
+    // (DecArgs::x_ready); the weight producer starts streaming at once.  An epilogue thread arrives
+    // (its release fence waits for this CTA's gather stores; the producers must not wait on it).
+    if (threadIdx.x == 64) red_release_add(L.gbar, 1u);
+    if (!C.bad) ffn_roles(&mapWg, &mapWu, &mapWd, &mapX, &mapH, p, C, base, C.tmem_base, S);
   }
   __syncwarp();
   __syncthreads();
@@ -1120,7 +1166,7 @@ bool moe_layer_fused_supported(int T, int E, int d, int f, int k) {
 
 struct LayerWs {
   Layout ffn;
-  size_t x_norm, x_perm, h, y_perm, idx, gates, margin, counts, offsets, perm, inv_perm, total;
+  size_t x_norm, x_perm, h, y_perm, idx, gates, margin, counts, offsets, perm, inv_perm, logits, total;
 };
 
 LayerWs layer_ws(int T, int E, int d, int f, int k) {
@@ -1144,6 +1190,7 @@ LayerWs layer_ws(int T, int E, int d, int f, int k) {
   W.offsets = take(static_cast<size_t>(E + 1) * 4);
   W.perm = take(static_cast<size_t>(n) * 4);
   W.inv_perm = take(static_cast<size_t>(n) * 4);
+  W.logits = take(static_cast<size_t>(T) * E * 4);
   W.total = o;
   return W;
 }
@@ -1187,12 +1234,23 @@ zmoe_status moe_layer_fused(const uint16_t* x, const float* h_in, const float* g
   L.inv_perm = reinterpret_cast<int32_t*>(w + W.inv_perm);
   L.x_perm = xp;
   L.gbar = reinterpret_cast<unsigned int*>(w + W.ffn.gbar);
+  L.logits = reinterpret_cast<float*>(w + W.logits);
+  // phase-0 items (token, expert group): as many groups as keep every SM busy, up to one per expert
+  {
+    const int nC = num_sms();
+    int G = nC / T;
+    G = G < 1 ? 1 : (G > E ? E : G);
+    L.EG = (E + G - 1) / G;
+    L.G = (E + L.EG - 1) / L.EG;
+  }
   a.fuse = 1;
   a.k = k;
   a.gates = L.gates;
   a.residual = h_in;
   a.out = y;
   a.comb_cnt = reinterpret_cast<unsigned int*>(w + W.ffn.comb);
+  a.x_ready = L.gbar;                                  // second grid arrival: x_perm complete
+  a.x_target = 2u * static_cast<unsigned int>(num_sms());
   return launch_coop(moe_layer_kernel, "zmoe_moe_layer (fused decode)", s, m.g, m.u, m.dn, m.x, m.h, a, L);
 }
 
