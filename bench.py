@@ -42,7 +42,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4, 5, 6])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle timing leg")
@@ -70,6 +70,9 @@ WORKLOADS = {
     4: "final MoE layer: T=16384, d_model=2048, d_ff=3072, E=16, top-2, Zipf(1.2) logit skew, bf16",
     5: "batch-1 decode stack: 9-codebook embedding sum + RMSNorm, 24 pre-norm MoE layers (d_model=2048, "
        "d_ff=3072, E=16, top-1, top-2 in the last), attention omitted, bf16, one token per step",
+    6: "batch-1 full decoder FFN stack: embedding sum + RMSNorm, 3 dense SwiGLU layers, the 24 MoE layers "
+       "(E=16, top-1, top-2 in the last), 1 dense layer; d_model=2048, d_ff=3072, pre-norm residual, "
+       "attention omitted, bf16, one token per step",
 }
 
 
@@ -180,7 +183,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
-    if args.config == 5:
+    if args.config >= 5:
         return run_reference_stack(args)
     from moe_inputs import make_config
     L = make_config(args.config)
@@ -248,7 +251,7 @@ def run_reference_stack(args):
     and kept, so later tokens time the arithmetic, not the drawing."""
     import oracle
     from moe_inputs import StackSpec
-    spec = StackSpec()
+    spec = StackSpec() if args.config == 5 else StackSpec(n_dense_front=3, n_dense_back=1)
     cache = {}
 
     def expert(l, e):
@@ -256,10 +259,7 @@ def run_reference_stack(args):
             cache[(l, e)] = spec.expert(l, e)
         return cache[(l, e)]
 
-    layers = []
-    for l in range(spec.n_layers):
-        wr, sb, gm = spec.layer_small(l)
-        layers.append(dict(w_router=wr, sel_bias=sb, gamma=gm, k=spec.k_of(l), experts=(lambda e, l=l: expert(l, e))))
+    layers = oracle_stack_layers(spec, expert)
     tables, g0 = spec.tables(), spec.gamma0()
     n = max(1, min(args.steps, 3))
     codes = spec.codes(n + 1)
@@ -269,12 +269,12 @@ def run_reference_stack(args):
         oracle.decode_stack_step(codes[i:i + 1], tables, g0, layers, spec.eps)
     el = time.perf_counter() - t0
     v = n / el
-    sample = (f"oracle.decode_stack_step (numpy float64), {n} token(s) through the 24-layer stack "
+    sample = (f"oracle.decode_stack_step (numpy float64), {n} token(s) through the {spec.total_layers}-layer stack "
               f"(experts drawn on first use, outside the timing where already drawn), {el:.1f} s")
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": n, "warmup": 1, "ms_per_step": 1e3 * el / n, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOADS[5], "us_per_token": 1e6 * el / n, "batch": 1},
+            "config": {"workload": WORKLOADS[args.config], "us_per_token": 1e6 * el / n, "batch": 1},
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -282,8 +282,18 @@ def run_reference_stack(args):
     return 0
 
 
+def oracle_stack_layers(spec, expert):
+    """The oracle's per-layer description of the stack (a dense FFN layer has no router)."""
+    layers = []
+    for l in range(spec.total_layers):
+        wr, sb, gm = spec.layer_small(l)
+        layers.append(dict(w_router=wr, sel_bias=sb, gamma=gm, k=spec.k_of(l), experts=(lambda e, l=l: expert(l, e))))
+    return layers
+
+
 def run_stack(args):
-    """Configuration 5: tokens/s (= 1 / s per token) of the 24-layer batch-1 stack."""
+    """Configuration 5: tokens/s (= 1 / s per token) of the 24-layer batch-1 stack; 6: the full 28-layer
+    FFN stack (3 dense + 24 MoE + 1 dense)."""
     import torch
     import torch.distributed as dist
 
@@ -297,9 +307,9 @@ def run_stack(args):
     from sparse_moe_decoder_b200 import zmoe_get_device_errors
     from sparse_moe_decoder_b200.layer import stack_from_bits
 
-    spec = StackSpec()
+    spec = StackSpec() if args.config == 5 else StackSpec(n_dense_front=3, n_dense_back=1)
     st = stack_from_bits(bf16_bits(spec.tables()), spec.gamma0(), spec.layer_small, stack_expert_bits(spec),
-                         spec.n_layers, spec.E, spec.d, spec.f, spec.k_of, spec.eps, T=1)
+                         spec.total_layers, spec.E, spec.d, spec.f, spec.k_of, spec.eps, T=1, E_of=spec.E_of)
     n = args.warmup + args.steps
     codes = spec.codes(n + 1)
     if rank > 0:
@@ -384,15 +394,11 @@ def run_stack(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         t0 = time.perf_counter()
-        layers = []
-        for l in range(spec.n_layers):
-            wr, sb, gm = spec.layer_small(l)
-            layers.append(dict(w_router=wr, sel_bias=sb, gamma=gm, k=spec.k_of(l),
-                               experts=(lambda e, l=l: spec.expert(l, e))))
+        layers = oracle_stack_layers(spec, spec.expert)
         oracle.decode_stack_step(codes[:1], spec.tables(), spec.gamma0(), layers, spec.eps)
         el = time.perf_counter() - t0
         cpu = {"value": 1.0 / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"oracle.decode_stack_step (numpy float64) on one token through all 24 layers, "
+               "sample": f"oracle.decode_stack_step (numpy float64) on one token through all {spec.total_layers} layers, "
                          f"drawing each touched expert's weights as it goes, {el:.1f} s"}
     used_graph = graph is not None
     graph = None          # release the graph before the process group goes away
@@ -401,20 +407,20 @@ def run_stack(args):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOADS[5], "us_per_token": ms_per_step * 1e3, "layers": spec.n_layers,
+            "config": {"workload": WORKLOADS[args.config], "us_per_token": ms_per_step * 1e3, "layers": spec.total_layers,
                        "d_model": spec.d, "d_ff": spec.f, "E": spec.E, "batch": 1,
                        "parallelism": f"dp{world} (replicated weights, no data-path collective)",
                        "l2": "inputs larger than L2 (14.5 GB of weights; ~0.9 GB read per token)",
                        "experts_touched_per_token": touched, "cuda_graph": used_graph},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                         "kernel": "whole decode step (embed + 24 x moe_layer_kernel: pre-norm, router, dispatch, "
-                                   "SwiGLU and combine in one launch per layer)",
+                         "kernel": f"whole decode step (embed + {spec.total_layers} x moe_layer_kernel: pre-norm, "
+                                   "router, dispatch, SwiGLU and combine in one launch per layer)",
                          "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peaks["source"]},
             "cpu_baseline": cpu,
             "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": spec.n_codebooks * 4, "d2h_bytes_per_step": spec.d * 4},
-            "gpu_launches": (1 + spec.n_layers) * args.steps,
+            "gpu_launches": (1 + spec.total_layers) * args.steps,
             "clocks": clk.summary(),
             "device_errors": dev_errors,
         }
@@ -429,7 +435,7 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
-    if args.config == 5:
+    if args.config >= 5:
         return run_stack(args)
 
     import torch

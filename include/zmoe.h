@@ -126,6 +126,8 @@ ZMOE_API zmoe_status zmoe_rmsnorm(const void* h, zmoe_dtype in_dtype, const floa
  *   x: [T, d], w_router: [E, d], both of `dtype`; logit_bias, sel_bias: f32 [E] or NULL
  *   (= zeros); expert_idx: int32 [T, k]; gates: f32 [T, k]; margin: f32 [T] or NULL.
  *   1 <= E <= 64, k in {1, 2}, k <= E, d % 8 == 0; x and w_router 16-byte aligned.
+ *   w_router (and x) may be NULL when E == 1 (a dense FFN layer): every token then gets expert 0
+ *   with gate 1 and margin +inf.
  */
 ZMOE_API zmoe_status zmoe_route(const void* x, const void* w_router, zmoe_dtype dtype, const float* logit_bias,
                        const float* sel_bias, int T, int d, int E, int k, int32_t* expert_idx, float* gates,
@@ -230,6 +232,8 @@ ZMOE_API size_t zmoe_moe_layer_workspace_size(int T, int d, int f, int E, int k,
  *   Outputs: y: f32 [T, d] (may alias h); expert_idx int32 [T, k], gates f32 [T, k],
  *   margin f32 [T] (as zmoe_route) and x_norm [T, d] of `dtype` (the routed input, with
  *   gamma only) are optional (NULL: kept in the workspace).
+ *   w_router may be NULL when E == 1: the layer is then the dense SwiGLU FFN of the decoder's
+ *   dense layers (gate 1), [DIGEST] item 5 (layers 0-2 and 27 are dense).
  *   workspace: zmoe_moe_layer_workspace_size() bytes, 256-byte aligned; it also holds the
  *   intermediates (x_perm, the hidden activations, y_perm).  1 <= E <= 64, k in {1, 2},
  *   k <= E, d % 8 == 0, f % 8 == 0 (bf16: multiples of 256); 16-byte aligned pointers.

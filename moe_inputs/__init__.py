@@ -205,10 +205,30 @@ class StackSpec:
     vocab_rows: int = VOCAB_ROWS
     sel_bias_var: float = 0.1
     eps: float = 1e-6
+    # dense FFN layers before and after the MoE layers (the full decoder has 3 and 1); layer
+    # indices below are stack positions: dense front, then the n_layers MoE layers, then dense back
+    n_dense_front: int = 0
+    n_dense_back: int = 0
+
+    @property
+    def total_layers(self) -> int:
+        return self.n_dense_front + self.n_layers + self.n_dense_back
+
+    def kind(self, layer: int):
+        """("dense", i) for the i-th dense layer, ("moe", m) for the m-th MoE layer."""
+        if layer < self.n_dense_front:
+            return "dense", layer
+        if layer < self.n_dense_front + self.n_layers:
+            return "moe", layer - self.n_dense_front
+        return "dense", layer - self.n_layers
+
+    def E_of(self, layer: int) -> int:
+        return 1 if self.kind(layer)[0] == "dense" else self.E
 
     def k_of(self, layer: int) -> int:
         """top-1 everywhere except top-2 in the last MoE layer."""
-        return 2 if layer == self.n_layers - 1 else 1
+        kind, m = self.kind(layer)
+        return 2 if kind == "moe" and m == self.n_layers - 1 else 1
 
     def _rng(self, *key: int) -> np.random.Generator:
         # Deterministic child stream addressed by an integer key path:
@@ -225,8 +245,13 @@ class StackSpec:
         return (1.0 + 0.1 * self._rng(0, 1).standard_normal(self.d, dtype=np.float32)).astype(np.float32)
 
     def layer_small(self, layer: int):
-        """(W_r [E, d] bf16-exact, b [E] f32, gamma [d] f32) of one layer."""
-        rng = self._rng(1, layer)
+        """(W_r [E, d] bf16-exact, b [E] f32, gamma [d] f32) of one layer; a dense layer has no router
+        (W_r and b are None)."""
+        kind, m = self.kind(layer)
+        if kind == "dense":
+            gamma = (1.0 + 0.1 * self._rng(5, m).standard_normal(self.d, dtype=np.float32)).astype(np.float32)
+            return None, None, gamma
+        rng = self._rng(1, m)
         w_router = _normal(rng, (self.E, self.d), 1.0 / self.d, True)
         sel_bias = (rng.standard_normal(self.E, dtype=np.float32)
                     * np.float32(np.sqrt(self.sel_bias_var))).astype(np.float32)
@@ -234,10 +259,13 @@ class StackSpec:
         return w_router, sel_bias, gamma
 
     def expert(self, layer: int, e: int):
-        """(W_gate [f, d], W_up [f, d], W_down [d, f]) of one expert, bf16-exact."""
-        wg = _normal(self._rng(2, layer, e, 0), (self.f, self.d), 1.0 / self.d, True)
-        wu = _normal(self._rng(2, layer, e, 1), (self.f, self.d), 1.0 / self.d, True)
-        wd = _normal(self._rng(2, layer, e, 2), (self.d, self.f), 1.0 / self.f, True)
+        """(W_gate [f, d], W_up [f, d], W_down [d, f]) of one expert (the FFN of a dense layer, e = 0),
+        bf16-exact."""
+        kind, m = self.kind(layer)
+        key = (2, m, e) if kind == "moe" else (4, m)
+        wg = _normal(self._rng(*key, 0), (self.f, self.d), 1.0 / self.d, True)
+        wu = _normal(self._rng(*key, 1), (self.f, self.d), 1.0 / self.d, True)
+        wd = _normal(self._rng(*key, 2), (self.d, self.f), 1.0 / self.f, True)
         return wg, wu, wd
 
     def codes(self, steps: int) -> np.ndarray:
@@ -251,8 +279,8 @@ class StackSpec:
 # --------------------------------------------------------------------------------------------
 
 def _expert_bits_job(args):
-    seed, layer, e, d, f = args
-    spec = StackSpec(seed=seed, d=d, f=f)
+    seed, layer, e, d, f, front, back = args
+    spec = StackSpec(seed=seed, d=d, f=f, n_dense_front=front, n_dense_back=back)
     return layer, e, tuple(bf16_bits(w) for w in spec.expert(layer, e))
 
 
@@ -261,7 +289,8 @@ def stack_expert_bits(spec: StackSpec, workers: Optional[int] = None):
     the stack, drawn in worker processes (spawned, so it is safe after CUDA has been initialised)."""
     import multiprocessing as mp
     import os as _os
-    jobs = [(spec.seed, l, e, spec.d, spec.f) for l in range(spec.n_layers) for e in range(spec.E)]
+    jobs = [(spec.seed, l, e, spec.d, spec.f, spec.n_dense_front, spec.n_dense_back)
+            for l in range(spec.total_layers) for e in range(spec.E_of(l))]
     n = workers or max(1, min(16, (_os.cpu_count() or 2) - 1))
     if n == 1:
         for j in jobs:

@@ -20,7 +20,7 @@ from typing import Callable, Optional, Sequence
 import numpy as np
 
 from .embed import embed_sum_rmsnorm, rmsnorm
-from .ffn import grouped_swiglu
+from .ffn import grouped_swiglu, swiglu_ffn
 from .permute import permute
 from .route import route
 
@@ -107,15 +107,23 @@ def decode_stack_step(ids: np.ndarray, tables: np.ndarray, gamma0: np.ndarray,
     """Batch-1 (or batch-T) decode through the MoE stack, float64, no intermediate rounding.
 
     ``layers[l]`` holds ``w_router``, ``sel_bias``, ``gamma``, ``k`` and ``experts``
-    (a callable e -> (W_gate, W_up, W_down)).  Returns the final h and per-layer records.
+    (a callable e -> (W_gate, W_up, W_down)); ``w_router`` None marks a dense FFN layer (expert 0,
+    gate 1).  Returns the final h and per-layer records.
     """
     ids = np.atleast_2d(np.asarray(ids))
     h = embed_sum_rmsnorm(ids, tables, gamma0, eps)
     records = []
     for L in layers:
         x = rmsnorm(h, L["gamma"], eps)
-        out = moe_layer(x, L["w_router"], None, None, None, L["k"], sel_bias=L["sel_bias"],
-                        experts=L["experts"])
+        if L["w_router"] is None:
+            # a dense FFN layer (ZONOS2 digest item 5: layers 0-2 and 27): the SwiGLU FFN itself
+            wg, wu, wd = L["experts"](0)
+            y = swiglu_ffn(x, wg, wu, wd)
+            out = dict(expert_idx=np.zeros((x.shape[0], 1), np.int64), gates=np.ones((x.shape[0], 1)),
+                       margin=np.full(x.shape[0], np.inf), y=y)
+        else:
+            out = moe_layer(x, L["w_router"], None, None, None, L["k"], sel_bias=L["sel_bias"],
+                            experts=L["experts"])
         h = h + out["y"]
         records.append(dict(x=x, expert_idx=out["expert_idx"], gates=out["gates"],
                             margin=out["margin"], y=out["y"], h=h.copy()))

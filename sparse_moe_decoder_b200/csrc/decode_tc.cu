@@ -733,7 +733,7 @@ __device__ __forceinline__ bool route_item(const LayerArgs& L, const DecArgs& p,
                     bytes, &C.rbar[1]);
   }
   bool ok = mbar_wait(&C.rbar[1], static_cast<uint32_t>(it & 1), abort_flag, kTimeoutNs);
-  if (it == 0 && (L.gamma || R.wr)) ok = ok && mbar_wait(&C.rbar[0], 0, abort_flag, kTimeoutNs);
+  if (it == 0 && (L.gamma || (R.wr && L.w_r))) ok = ok && mbar_wait(&C.rbar[0], 0, abort_flag, kTimeoutNs);
   if (!__syncthreads_and(ok)) {
     if (threadIdx.x == 0) set_abort(C, p.timeouts);
     return false;
@@ -768,6 +768,11 @@ __device__ __forceinline__ bool route_item(const LayerArgs& L, const DecArgs& p,
       unpack_bf16x8(reinterpret_cast<const uint4*>(R.raw)[v], R.xs + 8 * v);
   }
   __syncthreads();
+  if (!L.w_r) {
+    // no router (E == 1, a dense FFN layer): the single logit is 0 and its gate 1
+    if (threadIdx.x == 0) L.logits[static_cast<size_t>(t) * E] = 0.f;
+    return true;
+  }
   // logits, fp32 accumulation: thread i owns the 8-wide slices i, i + 224, ... of the row and
   // accumulates up to 16 experts on them, then the partial sums are reduced over each warp and
   // across the warps
@@ -982,7 +987,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // there is at most one item per CTA, so the router rows of one group serve all of them
   const int g0 = static_cast<int>(blockIdx.x) % L.G;
   const int ne0 = (p.E - g0 * L.EG) < L.EG ? (p.E - g0 * L.EG) : L.EG;
-  const uint32_t wb = R.wr ? static_cast<uint32_t>(ne0) * p.d * 2u : 0u;
+  const uint32_t wb = (R.wr && L.w_r) ? static_cast<uint32_t>(ne0) * p.d * 2u : 0u;
   const uint32_t gb = L.gamma ? static_cast<uint32_t>(p.d) * 4u : 0u;
   const bool armed0 = static_cast<int>(blockIdx.x) < L.T * L.G && wb + gb > 0;
   if (threadIdx.x == 0 && armed0) {

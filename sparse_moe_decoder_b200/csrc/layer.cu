@@ -90,9 +90,10 @@ zmoe_status zmoe_moe_layer(const void* x, const float* h, const float* gamma, fl
   ZMOE_REQUIRE((k == 1 || k == 2) && k <= E, "zmoe_moe_layer: k must be 1 or 2 and <= E");
   ZMOE_REQUIRE(d >= 8 && d % 8 == 0 && f >= 8 && f % 8 == 0, "zmoe_moe_layer: d and f must be multiples of 8");
   if (T == 0) return ZMOE_OK;
-  ZMOE_REQUIRE(w_router && w_gate && w_up && w_down && y, "zmoe_moe_layer: NULL pointer");
+  ZMOE_REQUIRE((w_router || E == 1) && w_gate && w_up && w_down && y,
+               "zmoe_moe_layer: NULL pointer (w_router may be NULL only when E == 1)");
   ZMOE_REQUIRE(gamma ? h != nullptr : x != nullptr, "zmoe_moe_layer: needs x, or h with gamma");
-  ZMOE_REQUIRE((!x || aligned16(x)) && (!h || aligned16(h)) && aligned16(y) && aligned16(w_router) &&
+  ZMOE_REQUIRE((!x || aligned16(x)) && (!h || aligned16(h)) && aligned16(y) && (!w_router || aligned16(w_router)) &&
                    aligned16(w_gate) && aligned16(w_up) && aligned16(w_down) && (!x_norm || aligned16(x_norm)) &&
                    (!gamma || aligned16(gamma)),
                "zmoe_moe_layer: pointers must be 16-byte aligned");

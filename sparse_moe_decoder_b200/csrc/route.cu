@@ -227,6 +227,17 @@ void launch_route(const void* x, const void* w, const float* lb, const float* sb
   }
 }
 
+// E == 1 without a router: expert 0, gate softmax over one logit = 1, no second choice (margin +inf).
+__global__ void single_expert_kernel(int T, int32_t* __restrict__ expert_idx, float* __restrict__ gates,
+                                     float* __restrict__ margin) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < T) {
+    expert_idx[t] = 0;
+    gates[t] = 1.f;
+    if (margin) margin[t] = INFINITY;
+  }
+}
+
 }  // namespace
 }  // namespace zmoe
 
@@ -241,10 +252,16 @@ extern "C" zmoe_status zmoe_route(const void* x, const void* w_router, zmoe_dtyp
   ZMOE_REQUIRE(k <= E, "zmoe_route: k must be <= E");
   ZMOE_REQUIRE(d >= 8 && d % 8 == 0, "zmoe_route: d must be a positive multiple of 8");
   if (T == 0) return ZMOE_OK;
-  ZMOE_REQUIRE(x && w_router && expert_idx && gates, "zmoe_route: NULL pointer");
-  ZMOE_REQUIRE(aligned16(x) && aligned16(w_router), "zmoe_route: x/w_router not 16-byte aligned");
+  ZMOE_REQUIRE(expert_idx && gates && (!w_router ? E == 1 : x != nullptr),
+               "zmoe_route: NULL pointer (w_router may be NULL only when E == 1)");
+  ZMOE_REQUIRE((!x || aligned16(x)) && (!w_router || aligned16(w_router)), "zmoe_route: x/w_router not 16-byte aligned");
   clear_error();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!w_router) {
+    // one expert and no router (a dense FFN layer): every token goes to expert 0 with gate 1
+    single_expert_kernel<<<(T + 255) / 256, 256, 0, s>>>(T, expert_idx, gates, margin);
+    return check_launch("zmoe_route");
+  }
   if (dtype == ZMOE_BF16)
     launch_route<uint16_t>(x, w_router, logit_bias, sel_bias, T, d, E, k, expert_idx, gates, margin, s);
   else

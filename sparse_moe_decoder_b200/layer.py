@@ -24,9 +24,11 @@ from . import zmoe as Z
 
 @dataclass
 class MoEWeights:
-    """One layer's device weights.  Shapes: W_r [E, d], W_gate/W_up [E, f, d], W_down [E, d, f]."""
+    """One layer's device weights.  Shapes: W_r [E, d], W_gate/W_up [E, f, d], W_down [E, d, f].
 
-    w_router: torch.Tensor
+    A dense FFN layer is the E = 1 case; its router may be None (the gate is 1)."""
+
+    w_router: Optional[torch.Tensor]
     w_gate: torch.Tensor
     w_up: torch.Tensor
     w_down: torch.Tensor
@@ -37,11 +39,11 @@ class MoEWeights:
 
     @property
     def E(self) -> int:
-        return self.w_router.shape[0]
+        return self.w_gate.shape[0]
 
     @property
     def d(self) -> int:
-        return self.w_router.shape[1]
+        return self.w_gate.shape[2]
 
     @property
     def f(self) -> int:
@@ -49,7 +51,7 @@ class MoEWeights:
 
     @property
     def dtype(self) -> torch.dtype:
-        return self.w_router.dtype
+        return self.w_gate.dtype
 
     @staticmethod
     def from_host(L, device="cuda", dtype: Optional[torch.dtype] = None) -> "MoEWeights":
@@ -123,7 +125,7 @@ class DecodeStack:
         L0 = layers[0]
         dev = tables.device
         self.dtype = L0.dtype
-        self.runners = {k: MoELayerRunner(T, L0.E, L0.d, L0.f, k, L0.dtype, dev) for k in {L.k for L in layers}}
+        self.runners = {(L.E, L.k): MoELayerRunner(T, L.E, L.d, L.f, L.k, L.dtype, dev) for L in layers}
         self.ids = torch.empty((T, tables.shape[0]), dtype=torch.int32, device=dev)
         self.h = torch.empty((T, L0.d), dtype=torch.float32, device=dev)
         self.x = torch.empty((T, L0.d), dtype=L0.dtype, device=dev)
@@ -140,7 +142,7 @@ class DecodeStack:
         if self.record_inputs:
             self.layer_inputs, self.layer_h, self.layer_idx = [], [], []
         for L in self.layers:
-            R = self.runners[L.k]
+            R = self.runners[(L.E, L.k)]
             if self.record_inputs:
                 self.layer_h.append(self.h.clone())
             # h <- h + MoE(RMSNorm(h) * gamma): one zmoe_moe_layer call, in place
@@ -153,12 +155,13 @@ class DecodeStack:
 
 
 def stack_from_bits(tables_bits, gamma0, layer_small, expert_bits, n_layers: int, E: int, d: int, f: int,
-                    k_of, eps: float = 1e-6, T: int = 1, device="cuda") -> DecodeStack:
+                    k_of, eps: float = 1e-6, T: int = 1, device="cuda", E_of=None) -> DecodeStack:
     """Builds a DecodeStack on the device from host arrays.
 
     tables_bits: uint16 [N, V, d] bf16 bit patterns; gamma0: f32 [d]; layer_small(l) -> (W_r f32 [E, d]
-    bf16-exact, sel_bias f32 [E], gamma f32 [d]); expert_bits: iterable of (l, e, (wg, wu, wd) uint16
-    bit arrays); k_of(l) -> experts per token in layer l.
+    bf16-exact, sel_bias f32 [E], gamma f32 [d]), W_r and sel_bias None for a dense layer; expert_bits:
+    iterable of (l, e, (wg, wu, wd) uint16 bit arrays); k_of(l) -> experts per token in layer l;
+    E_of(l) -> experts of layer l (default E; 1 for a dense FFN layer).
     """
     import numpy as np
 
@@ -168,11 +171,13 @@ def stack_from_bits(tables_bits, gamma0, layer_small, expert_bits, n_layers: int
     layers = []
     for l in range(n_layers):
         wr, sb, gm = layer_small(l)
-        layers.append(MoEWeights(torch.from_numpy(wr).to(device=device, dtype=torch.bfloat16),
-                                 torch.empty((E, f, d), dtype=torch.bfloat16, device=device),
-                                 torch.empty((E, f, d), dtype=torch.bfloat16, device=device),
-                                 torch.empty((E, d, f), dtype=torch.bfloat16, device=device),
-                                 torch.from_numpy(sb).to(device), None, torch.from_numpy(gm).to(device), k_of(l)))
+        El = E_of(l) if E_of is not None else E
+        layers.append(MoEWeights(None if wr is None else torch.from_numpy(wr).to(device=device, dtype=torch.bfloat16),
+                                 torch.empty((El, f, d), dtype=torch.bfloat16, device=device),
+                                 torch.empty((El, f, d), dtype=torch.bfloat16, device=device),
+                                 torch.empty((El, d, f), dtype=torch.bfloat16, device=device),
+                                 None if sb is None else torch.from_numpy(sb).to(device), None,
+                                 torch.from_numpy(gm).to(device), k_of(l)))
     for l, e, (wg, wu, wd) in expert_bits:
         layers[l].w_gate[e].copy_(bits_to_dev(wg))
         layers[l].w_up[e].copy_(bits_to_dev(wu))

@@ -168,16 +168,19 @@ def zmoe_rmsnorm(h: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6, out_dt
     return o
 
 
-def zmoe_route(x: torch.Tensor, w_router: torch.Tensor, k: int, logit_bias: Optional[torch.Tensor] = None,
+def zmoe_route(x: torch.Tensor, w_router: Optional[torch.Tensor], k: int, logit_bias: Optional[torch.Tensor] = None,
                sel_bias: Optional[torch.Tensor] = None, margin: bool = True, outs=None, stream=None):
-    """Returns (expert_idx int32 [T, k], gates f32 [T, k], margin f32 [T] or None)."""
+    """Returns (expert_idx int32 [T, k], gates f32 [T, k], margin f32 [T] or None).
+
+    w_router None means one expert without a router (a dense FFN layer): expert 0, gate 1."""
     _need(x, "x", None, 2)
-    _need(w_router, "w_router", x.dtype, 2)
+    if w_router is not None:
+        _need(w_router, "w_router", x.dtype, 2)
     for t, n in ((logit_bias, "logit_bias"), (sel_bias, "sel_bias")):
         if t is not None:
             _need(t, n, torch.float32, 1)
     T, d = x.shape
-    E = w_router.shape[0]
+    E = w_router.shape[0] if w_router is not None else 1
     if outs is None:
         idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
         g = torch.empty((T, k), dtype=torch.float32, device=x.device)
@@ -271,7 +274,7 @@ def zmoe_moe_layer_workspace_size(T: int, d: int, f: int, E: int, k: int, dtype:
     return int(lib().zmoe_moe_layer_workspace_size(T, d, f, E, k, _dtype_code(dtype)))
 
 
-def zmoe_moe_layer(w_router: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor, k: int,
+def zmoe_moe_layer(w_router: Optional[torch.Tensor], w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor, k: int,
                    x: Optional[torch.Tensor] = None, h: Optional[torch.Tensor] = None,
                    gamma: Optional[torch.Tensor] = None, eps: float = 1e-6,
                    logit_bias: Optional[torch.Tensor] = None, sel_bias: Optional[torch.Tensor] = None,
@@ -287,7 +290,7 @@ def zmoe_moe_layer(w_router: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Ten
         raise ValueError("zmoe_moe_layer: needs x, or h with gamma")
     T, d = src.shape
     E, f = w_gate.shape[0], w_gate.shape[1]
-    dt = w_router.dtype
+    dt = w_gate.dtype
     if x is not None:
         _need(x, "x", dt, 2)
     if h is not None:

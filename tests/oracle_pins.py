@@ -321,5 +321,34 @@ def pin_stack(decode_stack_step, embed_sum_rmsnorm, rmsnorm, moe_layer_bruteforc
     assert np.allclose(out0["h"], embed_sum_rmsnorm(ids, tables, gamma0, 1e-6), rtol=1e-15)
 
 
+def pin_stack_dense(decode_stack_step, embed_sum_rmsnorm, rmsnorm, moe_layer_bruteforce):
+    """A dense FFN layer (no router) in the stack is h <- h + SwiGLU(RMSNorm(h)), checked against a
+    torch composition, followed by a MoE layer checked by the per-token brute force."""
+    import torch
+    import torch.nn.functional as F
+    rng = np.random.default_rng(11)
+    N, V, d, f, E = 9, 6, 5, 4, 3
+    tables = rng.standard_normal((N, V, d))
+    gamma0 = 1 + 0.1 * rng.standard_normal(d)
+    ids = rng.integers(0, V, size=(2, N))
+    dense = (rng.standard_normal((f, d)), rng.standard_normal((f, d)), rng.standard_normal((d, f)))
+    moe = {e: (rng.standard_normal((f, d)), rng.standard_normal((f, d)), rng.standard_normal((d, f))) for e in range(E)}
+    g_dense, g_moe = 1 + 0.1 * rng.standard_normal(d), 1 + 0.1 * rng.standard_normal(d)
+    w_r, b = rng.standard_normal((E, d)), rng.standard_normal(E)
+    layers = [dict(w_router=None, sel_bias=None, gamma=g_dense, k=1, experts=lambda e: dense),
+              dict(w_router=w_r, sel_bias=b, gamma=g_moe, k=1, experts=lambda e: moe[e])]
+    out = decode_stack_step(ids, tables, gamma0, layers, 1e-6)
+    h = embed_sum_rmsnorm(ids, tables, gamma0, 1e-6)
+    t = torch.from_numpy(rmsnorm(h, g_dense, 1e-6))
+    wg, wu, wd = (torch.from_numpy(w) for w in dense)
+    h = h + F.linear(F.silu(F.linear(t, wg)) * F.linear(t, wu), wd).numpy()
+    xin = rmsnorm(h, g_moe, 1e-6)
+    _, _, y = moe_layer_bruteforce(xin, w_r, np.stack([moe[e][0] for e in range(E)]),
+                                   np.stack([moe[e][1] for e in range(E)]), np.stack([moe[e][2] for e in range(E)]),
+                                   1, sel_bias=b)
+    assert np.allclose(out["h"], h + y, rtol=1e-12, atol=1e-12)
+    assert (out["layers"][0]["expert_idx"] == 0).all() and (out["layers"][0]["gates"] == 1).all()
+
+
 def golden_path(name):
     return os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", name)

@@ -140,3 +140,28 @@ def test_fused_repeatable_bitwise():
     first = host(R.run(x, W)).copy()
     for _ in range(3):
         assert np.array_equal(host(R.run(x, W)), first)
+
+
+@pytest.mark.parametrize("T", [1, 40, 300])
+def test_dense_layer_without_router(T):
+    """E = 1 and no router: the decoder's dense FFN layers, h <- h + SwiGLU(RMSNorm(h) * gamma)
+    (fused below 64 tokens, the separate entry points above)."""
+    require_gpu()
+    L = make_moe_layer(T, 512, 512, 1, 1, seed=T, with_gamma=True, draw_x=False)
+    h = np.random.default_rng(T).standard_normal((T, 512)).astype(np.float32)
+    dt = torch.bfloat16
+    W = MoEWeights.from_host(L)
+    W.w_router = None
+    W.sel_bias = None
+    R = MoELayerRunner(T, 1, 512, 512, 1, dt)
+    hd = to_dev(h, torch.float32)
+    xn = torch.empty((T, 512), dtype=dt, device="cuda")
+    y = host(R.run(None, W, residual=hd, out=hd, gamma=to_dev(L.gamma, torch.float32), eps=EPS,
+                   x_norm=xn)).astype(np.float64)
+    torch.cuda.synchronize()
+    assert zmoe_get_device_errors() == 0
+    assert (host(R.idx) == 0).all() and (host(R.gates) == 1.0).all()
+    x = host(xn).astype(np.float64)
+    assert_close(x, oracle.rmsnorm(h.astype(np.float64), L.gamma.astype(np.float64), EPS), "bf16", "pre-norm")
+    want = oracle.swiglu_ffn(x, L.w_gate[0], L.w_up[0], L.w_down[0])
+    assert_close(y - h, want, "bf16", f"dense layer T={T}")

@@ -72,3 +72,11 @@ def test_route_exact_ties_lowest_index():
     assert ((sel == 1) | (sel == 3) | (sel == 4)).any(), "the tie must reach the top-2 somewhere"
     assert np.array_equal(idx, sel)
     assert np.allclose(g, gates, rtol=1e-5)
+
+
+def test_route_without_router_single_expert():
+    """E = 1 with no router (a dense FFN layer): expert 0, gate 1, margin +inf for every token."""
+    require_gpu()
+    x = torch.randn(37, 256, device="cuda").to(torch.bfloat16)
+    idx, g, mg = zmoe_route(x, None, 1)
+    assert (host(idx) == 0).all() and (host(g) == 1.0).all() and np.isinf(host(mg)).all()

@@ -1,5 +1,6 @@
 """The batch-1 decode stack (embedding sum + RMSNorm, 24 pre-norm MoE layers, top-2 in the last) on the
-GPU vs the oracle.
+GPU vs the oracle; and the decoder's full 28-layer FFN stack (3 dense layers, the 24 MoE layers, 1 dense
+layer), each layer one zmoe_moe_layer call.
 
 Full size: 24 layers x 16 experts of d_model 2048, d_ff 3072 (14.5 GB of bf16 weights), in the launch
 configuration the benchmark times (T = 1 per step).  Layer by layer the oracle is teacher-forced: it
@@ -32,9 +33,25 @@ def stack():
     return spec, st
 
 
+@pytest.fixture(scope="module")
+def stack28():
+    require_gpu()
+    spec = StackSpec(n_dense_front=3, n_dense_back=1)
+    st = stack_from_bits(bf16_bits(spec.tables()), spec.gamma0(), spec.layer_small, stack_expert_bits(spec),
+                         spec.total_layers, spec.E, spec.d, spec.f, spec.k_of, spec.eps, T=1, E_of=spec.E_of)
+    return spec, st
+
+
 def test_stack_teacher_forced_layers(stack):
-    spec, st = stack
-    codes = spec.codes(STEPS)
+    check_teacher_forced(*stack, STEPS)
+
+
+def test_full_ffn_stack_teacher_forced(stack28):
+    check_teacher_forced(*stack28, 1)
+
+
+def check_teacher_forced(spec, st, steps):
+    codes = spec.codes(steps)
     cache = {}
 
     def expert(l, e):
@@ -45,20 +62,24 @@ def test_stack_teacher_forced_layers(stack):
     st.record_inputs = True
     tables = spec.tables()
     exempt = 0
-    for s in range(STEPS):
+    for s in range(steps):
         ids = torch.from_numpy(codes[s:s + 1]).cuda()
         h_final = host(st.step(ids)).astype(np.float64)
         h0 = host(st.layer_h[0]).astype(np.float64)
         assert_close(h0, oracle.embed_sum_rmsnorm(codes[s:s + 1], tables, spec.gamma0(), spec.eps), "f32",
                      f"step {s} embedding")
         hs = [host(t).astype(np.float64) for t in st.layer_h] + [h_final]
-        for l in range(spec.n_layers):
+        for l in range(spec.total_layers):
             x = host(st.layer_inputs[l]).astype(np.float64)        # the GPU's bf16 layer input (exact)
             wr, sb, gm = spec.layer_small(l)
             k = spec.k_of(l)
             # the layer's pre-norm also matches the oracle on the GPU's residual stream
             assert_close(x, oracle.rmsnorm(hs[l], gm, spec.eps), "bf16", f"step {s} layer {l} rmsnorm")
-            sel, gates, margin, _ = oracle.route(x, wr, k, sb)
+            if wr is None:
+                # dense FFN layer: expert 0, gate 1
+                sel, gates, margin = np.zeros((1, 1), np.int64), np.ones((1, 1)), np.array([np.inf])
+            else:
+                sel, gates, margin, _ = oracle.route(x, wr, k, sb)
             gpu_idx = host(st.layer_idx[l])
             if margin[0] < MARGIN_EXEMPT:
                 exempt += 1
@@ -70,7 +91,7 @@ def test_stack_teacher_forced_layers(stack):
                 want += gates[0, i] * oracle.swiglu_ffn(x, wg, wu, wd)
             got = hs[l + 1] - hs[l]
             assert_close(got, want, "bf16", f"step {s} layer {l} output")
-    print(f"stack: {STEPS} steps x {spec.n_layers} layers teacher-forced; {exempt} low-margin layer routes exempt")
+    print(f"stack: {steps} steps x {spec.total_layers} layers teacher-forced; {exempt} low-margin layer routes exempt")
 
 
 def test_stack_free_running_report(stack):

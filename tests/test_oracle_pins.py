@@ -53,6 +53,11 @@ def test_pin_stack():
     P.pin_stack(oracle.decode_stack_step, oracle.embed_sum_rmsnorm, oracle.rmsnorm, oracle.moe_layer_bruteforce)
 
 
+def test_pin_stack_dense():
+    P.pin_stack_dense(oracle.decode_stack_step, oracle.embed_sum_rmsnorm, oracle.rmsnorm,
+                      oracle.moe_layer_bruteforce)
+
+
 def test_param_counts_match_published_totals():
     """8B total / 900M active (ZONOS2 Technical Report abstract) at d_model 2048, d_ff 3072."""
     c = oracle.param_counts()
@@ -181,6 +186,23 @@ def _stack_post_norm(ids, tables, gamma0, layers, eps):
     return dict(h=h, layers=[])
 
 
+def _stack_dense_no_residual(ids, tables, gamma0, layers, eps):
+    """Planted: a dense layer replaces the residual stream instead of adding to it."""
+    h = oracle.embed_sum_rmsnorm(np.atleast_2d(ids), tables, gamma0, eps)
+    records = []
+    for L in layers:
+        x = oracle.rmsnorm(h, L["gamma"], eps)
+        if L["w_router"] is None:
+            h = oracle.swiglu_ffn(x, *L["experts"](0))
+            records.append(dict(expert_idx=np.zeros((x.shape[0], 1), np.int64), gates=np.ones((x.shape[0], 1))))
+        else:
+            out = oracle.moe_layer(x, L["w_router"], None, None, None, L["k"], sel_bias=L["sel_bias"],
+                                   experts=L["experts"])
+            h = h + out["y"]
+            records.append(out)
+    return dict(h=h, layers=records)
+
+
 MUTANTS = {
     "shear reversed": lambda: P.pin_delay(_shear_reversed, oracle.delay_unshear, GOLDEN_DELAY),
     "shear too short": lambda: P.pin_delay(_shear_short, oracle.delay_unshear, GOLDEN_DELAY),
@@ -204,6 +226,8 @@ MUTANTS = {
                                                   oracle.moe_layer_bruteforce),
     "stack post-norm": lambda: P.pin_stack(_stack_post_norm, oracle.embed_sum_rmsnorm, oracle.rmsnorm,
                                            oracle.moe_layer_bruteforce),
+    "dense layer drops residual": lambda: P.pin_stack_dense(_stack_dense_no_residual, oracle.embed_sum_rmsnorm,
+                                                            oracle.rmsnorm, oracle.moe_layer_bruteforce),
 }
 
 
