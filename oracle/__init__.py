@@ -23,10 +23,11 @@ from .permute import permute
 from .ffn import silu, swiglu_ffn, grouped_swiglu
 from .layer import combine, moe_layer, moe_layer_bruteforce, decode_stack_step
 from .params import param_counts
+from .heads import head_logits, greedy, output_heads
 
 __all__ = [
     "delay_shear", "delay_unshear", "embed_sum", "rmsnorm", "embed_sum_rmsnorm",
     "router_logits", "softmax", "select_topk", "route", "permute", "silu", "swiglu_ffn",
     "grouped_swiglu", "combine", "moe_layer", "moe_layer_bruteforce", "decode_stack_step",
-    "param_counts",
+    "param_counts", "head_logits", "greedy", "output_heads",
 ]

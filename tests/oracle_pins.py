@@ -350,5 +350,44 @@ def pin_stack_dense(decode_stack_step, embed_sum_rmsnorm, rmsnorm, moe_layer_bru
     assert (out["layers"][0]["expert_idx"] == 0).all() and (out["layers"][0]["gates"] == 1).all()
 
 
+def pin_heads(head_logits, greedy, output_heads, rmsnorm):
+    """Heads: one-hot head rows pick coordinates of x (closed form); a brute-force loop; the greedy
+    choice on a hand-built example with an exact tie (lower id wins); the pre-norm is RMSNorm."""
+    rng = np.random.default_rng(3)
+    T, N, V, d = 3, 2, 5, 4
+    x = rng.standard_normal((T, d))
+    # one-hot rows: logits[t, n, v] = x[t, (n + v) % d]
+    W = np.zeros((N, V, d))
+    for n in range(N):
+        for v in range(V):
+            W[n, v, (n + v) % d] = 1.0
+    lg = head_logits(x, W)
+    for t in range(T):
+        for n in range(N):
+            for v in range(V):
+                assert lg[t, n, v] == x[t, (n + v) % d]
+    # brute force on random weights
+    W = rng.standard_normal((N, V, d))
+    lg = head_logits(x, W)
+    for t in range(T):
+        for n in range(N):
+            for v in range(V):
+                acc = 0.0
+                for c in range(d):
+                    acc += W[n, v, c] * x[t, c]
+                assert abs(lg[t, n, v] - acc) <= 1e-12
+    # greedy: ties go to the lower id; the maximum wins otherwise
+    ex = np.array([[[0.5, 2.0, -1.0, 2.0, 1.9]]])
+    assert greedy(ex).tolist() == [[1]]
+    assert greedy(-ex).tolist() == [[2]]
+    # with a gain the input is the RMSNorm of h; ids are the argmax of its logits
+    h = rng.standard_normal((T, d)) * 5.0
+    g = 1 + 0.1 * rng.standard_normal(d)
+    out = output_heads(h, W, g, 1e-6)
+    assert np.allclose(out["x"], rmsnorm(h, g, 1e-6), rtol=1e-15)
+    assert np.array_equal(out["ids"], np.argmax(head_logits(rmsnorm(h, g, 1e-6), W), axis=-1))
+    assert (out["margin"] >= 0).all()
+
+
 def golden_path(name):
     return os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", name)

@@ -53,6 +53,10 @@ def test_pin_stack():
     P.pin_stack(oracle.decode_stack_step, oracle.embed_sum_rmsnorm, oracle.rmsnorm, oracle.moe_layer_bruteforce)
 
 
+def test_pin_heads():
+    P.pin_heads(oracle.head_logits, oracle.greedy, oracle.output_heads, oracle.rmsnorm)
+
+
 def test_pin_stack_dense():
     P.pin_stack_dense(oracle.decode_stack_step, oracle.embed_sum_rmsnorm, oracle.rmsnorm,
                       oracle.moe_layer_bruteforce)
@@ -203,6 +207,18 @@ def _stack_dense_no_residual(ids, tables, gamma0, layers, eps):
     return dict(h=h, layers=records)
 
 
+def _greedy_ties_high(logits):
+    """Planted: ties go to the higher id."""
+    L = np.asarray(logits)
+    return (L.shape[-1] - 1 - np.argmax(L[..., ::-1], axis=-1)).astype(np.int64)
+
+
+def _head_logits_transposed(x, w):
+    """Planted: the head contracted over the wrong axis of W (rows and columns swapped)."""
+    w = np.asarray(w, np.float64)
+    return np.einsum("ncv,tc->tnv", w.reshape(w.shape[0], w.shape[2], w.shape[1]), np.asarray(x, np.float64))
+
+
 MUTANTS = {
     "shear reversed": lambda: P.pin_delay(_shear_reversed, oracle.delay_unshear, GOLDEN_DELAY),
     "shear too short": lambda: P.pin_delay(_shear_short, oracle.delay_unshear, GOLDEN_DELAY),
@@ -226,6 +242,10 @@ MUTANTS = {
                                                   oracle.moe_layer_bruteforce),
     "stack post-norm": lambda: P.pin_stack(_stack_post_norm, oracle.embed_sum_rmsnorm, oracle.rmsnorm,
                                            oracle.moe_layer_bruteforce),
+    "greedy ties to the higher id": lambda: P.pin_heads(oracle.head_logits, _greedy_ties_high, oracle.output_heads,
+                                                         oracle.rmsnorm),
+    "head contracted on the wrong axis": lambda: P.pin_heads(_head_logits_transposed, oracle.greedy,
+                                                              oracle.output_heads, oracle.rmsnorm),
     "dense layer drops residual": lambda: P.pin_stack_dense(_stack_dense_no_residual, oracle.embed_sum_rmsnorm,
                                                             oracle.rmsnorm, oracle.moe_layer_bruteforce),
 }
