@@ -245,6 +245,26 @@ ZMOE_API zmoe_status zmoe_moe_layer(const void* x, const float* h, const float* 
                                     float* gates, float* margin, void* x_norm, void* workspace, size_t ws_bytes,
                                     zmoe_stream_t stream);
 
+/* Bytes of workspace zmoe_output_heads needs (T tokens, N codebooks). */
+ZMOE_API size_t zmoe_output_heads_workspace_size(int T, int N);
+
+/*
+ * Output heads over the codebooks and the greedy next frame ([DIGEST] items 1 and 5: the decoder
+ * predicts the next frame Y[t+1, n] of the 9 delay-patterned DAC codebooks):
+ *   x = RMSNorm(h[t]) * gamma (gamma NULL: x = h[t]), rounded to `dtype`;
+ *   logits[t, n, v] = sum_c w_heads[n, v, c] x[c]   (fp32 accumulation, one bias-free head per codebook);
+ *   ids[t, n] = argmax_v logits[t, n, v], ties -> the lower id (-1, with a device error, only when
+ *   every logit of that (t, n) is NaN).
+ *   h: f32 [T, d]; gamma: f32 [d] or NULL; w_heads: [N, V, d] of `dtype`; ids: int32 [T, N];
+ *   logits: f32 [T, N, V] or NULL; x_out: [T, d] of `dtype` or NULL (the rounded input).
+ *   The weights are streamed once per 8 tokens.  d % 8 == 0, w_heads 16-byte aligned; workspace:
+ *   zmoe_output_heads_workspace_size() bytes.  The pages give no head formula: the final norm and
+ *   the bias-free linear heads are the plain pre-norm-transformer reading.
+ */
+ZMOE_API zmoe_status zmoe_output_heads(const float* h, const float* gamma, float eps, const void* w_heads,
+                                       zmoe_dtype dtype, int T, int N, int V, int d, int32_t* ids, float* logits,
+                                       void* x_out, void* workspace, size_t ws_bytes, zmoe_stream_t stream);
+
 /*
  * Reads and clears the device error counters of the current device.  Synchronises
  * `stream` (and the device) first.  *count = data errors (ids or indices out of range)

@@ -268,6 +268,14 @@ class StackSpec:
         wd = _normal(self._rng(*key, 2), (self.d, self.f), 1.0 / self.f, True)
         return wg, wu, wd
 
+    def heads(self) -> np.ndarray:
+        """Output heads [N, V, d], N(0, 1/d), bf16-exact (one bias-free linear per codebook)."""
+        return _normal(self._rng(6, 0), (self.n_codebooks, self.vocab_rows, self.d), 1.0 / self.d, True)
+
+    def gamma_out(self) -> np.ndarray:
+        """Gain of the final RMSNorm before the heads, N(1, 0.01)."""
+        return (1.0 + 0.1 * self._rng(6, 1).standard_normal(self.d, dtype=np.float32)).astype(np.float32)
+
     def codes(self, steps: int) -> np.ndarray:
         """One fresh frame of (already delay-sheared) ids per decode step: int32 [steps, N]."""
         return self._rng(3, 0).integers(0, CODEBOOK_SIZE, size=(steps, self.n_codebooks),

@@ -44,6 +44,8 @@ SIGNATURES = {
     "zmoe_grouped_swiglu": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _S, _P]),
     "zmoe_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "zmoe_moe_layer_workspace_size": (_S, [_I, _I, _I, _I, _I, _I]),
+    "zmoe_output_heads_workspace_size": (_S, [_I, _I]),
+    "zmoe_output_heads": (_I, [_P, _P, _F, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _S, _P]),
     "zmoe_moe_layer": (_I, [_P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                             _P, _S, _P]),
     "zmoe_get_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -306,6 +308,37 @@ def zmoe_moe_layer(w_router: Optional[torch.Tensor], w_gate: torch.Tensor, w_up:
                                 _ptr(outs.get("margin")), _ptr(outs.get("x_norm")), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(stream)), "zmoe_moe_layer")
     return y
+
+
+def zmoe_output_heads(h: torch.Tensor, w_heads: torch.Tensor, gamma: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                      want_logits: bool = False, want_x: bool = False, outs: Optional[dict] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """The codebook heads on the final hidden state h (f32 [T, d]) and the greedy next frame.
+
+    Returns dict(ids=int32 [T, N], logits=f32 [T, N, V] or None, x=[T, d] or None); ``outs`` may hold
+    preallocated tensors under the same names."""
+    _need(h, "h", torch.float32, 2)
+    _need(w_heads, "w_heads", None, 3)
+    T, d = h.shape
+    N, V = w_heads.shape[0], w_heads.shape[1]
+    outs = dict(outs or {})
+    ids = outs.get("ids")
+    if ids is None:
+        ids = torch.empty((T, N), dtype=torch.int32, device=h.device)
+    lg = outs.get("logits")
+    if lg is None and want_logits:
+        lg = torch.empty((T, N, V), dtype=torch.float32, device=h.device)
+    x = outs.get("x")
+    if x is None and want_x:
+        x = torch.empty((T, d), dtype=w_heads.dtype, device=h.device)
+    ws_bytes = int(lib().zmoe_output_heads_workspace_size(T, N))
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=h.device)
+    _check(lib().zmoe_output_heads(_ptr(h), _ptr(gamma), float(eps), _ptr(w_heads), _dtype_code(w_heads.dtype), T, N,
+                                   V, d, _ptr(ids), _ptr(lg), _ptr(x), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "zmoe_output_heads")
+    return dict(ids=ids, logits=lg, x=x)
 
 
 def zmoe_get_device_errors(stream=None) -> int:
