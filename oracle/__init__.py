@@ -24,10 +24,11 @@ from .ffn import silu, swiglu_ffn, grouped_swiglu
 from .layer import combine, moe_layer, moe_layer_bruteforce, decode_stack_step
 from .params import param_counts
 from .heads import head_logits, greedy, output_heads
+from .speaker import speaker_prefix
 
 __all__ = [
     "delay_shear", "delay_unshear", "embed_sum", "rmsnorm", "embed_sum_rmsnorm",
     "router_logits", "softmax", "select_topk", "route", "permute", "silu", "swiglu_ffn",
     "grouped_swiglu", "combine", "moe_layer", "moe_layer_bruteforce", "decode_stack_step",
-    "param_counts", "head_logits", "greedy", "output_heads",
+    "param_counts", "head_logits", "greedy", "output_heads", "speaker_prefix",
 ]

@@ -389,5 +389,22 @@ def pin_heads(head_logits, greedy, output_heads, rmsnorm):
     assert (out["margin"] >= 0).all()
 
 
+def pin_speaker(speaker_prefix):
+    """The prefix row is a textbook linear: a hand-worked 2 x 3 example, torch F.linear on random
+    non-square weights, and linearity in e."""
+    import torch
+    import torch.nn.functional as F
+    W = np.array([[1.0, 2.0, 3.0], [-1.0, 0.5, 0.0]])
+    assert speaker_prefix(np.array([1.0, 1.0, 2.0]), W, np.array([0.5, -0.5])).tolist() == [[9.5, -1.0]]
+    rng = np.random.default_rng(4)
+    W = rng.standard_normal((7, 11))
+    b = rng.standard_normal(7)
+    e = rng.standard_normal((3, 11))
+    ref = F.linear(torch.from_numpy(e), torch.from_numpy(W), torch.from_numpy(b)).numpy()
+    assert np.allclose(speaker_prefix(e, W, b), ref, rtol=1e-12, atol=1e-12)
+    e2 = rng.standard_normal((3, 11))
+    assert np.allclose(speaker_prefix(e + 2 * e2, W), speaker_prefix(e, W) + 2 * speaker_prefix(e2, W))
+
+
 def golden_path(name):
     return os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", name)

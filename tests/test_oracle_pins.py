@@ -53,6 +53,10 @@ def test_pin_stack():
     P.pin_stack(oracle.decode_stack_step, oracle.embed_sum_rmsnorm, oracle.rmsnorm, oracle.moe_layer_bruteforce)
 
 
+def test_pin_speaker():
+    P.pin_speaker(oracle.speaker_prefix)
+
+
 def test_pin_heads():
     P.pin_heads(oracle.head_logits, oracle.greedy, oracle.output_heads, oracle.rmsnorm)
 
@@ -219,6 +223,14 @@ def _head_logits_transposed(x, w):
     return np.einsum("ncv,tc->tnv", w.reshape(w.shape[0], w.shape[2], w.shape[1]), np.asarray(x, np.float64))
 
 
+def _speaker_transposed(e, w, b=None):
+    """Planted: the projection applied with W's axes swapped."""
+    e = np.atleast_2d(np.asarray(e, np.float64))
+    w = np.asarray(w, np.float64)
+    h = e @ w.reshape(w.shape[1], w.shape[0])
+    return h + (np.asarray(b, np.float64) if b is not None else 0.0)
+
+
 MUTANTS = {
     "shear reversed": lambda: P.pin_delay(_shear_reversed, oracle.delay_unshear, GOLDEN_DELAY),
     "shear too short": lambda: P.pin_delay(_shear_short, oracle.delay_unshear, GOLDEN_DELAY),
@@ -246,6 +258,7 @@ MUTANTS = {
                                                          oracle.rmsnorm),
     "head contracted on the wrong axis": lambda: P.pin_heads(_head_logits_transposed, oracle.greedy,
                                                               oracle.output_heads, oracle.rmsnorm),
+    "speaker projection transposed": lambda: P.pin_speaker(_speaker_transposed),
     "dense layer drops residual": lambda: P.pin_stack_dense(_stack_dense_no_residual, oracle.embed_sum_rmsnorm,
                                                             oracle.rmsnorm, oracle.moe_layer_bruteforce),
 }
