@@ -70,9 +70,9 @@ WORKLOADS = {
     4: "final MoE layer: T=16384, d_model=2048, d_ff=3072, E=16, top-2, Zipf(1.2) logit skew, bf16",
     5: "batch-1 decode stack: 9-codebook embedding sum + RMSNorm, 24 pre-norm MoE layers (d_model=2048, "
        "d_ff=3072, E=16, top-1, top-2 in the last), attention omitted, bf16, one token per step",
-    6: "batch-1 full decoder FFN stack: embedding sum + RMSNorm, 3 dense SwiGLU layers, the 24 MoE layers "
-       "(E=16, top-1, top-2 in the last), 1 dense layer; d_model=2048, d_ff=3072, pre-norm residual, "
-       "attention omitted, bf16, one token per step",
+    6: "batch-1 full decoder FFN step: embedding sum + RMSNorm, 3 dense SwiGLU layers, the 24 MoE layers "
+       "(E=16, top-1, top-2 in the last), 1 dense layer, final RMSNorm + 9 codebook heads (1025 x 2048) with "
+       "greedy next frame; d_model=2048, d_ff=3072, pre-norm residual, attention omitted, bf16, one token per step",
 }
 
 
@@ -263,10 +263,17 @@ def run_reference_stack(args):
     tables, g0 = spec.tables(), spec.gamma0()
     n = max(1, min(args.steps, 3))
     codes = spec.codes(n + 1)
-    oracle.decode_stack_step(codes[n:n + 1], tables, g0, layers, spec.eps)      # warm-up: draws experts
+    heads = (spec.heads(), spec.gamma_out()) if args.config == 6 else None
+
+    def one(i):
+        ref = oracle.decode_stack_step(codes[i:i + 1], tables, g0, layers, spec.eps)
+        if heads is not None:
+            oracle.output_heads(ref["h"], heads[0], heads[1], spec.eps)
+
+    one(n)      # warm-up: draws experts
     t0 = time.perf_counter()
     for i in range(n):
-        oracle.decode_stack_step(codes[i:i + 1], tables, g0, layers, spec.eps)
+        one(i)
     el = time.perf_counter() - t0
     v = n / el
     sample = (f"oracle.decode_stack_step (numpy float64), {n} token(s) through the {spec.total_layers}-layer stack "
@@ -308,8 +315,11 @@ def run_stack(args):
     from sparse_moe_decoder_b200.layer import stack_from_bits
 
     spec = StackSpec() if args.config == 5 else StackSpec(n_dense_front=3, n_dense_back=1)
+    full = args.config == 6   # the full step: 28 FFN layers, then the codebook heads and the next frame
     st = stack_from_bits(bf16_bits(spec.tables()), spec.gamma0(), spec.layer_small, stack_expert_bits(spec),
-                         spec.total_layers, spec.E, spec.d, spec.f, spec.k_of, spec.eps, T=1, E_of=spec.E_of)
+                         spec.total_layers, spec.E, spec.d, spec.f, spec.k_of, spec.eps, T=1, E_of=spec.E_of,
+                         heads_bits=bf16_bits(spec.heads()) if full else None,
+                         gamma_out=spec.gamma_out() if full else None)
     n = args.warmup + args.steps
     codes = spec.codes(n + 1)
     if rank > 0:
@@ -325,6 +335,8 @@ def run_stack(args):
     st.record_inputs = False
     per_expert = 3 * spec.f * spec.d * 2
     alg_bytes = touched * per_expert + spec.n_layers * spec.E * spec.d * 2 + spec.n_codebooks * spec.d * 2
+    if full:
+        alg_bytes += spec.n_codebooks * spec.vocab_rows * spec.d * 2     # the heads, streamed once per step
 
     graph = None
     try:
@@ -395,7 +407,9 @@ def run_stack(args):
         import oracle
         t0 = time.perf_counter()
         layers = oracle_stack_layers(spec, spec.expert)
-        oracle.decode_stack_step(codes[:1], spec.tables(), spec.gamma0(), layers, spec.eps)
+        ref = oracle.decode_stack_step(codes[:1], spec.tables(), spec.gamma0(), layers, spec.eps)
+        if full:
+            oracle.output_heads(ref["h"], spec.heads(), spec.gamma_out(), spec.eps)
         el = time.perf_counter() - t0
         cpu = {"value": 1.0 / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"oracle.decode_stack_step (numpy float64) on one token through all {spec.total_layers} layers, "
@@ -420,7 +434,7 @@ def run_stack(args):
             "cpu_baseline": cpu,
             "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": spec.n_codebooks * 4, "d2h_bytes_per_step": spec.d * 4},
-            "gpu_launches": (1 + spec.total_layers) * args.steps,
+            "gpu_launches": (1 + spec.total_layers + (1 if full else 0)) * args.steps,
             "clocks": clk.summary(),
             "device_errors": dev_errors,
         }

@@ -266,6 +266,16 @@ ZMOE_API zmoe_status zmoe_output_heads(const float* h, const float* gamma, float
                                        void* x_out, void* workspace, size_t ws_bytes, zmoe_stream_t stream);
 
 /*
+ * Speaker-embedding prefix row ([DIGEST] item 3: the LDA-reduced speaker embedding is projected to
+ * the model width and placed at position 0 of the decoder input):
+ *   out[b] = W_spk e[b] + b_spk    (fp32 accumulation)
+ *   e: f32 [B, n_in] (n_in = 1024 in ZONOS2); w_spk: [d, n_in] of `dtype`; b_spk: f32 [d] or NULL;
+ *   out: f32 [B, d].  n_in % 8 == 0, w_spk 16-byte aligned.
+ */
+ZMOE_API zmoe_status zmoe_speaker_prefix(const float* e, const void* w_spk, zmoe_dtype dtype, const float* b_spk,
+                                         int B, int d, int n_in, float* out, zmoe_stream_t stream);
+
+/*
  * Reads and clears the device error counters of the current device.  Synchronises
  * `stream` (and the device) first.  *count = data errors (ids or indices out of range)
  * plus bounded device-side waits that gave up, since the last read.  Returns

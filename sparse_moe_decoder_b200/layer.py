@@ -117,10 +117,11 @@ class MoELayerRunner:
 
 
 class DecodeStack:
-    """Embedding sum + RMSNorm, then L pre-norm residual MoE layers, for T tokens per step."""
+    """Embedding sum + RMSNorm, then L pre-norm residual MoE layers, for T tokens per step; with head
+    weights, also the codebook heads and the greedy next frame (``next_ids``)."""
 
     def __init__(self, tables: torch.Tensor, gamma0: torch.Tensor, layers: List[MoEWeights], eps: float = 1e-6,
-                 T: int = 1):
+                 T: int = 1, w_heads: Optional[torch.Tensor] = None, gamma_out: Optional[torch.Tensor] = None):
         self.tables, self.gamma0, self.layers, self.eps, self.T = tables, gamma0, layers, eps, T
         L0 = layers[0]
         dev = tables.device
@@ -129,6 +130,11 @@ class DecodeStack:
         self.ids = torch.empty((T, tables.shape[0]), dtype=torch.int32, device=dev)
         self.h = torch.empty((T, L0.d), dtype=torch.float32, device=dev)
         self.x = torch.empty((T, L0.d), dtype=L0.dtype, device=dev)
+        self.w_heads, self.gamma_out = w_heads, gamma_out
+        self.next_ids = torch.empty((T, tables.shape[0]), dtype=torch.int32, device=dev)
+        self.head_x = torch.empty((T, L0.d), dtype=L0.dtype, device=dev)
+        self.head_ws = torch.empty(max(int(Z.lib().zmoe_output_heads_workspace_size(T, tables.shape[0])), 16),
+                                   dtype=torch.uint8, device=dev) if w_heads is not None else None
         self.record_inputs = False
         self.layer_inputs: List[torch.Tensor] = []
         self.layer_h: List[torch.Tensor] = []
@@ -151,17 +157,23 @@ class DecodeStack:
             if self.record_inputs:
                 self.layer_inputs.append(self.x.clone())
                 self.layer_idx.append(R.idx.clone())
+        if self.w_heads is not None:
+            outs = dict(ids=self.next_ids, x=self.head_x) if self.record_inputs else dict(ids=self.next_ids)
+            Z.zmoe_output_heads(self.h, self.w_heads, self.gamma_out, self.eps, outs=outs, workspace=self.head_ws,
+                                stream=stream)
         return self.h
 
 
 def stack_from_bits(tables_bits, gamma0, layer_small, expert_bits, n_layers: int, E: int, d: int, f: int,
-                    k_of, eps: float = 1e-6, T: int = 1, device="cuda", E_of=None) -> DecodeStack:
+                    k_of, eps: float = 1e-6, T: int = 1, device="cuda", E_of=None, heads_bits=None,
+                    gamma_out=None) -> DecodeStack:
     """Builds a DecodeStack on the device from host arrays.
 
     tables_bits: uint16 [N, V, d] bf16 bit patterns; gamma0: f32 [d]; layer_small(l) -> (W_r f32 [E, d]
     bf16-exact, sel_bias f32 [E], gamma f32 [d]), W_r and sel_bias None for a dense layer; expert_bits:
     iterable of (l, e, (wg, wu, wd) uint16 bit arrays); k_of(l) -> experts per token in layer l;
-    E_of(l) -> experts of layer l (default E; 1 for a dense FFN layer).
+    E_of(l) -> experts of layer l (default E; 1 for a dense FFN layer); heads_bits: uint16 [N, V, d] bf16
+    bit patterns of the codebook heads (with gamma_out f32 [d], the final norm's gain), or None.
     """
     import numpy as np
 
@@ -183,4 +195,6 @@ def stack_from_bits(tables_bits, gamma0, layer_small, expert_bits, n_layers: int
         layers[l].w_up[e].copy_(bits_to_dev(wu))
         layers[l].w_down[e].copy_(bits_to_dev(wd))
     tables = bits_to_dev(tables_bits)
-    return DecodeStack(tables, torch.from_numpy(gamma0).to(device), layers, eps, T)
+    heads = bits_to_dev(heads_bits) if heads_bits is not None else None
+    g_out = torch.from_numpy(gamma_out).to(device) if gamma_out is not None else None
+    return DecodeStack(tables, torch.from_numpy(gamma0).to(device), layers, eps, T, heads, g_out)

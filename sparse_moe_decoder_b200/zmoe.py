@@ -45,6 +45,7 @@ SIGNATURES = {
     "zmoe_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "zmoe_moe_layer_workspace_size": (_S, [_I, _I, _I, _I, _I, _I]),
     "zmoe_output_heads_workspace_size": (_S, [_I, _I]),
+    "zmoe_speaker_prefix": (_I, [_P, _P, _I, _P, _I, _I, _I, _P, _P]),
     "zmoe_output_heads": (_I, [_P, _P, _F, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _S, _P]),
     "zmoe_moe_layer": (_I, [_P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                             _P, _S, _P]),
@@ -339,6 +340,21 @@ def zmoe_output_heads(h: torch.Tensor, w_heads: torch.Tensor, gamma: Optional[to
                                    workspace.numel() * workspace.element_size(), _stream(stream)),
            "zmoe_output_heads")
     return dict(ids=ids, logits=lg, x=x)
+
+
+def zmoe_speaker_prefix(e: torch.Tensor, w_spk: torch.Tensor, b_spk: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """h_spk = W_spk e + b_spk: e f32 [B, n_in], W_spk [d, n_in] -> f32 [B, d]."""
+    _need(e, "e", torch.float32, 2)
+    _need(w_spk, "w_spk", None, 2)
+    if b_spk is not None:
+        _need(b_spk, "b_spk", torch.float32, 1)
+    B, n_in = e.shape
+    d = w_spk.shape[0]
+    y = out if out is not None else torch.empty((B, d), dtype=torch.float32, device=e.device)
+    _check(lib().zmoe_speaker_prefix(_ptr(e), _ptr(w_spk), _dtype_code(w_spk.dtype), _ptr(b_spk), B, d, n_in, _ptr(y),
+                                     _stream(stream)), "zmoe_speaker_prefix")
+    return y
 
 
 def zmoe_get_device_errors(stream=None) -> int:

@@ -38,7 +38,8 @@ def stack28():
     require_gpu()
     spec = StackSpec(n_dense_front=3, n_dense_back=1)
     st = stack_from_bits(bf16_bits(spec.tables()), spec.gamma0(), spec.layer_small, stack_expert_bits(spec),
-                         spec.total_layers, spec.E, spec.d, spec.f, spec.k_of, spec.eps, T=1, E_of=spec.E_of)
+                         spec.total_layers, spec.E, spec.d, spec.f, spec.k_of, spec.eps, T=1, E_of=spec.E_of,
+                         heads_bits=bf16_bits(spec.heads()), gamma_out=spec.gamma_out())
     return spec, st
 
 
@@ -47,7 +48,16 @@ def test_stack_teacher_forced_layers(stack):
 
 
 def test_full_ffn_stack_teacher_forced(stack28):
-    check_teacher_forced(*stack28, 1)
+    """Every layer teacher-forced, then the heads on the final residual stream: the next frame's ids
+    bit-exact except where the oracle's top-two logit margin is below 1e-4."""
+    spec, st = stack28
+    check_teacher_forced(spec, st, 1)
+    h = host(st.h).astype(np.float64)
+    x = host(st.head_x).astype(np.float64)
+    assert_close(x, oracle.rmsnorm(h, spec.gamma_out(), spec.eps), "bf16", "final norm")
+    ref = oracle.output_heads(h, spec.heads(), spec.gamma_out(), spec.eps, x_rounded=x)
+    ok = ref["margin"] >= MARGIN_EXEMPT
+    assert np.array_equal(host(st.next_ids)[ok], ref["ids"][ok])
 
 
 def check_teacher_forced(spec, st, steps):
