@@ -61,6 +61,14 @@ NULL = None
     lambda L: L.zmoe_grouped_swiglu(NULL, NULL, 4, NULL, NULL, NULL, 1, 16, 64, 64, NULL, NULL, NULL, 0, NULL),
     lambda L: L.zmoe_combine(NULL, NULL, NULL, NULL, 4, 64, 3, NULL, NULL),    # k = 3
     lambda L: L.zmoe_combine(NULL, NULL, NULL, NULL, 4, 6, 1, NULL, NULL),     # d % 4
+    lambda L: L.zmoe_moe_layer(NULL, NULL, NULL, 1e-6, NULL, NULL, NULL, NULL, NULL, NULL, 1, 4, 256, 256, 16, 3,
+                               NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL),     # k = 3
+    lambda L: L.zmoe_moe_layer(NULL, NULL, NULL, 1e-6, NULL, NULL, NULL, NULL, NULL, NULL, 1, 4, 256, 256, 16, 1,
+                               NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL),     # no router with E = 16
+    lambda L: L.zmoe_output_heads(NULL, NULL, 1e-6, NULL, 1, 2, 9, 1025, 12, NULL, NULL, NULL, NULL, 0, NULL),  # d % 8
+    lambda L: L.zmoe_output_heads(NULL, NULL, 1e-6, NULL, 1, 2, 9, 1025, 16, NULL, NULL, NULL, NULL, 0, NULL),  # NULL
+    lambda L: L.zmoe_speaker_prefix(NULL, NULL, 1, NULL, 2, 2048, 1020, NULL, NULL),   # n_in % 8
+    lambda L: L.zmoe_speaker_prefix(NULL, NULL, 1, NULL, 2, 2048, 1024, NULL, NULL),   # NULL
 ])
 def test_bad_arguments_rejected_on_host(L, call):
     assert call(L) == 1   # ZMOE_ERR_INVALID_ARG, nothing launched
@@ -81,6 +89,14 @@ def test_empty_problems_are_no_ops(L):
     assert L.zmoe_route(NULL, NULL, 1, NULL, NULL, 0, 64, 16, 1, NULL, NULL, NULL, NULL) == 0
     assert L.zmoe_combine(NULL, NULL, NULL, NULL, 0, 64, 1, NULL, NULL) == 0
     assert L.zmoe_delay_shear(NULL, NULL, 0, 5, 9, 1024, NULL) == 0
+
+
+def test_empty_new_entry_points_are_no_ops(L):
+    assert L.zmoe_moe_layer(NULL, NULL, NULL, 1e-6, NULL, NULL, NULL, NULL, NULL, NULL, 1, 0, 256, 256, 16, 1,
+                            NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL) == 0
+    assert L.zmoe_output_heads(NULL, NULL, 1e-6, NULL, 1, 0, 9, 1025, 2048, NULL, NULL, NULL, NULL, 0, NULL) == 0
+    assert L.zmoe_speaker_prefix(NULL, NULL, 1, NULL, 0, 2048, 1024, NULL, NULL) == 0
+    assert L.zmoe_output_heads_workspace_size(0, 9) >= 0 and L.zmoe_output_heads_workspace_size(4, 9) >= 4 * 9 * 8
 
 
 def test_workspace_queries(L):
