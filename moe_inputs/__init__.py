@@ -66,6 +66,34 @@ def round_to_bf16(a: np.ndarray, inplace: bool = False) -> np.ndarray:
     return a
 
 
+def quantize_e4m3_rows(w: np.ndarray):
+    """Weights stored as fp8: per output row (last axis = the contraction), scale = max|w| / 448 and
+    codes = the E4M3 (bias 7, no infinities, largest finite 448) value nearest w / scale, ties to even.
+
+    Returns (codes uint8 of w's shape, scales float32 of w.shape[:-1]).  This is the storage format the
+    fp8 path reads (a checkpoint would hold it); both the GPU and the oracle consume these arrays.
+    """
+    w = np.asarray(w, np.float32)
+    amax = np.max(np.abs(w), axis=-1)
+    scales = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    v = (w / scales[..., None]).astype(np.float64)
+    a = np.abs(v)
+    # binade of each value (subnormals share the lowest normal binade's spacing, 2^-9)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.clip(e, -6, 8)
+    ulp = np.exp2(e - 3)
+    q = np.round(a / ulp) * ulp                 # numpy rounds half to even
+    q = np.minimum(q, 448.0)
+    # encode: exponent field and 3 mantissa bits (subnormals: exponent field 0)
+    eq = np.floor(np.log2(np.where(q > 0, q, 1.0)))
+    normal = (q >= 2.0 ** -6)
+    efield = np.where(normal, eq + 7, 0).astype(np.int64)
+    mant = np.where(normal, np.round((q / np.exp2(eq) - 1.0) * 8), np.round(q / 2.0 ** -9)).astype(np.int64)
+    codes = ((efield << 3) | mant) & 0x7F
+    codes = np.where(q == 0, 0, codes) | np.where(v < 0, 0x80, 0)
+    return codes.astype(np.uint8), scales
+
+
 def bf16_bits(a: np.ndarray) -> np.ndarray:
     """The bf16 bit patterns (uint16) of a float32 array already rounded to bf16."""
     a = np.ascontiguousarray(a, dtype=np.float32)

@@ -406,5 +406,37 @@ def pin_speaker(speaker_prefix):
     assert np.allclose(speaker_prefix(e + 2 * e2, W), speaker_prefix(e, W) + 2 * speaker_prefix(e2, W))
 
 
+def pin_fp8(e4m3_decode, dequantize_rows, moe_layer_fp8):
+    """E4M3 decoding: closed forms of the format's corner codes and all 256 codes against torch's
+    float8_e4m3fn; a row-scaled 1-expert fp8 layer equals the dense SwiGLU (torch) on w = code * scale."""
+    import torch
+    import torch.nn.functional as F
+    assert e4m3_decode(np.array([0x7E]))[0] == 448.0          # largest finite: 2^8 * 1.75
+    assert e4m3_decode(np.array([0x01]))[0] == 2.0 ** -9      # smallest subnormal
+    assert e4m3_decode(np.array([0x08]))[0] == 2.0 ** -6      # smallest normal
+    assert e4m3_decode(np.array([0x38]))[0] == 1.0
+    assert e4m3_decode(np.array([0xC0]))[0] == -2.0
+    assert np.isnan(e4m3_decode(np.array([0x7F, 0xFF]))).all()
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    got = e4m3_decode(codes)
+    fin = ~np.isnan(ref)
+    assert np.array_equal(np.isnan(got), ~fin) and np.array_equal(got[fin], ref[fin])
+    rng = np.random.default_rng(8)
+    d, f, T = 16, 12, 5
+    qg, qu, qd = (rng.integers(0, 0x7F, size=sh).astype(np.uint8) | (rng.integers(0, 2, size=sh) << 7).astype(np.uint8)
+                  for sh in ((1, f, d), (1, f, d), (1, d, f)))
+    sg, su, sd = rng.random((1, f)) + 0.01, rng.random((1, f)) + 0.01, rng.random((1, d)) + 0.01
+    x = rng.standard_normal((T, d))
+    out = moe_layer_fp8(x, rng.standard_normal((1, d)), qg, sg, qu, su, qd, sd, 1)
+    tg = torch.from_numpy(qg[0]).view(torch.float8_e4m3fn).double() * torch.from_numpy(sg[0])[:, None]
+    tu = torch.from_numpy(qu[0]).view(torch.float8_e4m3fn).double() * torch.from_numpy(su[0])[:, None]
+    td = torch.from_numpy(qd[0]).view(torch.float8_e4m3fn).double() * torch.from_numpy(sd[0])[:, None]
+    tx = torch.from_numpy(x)
+    ref = F.linear(F.silu(F.linear(tx, tg)) * F.linear(tx, tu), td).numpy()
+    assert np.allclose(out["y"], ref, rtol=1e-12, atol=1e-12)
+    assert np.array_equal(dequantize_rows(qg, sg), e4m3_decode(qg) * sg[..., None])
+
+
 def golden_path(name):
     return os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", name)

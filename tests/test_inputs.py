@@ -27,3 +27,18 @@ def test_moe_layers_unchanged_by_dense_layers():
     # the dense layers have weights of their own
     assert not np.array_equal(full.expert(0, 0)[0], full.expert(27, 0)[0])
     assert not np.array_equal(full.expert(0, 0)[0], base.expert(0, 0)[0])
+
+
+def test_e4m3_row_quantizer_matches_torch_and_bounds_the_error():
+    import torch
+    from moe_inputs import quantize_e4m3_rows
+    w = np.random.default_rng(1).standard_normal((4, 33, 50)).astype(np.float32)
+    w[0, 0] = 0.0                                     # an all-zero row: scale 1, codes 0
+    q, s = quantize_e4m3_rows(w)
+    assert q.dtype == np.uint8 and s.shape == (4, 33) and s[0, 0] == 1.0 and not q[0, 0].any()
+    tq = (torch.from_numpy(w) / torch.from_numpy(s)[..., None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(q, tq)
+    deq = torch.from_numpy(q).view(torch.float8_e4m3fn).double().numpy() * s[..., None]
+    # half a unit in the last place of the code's binade (3 mantissa bits), times the row scale
+    assert (np.abs(deq - w) <= np.abs(w) * 2.0 ** -4 + s[..., None] * 2.0 ** -10 + 1e-12).all()
+    assert np.allclose(np.max(np.abs(deq), axis=-1)[s != 1.0], np.max(np.abs(w), axis=-1)[s != 1.0], rtol=1e-6)

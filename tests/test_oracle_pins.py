@@ -53,6 +53,10 @@ def test_pin_stack():
     P.pin_stack(oracle.decode_stack_step, oracle.embed_sum_rmsnorm, oracle.rmsnorm, oracle.moe_layer_bruteforce)
 
 
+def test_pin_fp8():
+    P.pin_fp8(oracle.e4m3_decode, oracle.dequantize_rows, oracle.moe_layer_fp8)
+
+
 def test_pin_speaker():
     P.pin_speaker(oracle.speaker_prefix)
 
@@ -231,6 +235,20 @@ def _speaker_transposed(e, w, b=None):
     return h + (np.asarray(b, np.float64) if b is not None else 0.0)
 
 
+def _e4m3_decode_bias8(codes):
+    """Planted: exponent bias 8 instead of 7."""
+    return oracle.e4m3_decode(codes) / 2.0
+
+
+def _moe_fp8_scale_per_column(x, w_router, q_gate, s_gate, q_up, s_up, q_down, s_down, k, **kw):
+    """Planted: the down projection's scales applied along the contraction (its first f scales) instead
+    of along the output rows."""
+    deq = lambda q, s: oracle.e4m3_decode(q) * np.asarray(s)[..., None]
+    f = q_down.shape[2]
+    wd = oracle.e4m3_decode(q_down) * np.resize(np.asarray(s_down), (q_down.shape[0], 1, f))
+    return oracle.moe_layer(x, w_router, deq(q_gate, s_gate), deq(q_up, s_up), wd, k, **kw)
+
+
 MUTANTS = {
     "shear reversed": lambda: P.pin_delay(_shear_reversed, oracle.delay_unshear, GOLDEN_DELAY),
     "shear too short": lambda: P.pin_delay(_shear_short, oracle.delay_unshear, GOLDEN_DELAY),
@@ -258,6 +276,9 @@ MUTANTS = {
                                                          oracle.rmsnorm),
     "head contracted on the wrong axis": lambda: P.pin_heads(_head_logits_transposed, oracle.greedy,
                                                               oracle.output_heads, oracle.rmsnorm),
+    "e4m3 exponent bias 8": lambda: P.pin_fp8(_e4m3_decode_bias8, oracle.dequantize_rows, oracle.moe_layer_fp8),
+    "fp8 down scales per column": lambda: P.pin_fp8(oracle.e4m3_decode, oracle.dequantize_rows,
+                                                    _moe_fp8_scale_per_column),
     "speaker projection transposed": lambda: P.pin_speaker(_speaker_transposed),
     "dense layer drops residual": lambda: P.pin_stack_dense(_stack_dense_no_residual, oracle.embed_sum_rmsnorm,
                                                             oracle.rmsnorm, oracle.moe_layer_bruteforce),
