@@ -42,7 +42,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4, 5, 6])
+    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4, 5, 6, 7])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle timing leg")
@@ -64,6 +64,8 @@ def load_peaks():
 
 
 WORKLOADS = {
+    7: "decode step with fp8 expert weights: one MoE layer, T=64, d_model=2048, d_ff=3072, E=16, top-1; expert "
+       "weights E4M3 with one fp32 scale per row, bf16 router, f16 tensor-core operands, fp32 accumulate",
     2: "decode step: one MoE layer, T=64 tokens (64 streams x 1 position), d_model=2048, d_ff=3072, E=16, top-1, "
        "bf16 weights/activations, fp32 accumulate",
     3: "prefill MoE layer: T=16384 (8 x 2048), d_model=2048, d_ff=3072, E=16, top-1, b~N(0,0.5), bf16",
@@ -183,14 +185,21 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
-    if args.config >= 5:
+    if args.config in (5, 6):
         return run_reference_stack(args)
     from moe_inputs import make_config
-    L = make_config(args.config)
+    L = make_config(2 if args.config == 7 else args.config)
+    if args.config == 7:
+        from moe_inputs import quantize_e4m3_rows
+        Q = [quantize_e4m3_rows(w) for w in (L.w_gate, L.w_up, L.w_down)]
 
     def one(lo, n):
         idx = (np.arange(n) + lo) % L.T
-        oracle.moe_layer(L.x[idx], L.w_router, L.w_gate, L.w_up, L.w_down, L.k, L.sel_bias, L.logit_bias)
+        if args.config == 7:
+            oracle.moe_layer_fp8(L.x[idx], L.w_router, Q[0][0], Q[0][1], Q[1][0], Q[1][1], Q[2][0], Q[2][1], L.k,
+                                 sel_bias=L.sel_bias)
+        else:
+            oracle.moe_layer(L.x[idx], L.w_router, L.w_gate, L.w_up, L.w_down, L.k, L.sel_bias, L.logit_bias)
 
     t0 = time.perf_counter()
     one(0, min(L.T, 64))                                  # calibration on up to 64 tokens
@@ -445,10 +454,132 @@ def run_stack(args):
     return 0
 
 
+def run_fp8(args):
+    """Workload 7: the decode step (configuration 2's tokens and weights) with the expert weights stored
+    as E4M3 codes + row scales, one zmoe_moe_layer_fp8 call per step."""
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+    from moe_inputs import make_config, quantize_e4m3_rows
+    from sparse_moe_decoder_b200 import zmoe_get_device_errors, zmoe_moe_layer_fp8
+    L = make_config(2)
+    if rank > 0:
+        from moe_inputs import round_to_bf16
+        L.x = round_to_bf16(np.random.default_rng(1000 + rank).standard_normal(L.x.shape, dtype=np.float32))
+    Q = [quantize_e4m3_rows(w) for w in (L.w_gate, L.w_up, L.w_down)]
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    n_copies = args.weight_copies if args.weight_copies > 0 else 8     # 8 x 302 MB of codes > L2
+    copies = [[dev(q).clone() for q, _ in Q] for _ in range(n_copies)]
+    scales = [dev(sc) for _, sc in Q]
+    w_r = torch.from_numpy(L.w_router).cuda().to(torch.bfloat16)
+    sb = dev(L.sel_bias)
+    x = torch.from_numpy(L.x).cuda().to(torch.bfloat16)
+    T = L.T
+    idx = torch.empty((T, 1), dtype=torch.int32, device="cuda")
+    y = torch.empty((T, L.d), dtype=torch.float32, device="cuda")
+    ws = torch.empty(int(__import__("sparse_moe_decoder_b200").zmoe.lib().zmoe_moe_layer_fp8_workspace_size(
+        T, L.d, L.f, L.E, 1)), dtype=torch.uint8, device="cuda")
+
+    def step(i, xin=None):
+        c = copies[i % n_copies]
+        return zmoe_moe_layer_fp8(w_r, c[0], scales[0], c[1], scales[1], c[2], scales[2], 1, x=x if xin is None else xin,
+                                  sel_bias=sb, out=y, outs=dict(expert_idx=idx), workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    touched = int(torch.unique(idx).numel())
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step(i)
+            ev[i][1].record(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    elapsed = e0.elapsed_time(e1)
+    k_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if world > 1:
+        t = torch.tensor([elapsed, k_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed, k_ms = float(t[0]), float(t[1])
+    value = T * world * args.steps / (elapsed / 1e3)
+    # e2e from pinned host memory
+    xh = torch.from_numpy(L.x).to(torch.bfloat16).pin_memory()
+    yh = torch.empty((T, L.d), dtype=torch.float32).pin_memory()
+    xd = torch.empty_like(x)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for i in range(args.steps):
+        xd.copy_(xh, non_blocking=True)
+        step(i, xd)
+        yh.copy_(y, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a0.elapsed_time(a1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    errs = zmoe_get_device_errors()
+    peaks = load_peaks()
+    M = T
+    alg = (touched * 3 * L.f * L.d + touched * (2 * L.f + L.d) * 4 + T * L.d * 2 + L.E * L.d * 2
+           + 2 * M * L.d * 2 + 2 * (M * 2 * L.f * 2) + M * L.d * 4 + T * L.d * 4)
+    achieved = alg / (k_ms / 1e3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        t0, n = time.perf_counter(), 0
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            oracle.moe_layer_fp8(L.x, L.w_router, Q[0][0], Q[0][1], Q[1][0], Q[1][1], Q[2][0], Q[2][1], 1,
+                                 sel_bias=L.sel_bias)
+            n += 1
+        el = time.perf_counter() - t0
+        cpu = {"value": T * n / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"oracle.moe_layer_fp8 (numpy float64) on the 64-token layer, {n} step(s), {el:.1f} s"}
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8", "data": "synthetic",
+            "config": {"workload": WORKLOADS[7], "T": T, "d_model": L.d, "d_ff": L.f, "E": L.E, "k": 1,
+                       "parallelism": f"dp{world} (replicated weights, no data-path collective)",
+                       "l2": f"fp8 weights rotated over {n_copies} device copies ({n_copies * 0.302:.1f} GB > 126 MB L2)",
+                       "experts_touched": touched},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "kernel": "moe_layer_kernel<fp8>: router, dispatch, fp8 SwiGLU and combine in one launch",
+                         "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"]},
+            "cpu_baseline": cpu,
+            "e2e": {"value": T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": T * L.d * 2, "d2h_bytes_per_step": T * L.d * 4},
+            "gpu_launches": args.steps, "clocks": clk.summary(), "layer_ms_per_step": k_ms, "device_errors": errs,
+        }), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.config == 7:
+        return run_fp8(args)
     if args.config >= 5:
         return run_stack(args)
 

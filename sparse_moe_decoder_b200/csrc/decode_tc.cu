@@ -60,18 +60,24 @@ constexpr int W_BYTES = BM * KS * 2;          // 32 KB
 constexpr int X_BYTES = NT * KS * 2;          // 4 KB  x slice
 constexpr int HP_BYTES = NT * KS * 2 * 2;     // 8 KB  h_hi + h_lo slice
 constexpr int STAGE_BYTES = W_BYTES + HP_BYTES;
-constexpr int kThreads = 224;                 // 7 warps
+constexpr int kThreads = 224;                 // 7 warps (bf16 weights; fp8 adds 4 converter warps)
 constexpr int kWarps = kThreads / 32;
+constexpr int kMaxWarps = 11;
 constexpr int kWarpTok = 6;
+constexpr int kWarpConv = 7;                  // fp8: warps 7..10 expand weight boxes to f16
 constexpr uint32_t TMEM_COLS = 64;            // 2 accumulator buffers x (gate 16 | up 16)
 constexpr int kMaxE = 64;
 constexpr int kMaxCtas = 256;
 constexpr int kMaxAssign = 1024;              // T * k of the fused layer
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 constexpr uint32_t kIdesc = idesc_bf16_f32(BM, NT);
+// kind::f16 with f16 A and B (format field 0): the fp8 path's expanded weights and f16 tokens.
+constexpr uint32_t kIdescF16 = (1u << 4) | (static_cast<uint32_t>(NT >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
 // fused layer, phase 0 scratch in the (then idle) ring: ids, ranks, the routed row (f32), the raw
 // token row, gamma, and the router matrix when it fits
-constexpr int kRingBytes = STAGES * STAGE_BYTES;
+// Phase-0 scratch bound, common to both weight formats (the fp8 ring plus its conversion buffers is the
+// smaller of the two shared-memory ring regions).
+constexpr int kRingBytes = STAGES * (BM * KS + HP_BYTES) + 2 * W_BYTES;
 
 constexpr int kScratch0 = 2 * kMaxAssign * 4;
 
@@ -94,6 +100,10 @@ struct DecArgs {
   const float* residual;    // [T, d] or null
   float* out;               // [T, d] (may alias residual)
   unsigned int* comb_cnt;   // [T, d / BM] units of each token's row block done (k = 2)
+  // fp8 weights: fp32 scale of each weight row (w = code * scale), applied in the final epilogue
+  const float* s_gate;      // [E, f]
+  const float* s_up;        // [E, f]
+  const float* s_down;      // [E, d]
   // fused layer: x_perm is complete once this counter reaches x_target (grid-wide arrivals)
   const unsigned int* x_ready;
   unsigned int x_target;
@@ -130,6 +140,8 @@ struct __align__(16) Ctrl {
   uint64_t tempty[2];
   uint64_t drain;
   uint64_t rbar[2];          // fused layer: router matrix (+ gamma), token row
+  uint64_t cfull[2];         // fp8: f16 conversion buffer written
+  uint64_t cempty[2];        // fp8: f16 conversion buffer consumed by the MMAs
   uint32_t tmem_base;
   int abort;
   int bad;
@@ -142,16 +154,29 @@ struct __align__(16) Ctrl {
   int rowsrc[kMaxAssign];    // permuted row -> token
   int invp[kMaxAssign];      // assignment (t, i) -> permuted row
   float gsm[kMaxAssign];     // gate of assignment (t, i)
-  int wcnt[kWarps][kMaxE];
+  int wcnt[kMaxWarps][kMaxE];
   int run[kMaxE];
-  float red[kWarps + 1];
-  float wpart[kWarps][16];
+  float red[kMaxWarps + 1];
+  float wpart[kMaxWarps][16];
   float lbias[kMaxE];        // logit_bias (0 when absent)
   float sbias[kMaxE];        // selection bias (0 when absent)
 };
 
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + sizeof(Ctrl);
-static_assert(kSmemBytes <= 227 * 1024, "ring + control block exceed the 227 KB a B200 CTA may use");
+// Shared-memory layout per weight format: the ring of STAGES slots (weight box + token slice), for fp8
+// two f16 conversion buffers (the MMA's A operand), then the control block.
+template <bool FP8>
+struct Lay {
+  static constexpr int W_IN = FP8 ? BM * KS : W_BYTES;       // bytes of one weight box in the ring
+  static constexpr int SLOT = W_IN + HP_BYTES;
+  static constexpr int CBUF = STAGES * SLOT;                 // offset of the conversion buffers
+  static constexpr int RING = CBUF + (FP8 ? 2 * W_BYTES : 0);
+  static constexpr int THREADS = FP8 ? kThreads + 128 : kThreads;
+  static constexpr size_t SMEM = 1024 + static_cast<size_t>(RING) + sizeof(Ctrl);
+  static_assert(SLOT % 1024 == 0 && W_IN % 1024 == 0, "swizzled operands need 1024-byte alignment");
+  static_assert(SMEM <= 227 * 1024, "ring + control block exceed the 227 KB a B200 CTA may use");
+  static_assert(RING >= kRingBytes, "phase-0 scratch must fit in the ring");
+};
+constexpr size_t kSmemBytes = Lay<false>::SMEM;
 
 // ------------------------------------------------------------------------------------------
 // work geometry (every role walks the same sequence)
@@ -262,6 +287,10 @@ __device__ __forceinline__ void init_ctrl(Ctrl& C) {
     mbar_init(&C.drain, 1);
     mbar_init(&C.rbar[0], 1);
     mbar_init(&C.rbar[1], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&C.cfull[b], 4);    // one arrival per converter warp
+      mbar_init(&C.cempty[b], 1);   // tcgen05.commit of the stage's MMAs
+    }
     C.abort = 0;
     C.bad = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -306,9 +335,14 @@ __device__ __forceinline__ void build_tables(Ctrl& C, const DecArgs& p, const in
 // ------------------------------------------------------------------------------------------
 // the SwiGLU roles (both kernels)
 // ------------------------------------------------------------------------------------------
+// FP8: weight boxes arrive as E4M3 codes [128 rows][128 B] (no swizzle); warps 7..10 expand each into
+// an f16 tile in the K-major 128-byte-swizzle layout ([chunk][row][128 B]) that the MMA reads, tokens
+// are f16, and the row scales multiply the finished sums.
+template <bool FP8>
 __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensorMap* mWu, const CUtensorMap* mWd,
                                           const CUtensorMap* mX, const CUtensorMap* mH, const DecArgs& p, Ctrl& C,
                                           unsigned char* base, uint32_t tmem, const int* S) {
+  using LY = Lay<FP8>;
   volatile int* abort_flag = &C.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
@@ -345,16 +379,22 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
               ok = false;
               break;
             }
-            unsigned char* dst = base + slot * STAGE_BYTES;
+            unsigned char* dst = base + slot * LY::SLOT;
             if (wt) {
-              mbar_expect_tx(&full[slot], W_BYTES);
-              if (ph == 0)
+              mbar_expect_tx(&full[slot], LY::W_IN);
+              if (FP8) {
+                if (ph == 0)
+                  tma_load_2d(dst, (j & 1) ? mWu : mWg, &full[slot], (j >> 1) * KS, U.e * p.f + U.rb * BM);
+                else
+                  tma_load_2d(dst, mWd, &full[slot], j * KS, U.e * p.d + U.rb * BM);
+              } else if (ph == 0) {
                 tma_load_3d(dst, (j & 1) ? mWu : mWg, &full[slot], 0, U.e * p.f + U.rb * BM, (j >> 1) * CH);
-              else
+              } else {
                 tma_load_3d(dst, mWd, &full[slot], 0, U.e * p.d + U.rb * BM, j * CH);
+              }
             } else if (ph == 0) {
               mbar_expect_tx(&full[slot], X_BYTES);
-              tma_load_3d(dst + W_BYTES, mX, &full[slot], 0, U.row0, (j >> 1) * CH);
+              tma_load_3d(dst + LY::W_IN, mX, &full[slot], 0, U.row0, (j >> 1) * CH);
             } else {
               if (U.e != ready_e) {
                 // every phase-A unit of expert e must have stored its h rows
@@ -371,7 +411,7 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
                 asm volatile("fence.proxy.async.global;" ::: "memory");
               }
               mbar_expect_tx(&full[slot], HP_BYTES);
-              tma_load_4d(dst + W_BYTES, mH, &full[slot], 0, U.row0, 0, j * CH);
+              tma_load_4d(dst + LY::W_IN, mH, &full[slot], 0, U.row0, 0, j * CH);
             }
             ++q;
           }
@@ -399,14 +439,17 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
           for (int j = g.j0; j < g.j1; ++j, ++q) {
             const int slot = q % STAGES;
             const uint32_t par = static_cast<uint32_t>((q / STAGES) & 1);
-            if (!mbar_wait(&C.full_w[slot], par, abort_flag, kTimeoutNs) ||
+            const int cb = q & 1;   // fp8: the conversion buffer holding this stage's f16 weights
+            if (!mbar_wait(FP8 ? &C.cfull[cb] : &C.full_w[slot], FP8 ? static_cast<uint32_t>((q >> 1) & 1) : par,
+                           abort_flag, kTimeoutNs) ||
                 !mbar_wait(&C.full_t[slot], par, abort_flag, kTimeoutNs)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t sa = smem_u32(base + slot * STAGE_BYTES);
-            const uint32_t sb = sa + W_BYTES;
+            const uint32_t sa = FP8 ? smem_u32(base + LY::CBUF + cb * W_BYTES) : smem_u32(base + slot * LY::SLOT);
+            const uint32_t sb = smem_u32(base + slot * LY::SLOT + LY::W_IN);
+            constexpr uint32_t idesc = FP8 ? kIdescF16 : kIdesc;
             if (ph == 0) {
               // gate and up stages alternate: the first stage of each matrix in the segment is one of
               // the first two, and its first MMA overwrites that accumulator
@@ -417,7 +460,7 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                   umma_bf16(d_tmem, sw128_desc(sa + c * (BM * 128) + kk * 32), sw128_desc(sb + c * (NT * 128) + kk * 32),
-                            kIdesc, (fresh && c == 0 && kk == 0) ? 0u : 1u);
+                            idesc, (fresh && c == 0 && kk == 0) ? 0u : 1u);
             } else {
               // h_hi and h_lo slices of chunk c sit at 2c and 2c + 1 (2 KB each)
               const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * 32);
@@ -427,12 +470,13 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                   const uint64_t ad = sw128_desc(sa + c * (BM * 128) + kk * 32);
-                  umma_bf16(d_tmem, ad, sw128_desc(sb + (2 * c) * (NT * 128) + kk * 32), kIdesc,
+                  umma_bf16(d_tmem, ad, sw128_desc(sb + (2 * c) * (NT * 128) + kk * 32), idesc,
                             (fresh && c == 0 && kk == 0) ? 0u : 1u);
-                  umma_bf16(d_tmem, ad, sw128_desc(sb + (2 * c + 1) * (NT * 128) + kk * 32), kIdesc, 1u);
+                  umma_bf16(d_tmem, ad, sw128_desc(sb + (2 * c + 1) * (NT * 128) + kk * 32), idesc, 1u);
                 }
             }
             umma_commit(&C.empty[slot]);
+            if (FP8) umma_commit(&C.cempty[cb]);
           }
           if (!ok) break;
           umma_commit(&C.tfull[b]);
@@ -446,7 +490,7 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
       while (!mbar_try_wait(&C.drain, 0) && globaltimer() - t1 < kTimeoutNs) {
       }
     }
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // ===================================== epilogue (warps 2..5) =====================================
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;                 // accumulator row = TMEM lane
@@ -538,16 +582,34 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
         }
         // the unit's final epilogue
         const int n = U.rb * BM + row;
+        if (FP8) {
+          // w = code * scale: the row's scale multiplies its finished sums
+          const float sa = __ldg((ph == 0 ? p.s_gate : p.s_down) + static_cast<size_t>(U.e) * (ph == 0 ? p.f : p.d) + n);
+          const float su = ph == 0 ? __ldg(p.s_up + static_cast<size_t>(U.e) * p.f + n) : 1.f;
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            g[t] *= sa;
+            v[t] *= su;
+          }
+        }
         if (ph == 0) {
           const size_t ld = static_cast<size_t>(2) * p.f;
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
             if (t < U.rows) {
               const float hv = g[t] / (1.f + expf(-g[t])) * v[t];
-              const uint16_t hi = f32_to_bf16_bits(hv);
               uint16_t* hr = p.h + static_cast<size_t>(U.row0 + t) * ld;
-              hr[n] = hi;
-              hr[p.f + n] = f32_to_bf16_bits(hv - bf16_to_f32(hi));
+              if (FP8) {
+                // the f16 pair: the fp8 path's MMAs take f16 operands
+                const __half hh = __float2half_rn(hv);
+                if (__hisinf(hh)) record_device_error(p.errors);   // |h| beyond the f16 range
+                hr[n] = __half_as_ushort(hh);
+                hr[p.f + n] = __half_as_ushort(__float2half_rn(hv - __half2float(hh)));
+              } else {
+                const uint16_t hi = f32_to_bf16_bits(hv);
+                hr[n] = hi;
+                hr[p.f + n] = f32_to_bf16_bits(hv - bf16_to_f32(hi));
+              }
             }
           }
           epi_bar();
@@ -599,6 +661,54 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
       }
     }
     if (!ok) set_abort(C, p.timeouts);
+  } else if (FP8 && warp >= kWarpConv) {
+    // ========================= fp8 converters (warps 7..10): E4M3 box -> f16 tile =========================
+    // Each warp expands 4 rows per step (rows 4 cw + 16 i + lane / 8): lane l takes the 16-byte segment
+    // l % 8 of its 128-byte code row (k = 16 (l % 8) .. + 15) and writes the 16 f16 values, two 16-byte
+    // units, into chunk (l % 8) / 4 of the swizzled tile.
+    const int cw = warp - kWarpConv;
+    const int rsub = lane >> 3, sgm = lane & 7;
+    const int c = sgm >> 2, u0 = (sgm & 3) * 2;
+    int q = 0;
+    bool ok = true;
+    for (int ph = 0; ph < 2 && ok; ++ph) {
+      const Plan P = make_plan(C.rlo[ph][cta], C.rlo[ph][cta + 1], S[ph]);
+      for (int i = 0; i < P.n && ok; ++i) {
+        const Seg g = seg_at(P, i);
+        for (int j = g.j0; j < g.j1; ++j, ++q) {
+          const int slot = q % STAGES, cb = q & 1;
+          if (!mbar_wait(&C.full_w[slot], static_cast<uint32_t>((q / STAGES) & 1), abort_flag, kTimeoutNs) ||
+              !mbar_wait(&C.cempty[cb], static_cast<uint32_t>((q >> 1) & 1) ^ 1u, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          const unsigned char* src = base + slot * LY::SLOT;
+          unsigned char* dst = base + LY::CBUF + cb * W_BYTES;
+#pragma unroll 2
+          for (int r0 = cw * 4; r0 < BM; r0 += 16) {
+            const int r = r0 + rsub;
+            const uint4 wv = *reinterpret_cast<const uint4*>(src + r * 128 + sgm * 16);
+            uint4 o0, o1;
+            o0.x = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.x));
+            o0.y = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.x >> 16));
+            o0.z = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.y));
+            o0.w = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.y >> 16));
+            o1.x = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.z));
+            o1.y = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.z >> 16));
+            o1.z = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.w));
+            o1.w = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.w >> 16));
+            unsigned char* rowp = dst + c * (BM * 128) + r * 128;
+            *reinterpret_cast<uint4*>(rowp + ((u0 ^ (r & 7)) << 4)) = o0;
+            *reinterpret_cast<uint4*>(rowp + (((u0 + 1) ^ (r & 7)) << 4)) = o1;
+          }
+          // generic-proxy writes, read next by the tensor core (async proxy)
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&C.cfull[cb]);
+        }
+      }
+    }
+    if (!ok) set_abort(C, p.timeouts);
   }
 }
 
@@ -619,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   build_tables(C, p, S);
   const uint32_t tmem = C.tmem_base;
-  if (!C.bad) ffn_roles(&mapWg, &mapWu, &mapWd, &mapX, &mapH, p, C, base, tmem, S);
+  if (!C.bad) ffn_roles<false>(&mapWg, &mapWu, &mapWd, &mapX, &mapH, p, C, base, tmem, S);
   // The producer and MMA roles run on lane 0 alone: the other lanes wait here for it, so that every
   // warp meets the CTA barrier (and warp 1 the TMEM release) converged.
   __syncwarp();
@@ -653,6 +763,10 @@ __device__ __forceinline__ bool grid_barrier(unsigned int* ctr, unsigned int rou
   return *reinterpret_cast<volatile int*>(&C.abort) == 0;
 }
 
+// Phase 0 runs on every warp of the CTA (7 with bf16 weights, 11 with fp8).
+__device__ __forceinline__ int nthreads() { return static_cast<int>(blockDim.x); }
+__device__ __forceinline__ int nwarps() { return static_cast<int>(blockDim.x >> 5); }
+
 __device__ __forceinline__ float block_sum(float v, Ctrl& C) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
@@ -661,11 +775,11 @@ __device__ __forceinline__ float block_sum(float v, Ctrl& C) {
   __syncthreads();
   if (threadIdx.x == 0) {
     float s = 0.f;
-    for (int w = 0; w < kWarps; ++w) s += C.red[w];
-    C.red[kWarps] = s;
+    for (int w = 0; w < nwarps(); ++w) s += C.red[w];
+    C.red[nwarps()] = s;
   }
   __syncthreads();
-  return C.red[kWarps];
+  return C.red[nwarps()];
 }
 
 // Larger score first, then lower expert index.
@@ -741,13 +855,13 @@ __device__ __forceinline__ bool route_item(const LayerArgs& L, const DecArgs& p,
   if (L.gamma) {
     const float* hr = reinterpret_cast<const float*>(R.raw);
     float ss = 0.f;
-    for (int v = threadIdx.x; v < d / 4; v += kThreads) {
+    for (int v = threadIdx.x; v < d / 4; v += nthreads()) {
       const float4 a = reinterpret_cast<const float4*>(hr)[v];
       ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
     }
     ss = block_sum(ss, C);
     const float inv = rsqrtf(ss / static_cast<float>(d) + L.eps);
-    for (int v = threadIdx.x; v < d / 8; v += kThreads) {
+    for (int v = threadIdx.x; v < d / 8; v += nthreads()) {
       uint16_t b[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -764,7 +878,7 @@ __device__ __forceinline__ bool route_item(const LayerArgs& L, const DecArgs& p,
       }
     }
   } else {
-    for (int v = threadIdx.x; v < d / 8; v += kThreads)
+    for (int v = threadIdx.x; v < d / 8; v += nthreads())
       unpack_bf16x8(reinterpret_cast<const uint4*>(R.raw)[v], R.xs + 8 * v);
   }
   __syncthreads();
@@ -780,7 +894,7 @@ __device__ __forceinline__ bool route_item(const LayerArgs& L, const DecArgs& p,
     float acc[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-    for (int v = threadIdx.x; v < d / 8; v += kThreads) {
+    for (int v = threadIdx.x; v < d / 8; v += nthreads()) {
       float xv[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) xv[i] = R.xs[8 * v + i];
@@ -807,7 +921,7 @@ __device__ __forceinline__ bool route_item(const LayerArgs& L, const DecArgs& p,
     __syncthreads();
     if (threadIdx.x < 16 && j0 + threadIdx.x < ne) {
       float sum = 0.f;
-      for (int w = 0; w < kWarps; ++w) sum += C.wpart[w][threadIdx.x];
+      for (int w = 0; w < nwarps(); ++w) sum += C.wpart[w][threadIdx.x];
       L.logits[static_cast<size_t>(t) * E + e0 + j0 + threadIdx.x] = sum;
     }
     __syncthreads();
@@ -827,15 +941,15 @@ __device__ __forceinline__ void select_all(const LayerArgs& L, const DecArgs& p,
   const size_t nl = static_cast<size_t>(L.T) * E;
   const float* lbase = L.logits;
   if (nl * 4 <= scratch_bytes) {
-    for (size_t i = threadIdx.x; i < nl; i += kThreads) scratch[i] = __ldcg(L.logits + i);
+    for (size_t i = threadIdx.x; i < nl; i += nthreads()) scratch[i] = __ldcg(L.logits + i);
     lbase = scratch;
   }
-  for (int e = threadIdx.x; e < E; e += kThreads) {
+  for (int e = threadIdx.x; e < E; e += nthreads()) {
     C.lbias[e] = L.logit_bias ? L.logit_bias[e] : 0.f;
     C.sbias[e] = L.sel_bias ? L.sel_bias[e] : 0.f;
   }
   __syncthreads();
-  for (int t = threadIdx.x; t < L.T; t += kThreads) {
+  for (int t = threadIdx.x; t < L.T; t += nthreads()) {
     const float* lg = lbase + static_cast<size_t>(t) * E;
     float s1 = NEG, s2 = NEG, s3 = NEG, q1 = NEG, q2 = NEG, m = NEG;
     int e1 = -1, e2 = -1;
@@ -900,13 +1014,14 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // Phase 0b, after select_all (every CTA, redundantly): counts, offsets and the stable (expert, token)
 // order of all T * k assignments in ids into C.off / C.rowsrc / C.invp; CTA 0 publishes them; each
 // CTA gathers its share of x_perm.  ids and per-assignment ranks use the (idle) ring as scratch.
-__device__ __forceinline__ void permute_all(const LayerArgs& L, const DecArgs& p, Ctrl& C, int* ids, int* rel) {
+__device__ __forceinline__ void permute_all(const LayerArgs& L, const DecArgs& p, Ctrl& C, int* ids, int* rel,
+                                            bool to_f16) {
   const int n = L.T * p.k, E = p.E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < E) C.run[threadIdx.x] = 0;
   __syncthreads();
-  for (int b0 = 0; b0 < n; b0 += kThreads) {
-    for (int i = threadIdx.x; i < kWarps * kMaxE; i += kThreads) (&C.wcnt[0][0])[i] = 0;
+  for (int b0 = 0; b0 < n; b0 += nthreads()) {
+    for (int i = threadIdx.x; i < nwarps() * kMaxE; i += nthreads()) (&C.wcnt[0][0])[i] = 0;
     __syncthreads();
     const int a = b0 + threadIdx.x;
     const int e = a < n ? ids[a] : -1;
@@ -916,7 +1031,7 @@ __device__ __forceinline__ void permute_all(const LayerArgs& L, const DecArgs& p
     __syncthreads();
     if (threadIdx.x < E) {
       int r = C.run[threadIdx.x];
-      for (int w = 0; w < kWarps; ++w) {
+      for (int w = 0; w < nwarps(); ++w) {
         const int c = C.wcnt[w][threadIdx.x];
         C.wcnt[w][threadIdx.x] = r;
         r += c;
@@ -932,7 +1047,7 @@ __device__ __forceinline__ void permute_all(const LayerArgs& L, const DecArgs& p
     for (int e = 0; e < E; ++e) C.off[e + 1] = C.off[e] + C.run[e];
   }
   __syncthreads();
-  for (int a = threadIdx.x; a < n; a += kThreads) {
+  for (int a = threadIdx.x; a < n; a += nthreads()) {
     const int e = ids[a];
     if (e >= 0) {
       const int pos = C.off[e] + rel[a];
@@ -945,15 +1060,15 @@ __device__ __forceinline__ void permute_all(const LayerArgs& L, const DecArgs& p
   __syncthreads();
   const int rows = C.off[E];
   if (blockIdx.x == 0) {
-    for (int i = threadIdx.x; i < E; i += kThreads) L.counts[i] = C.run[i];
-    for (int i = threadIdx.x; i <= E; i += kThreads) L.offsets[i] = C.off[i];
-    for (int i = threadIdx.x; i < rows; i += kThreads) L.perm[i] = C.rowsrc[i];
-    for (int i = threadIdx.x; i < n; i += kThreads) L.inv_perm[i] = C.invp[i];
+    for (int i = threadIdx.x; i < E; i += nthreads()) L.counts[i] = C.run[i];
+    for (int i = threadIdx.x; i <= E; i += nthreads()) L.offsets[i] = C.off[i];
+    for (int i = threadIdx.x; i < rows; i += nthreads()) L.perm[i] = C.rowsrc[i];
+    for (int i = threadIdx.x; i < n; i += nthreads()) L.inv_perm[i] = C.invp[i];
   }
   // x_perm rows, one warp per row, spread over the grid
   const uint16_t* xsrc = L.gamma ? L.x_norm : L.x_in;
   const int vecs = p.d / 8;
-  for (int r = blockIdx.x * kWarps + warp; r < rows; r += gridDim.x * kWarps) {
+  for (int r = blockIdx.x * nwarps() + warp; r < rows; r += gridDim.x * nwarps()) {
     const uint4* s = reinterpret_cast<const uint4*>(xsrc + static_cast<size_t>(C.rowsrc[r]) * p.d);
     uint4* dst = reinterpret_cast<uint4*>(L.x_perm + static_cast<size_t>(r) * p.d);
     for (int v0 = 0; v0 < vecs; v0 += 32 * 8) {
@@ -963,19 +1078,37 @@ __device__ __forceinline__ void permute_all(const LayerArgs& L, const DecArgs& p
         if (v0 + j * 32 + lane < vecs) buf[j] = __ldcg(s + v0 + j * 32 + lane);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (v0 + j * 32 + lane < vecs) dst[v0 + j * 32 + lane] = buf[j];
+        if (v0 + j * 32 + lane < vecs) {
+          if (to_f16) {
+            // fp8 weights: the MMA operands are f16 (exact for bf16 values in f16's normal range)
+            float f8[8];
+            unpack_bf16x8(buf[j], f8);
+            uint32_t w[4];
+            bool inf = false;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const __half2 h2 = __floats2half2_rn(f8[2 * i], f8[2 * i + 1]);
+              inf |= __hisinf(__low2half(h2)) || __hisinf(__high2half(h2));
+              w[i] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            if (inf) record_device_error(p.errors);
+            buf[j] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          dst[v0 + j * 32 + lane] = buf[j];
+        }
     }
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool FP8>
+__global__ void __launch_bounds__(Lay<FP8>::THREADS, 1)
     moe_layer_kernel(const __grid_constant__ CUtensorMap mapWg, const __grid_constant__ CUtensorMap mapWu,
                      const __grid_constant__ CUtensorMap mapWd, const __grid_constant__ CUtensorMap mapX,
                      const __grid_constant__ CUtensorMap mapH, DecArgs p, LayerArgs L) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  Ctrl& C = *reinterpret_cast<Ctrl*>(base + STAGES * STAGE_BYTES);
+  Ctrl& C = *reinterpret_cast<Ctrl*>(base + Lay<FP8>::RING);
   const int S[2] = {2 * (p.d / KS), p.f / KS};
   init_ctrl(C);
   __syncthreads();
@@ -1010,7 +1143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (grid_barrier(L.gbar, 1, C, p.timeouts)) {
     select_all(L, p, C, ids, reinterpret_cast<float*>(base + kScratch0), kRingBytes - kScratch0);
-    permute_all(L, p, C, ids, rel);
+    permute_all(L, p, C, ids, rel, FP8);
     // generic-proxy writes to the ring are ordered before the TMA writes that will reuse it
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     build_tables(C, p, S);   // ends with a CTA barrier: this CTA's x_perm rows are written
@@ -1018,7 +1151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (DecArgs::x_ready); the weight producer starts streaming at once.  An epilogue thread arrives
     // (its release fence waits for this CTA's gather stores; the producers must not wait on it).
     if (threadIdx.x == 64) red_release_add(L.gbar, 1u);
-    if (!C.bad) ffn_roles(&mapWg, &mapWu, &mapWd, &mapX, &mapH, p, C, base, C.tmem_base, S);
+    if (!C.bad) ffn_roles<FP8>(&mapWg, &mapWu, &mapWd, &mapX, &mapH, p, C, base, C.tmem_base, S);
   }
   __syncwarp();
   __syncthreads();
@@ -1093,14 +1226,14 @@ bool encode_maps(Maps* m, const uint16_t* x_perm, int M_total, const uint16_t* w
 }
 
 template <typename K, typename... Args>
-zmoe_status launch_coop(K kernel, const char* what, cudaStream_t s, Args... args) {
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes)) !=
+zmoe_status launch_coop(K kernel, const char* what, cudaStream_t s, int threads, size_t smem, Args... args) {
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
     return check_launch(what);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(num_sms()));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: CTAs wait on one another
@@ -1158,7 +1291,8 @@ zmoe_status grouped_swiglu_dec_tc(const uint16_t* x_perm, const int32_t* offsets
   if (cudaMemsetAsync(ws, 0, Lo.counters_end, s) != cudaSuccess)
     return check_launch("grouped_swiglu (decode): clearing the counters");
   const DecArgs args = dec_args(Lo, ws, offsets, h, y_perm, E, d, f, M_total);
-  return launch_coop(dec_tc_kernel, "grouped_swiglu (decode)", s, m.g, m.u, m.dn, m.x, m.h, args);
+  return launch_coop(dec_tc_kernel, "grouped_swiglu (decode)", s, kThreads, kSmemBytes, m.g, m.u, m.dn, m.x, m.h,
+                     args);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1202,11 +1336,13 @@ LayerWs layer_ws(int T, int E, int d, int f, int k) {
 
 size_t moe_layer_fused_workspace(int T, int E, int d, int f, int k) { return layer_ws(T, E, d, f, k).total; }
 
+// fp8 weights when s_gate is given: w_gate / w_up / w_down are E4M3 codes with row scales s_*.
 zmoe_status moe_layer_fused(const uint16_t* x, const float* h_in, const float* gamma, float eps, const uint16_t* w_r,
-                            const float* logit_bias, const float* sel_bias, const uint16_t* w_gate,
-                            const uint16_t* w_up, const uint16_t* w_down, int T, int d, int f, int E, int k, float* y,
-                            int32_t* expert_idx, float* gates, float* margin, uint16_t* x_norm_out, void* ws,
-                            cudaStream_t s) {
+                            const float* logit_bias, const float* sel_bias, const void* w_gate, const void* w_up,
+                            const void* w_down, int T, int d, int f, int E, int k, float* y, int32_t* expert_idx,
+                            float* gates, float* margin, uint16_t* x_norm_out, void* ws, cudaStream_t s,
+                            const float* s_gate, const float* s_up, const float* s_down) {
+  const bool fp8 = s_gate != nullptr;
   const LayerWs W = layer_ws(T, E, d, f, k);
   unsigned char* w = static_cast<unsigned char*>(ws);
   const int n = T * k;
@@ -1215,8 +1351,20 @@ zmoe_status moe_layer_fused(const uint16_t* x, const float* h_in, const float* g
   uint16_t* hh = reinterpret_cast<uint16_t*>(w + W.h);
   float* yp = reinterpret_cast<float*>(w + W.y_perm);
   Maps m;
-  if (!encode_maps(&m, xp, n, w_gate, w_up, w_down, E, d, f, hh))
-    return fail(ZMOE_ERR_CUDA, "zmoe_moe_layer: cuTensorMapEncodeTiled failed");
+  bool okm = encode_maps(&m, xp, n, static_cast<const uint16_t*>(w_gate), static_cast<const uint16_t*>(w_up),
+                         static_cast<const uint16_t*>(w_down), E, d, f, hh);
+  if (okm && fp8) {
+    // E4M3 codes [rows][K]: a 128-row x 128-byte box, unswizzled (the converter warps swizzle)
+    const cuuint64_t dg[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(E) * f};
+    const cuuint64_t sg[1] = {static_cast<cuuint64_t>(d)};
+    const cuuint64_t dd[2] = {static_cast<cuuint64_t>(f), static_cast<cuuint64_t>(E) * d};
+    const cuuint64_t sd[1] = {static_cast<cuuint64_t>(f)};
+    const cuuint32_t box[2] = {KS, BM};
+    okm = encode_map(&m.g, w_gate, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, dg, sg, box, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+          encode_map(&m.u, w_up, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, dg, sg, box, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+          encode_map(&m.dn, w_down, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, dd, sd, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
+  if (!okm) return fail(ZMOE_ERR_CUDA, "zmoe_moe_layer: cuTensorMapEncodeTiled failed");
   if (cudaMemsetAsync(ws, 0, W.ffn.counters_end, s) != cudaSuccess)
     return check_launch("zmoe_moe_layer: clearing the counters");
   DecArgs a = dec_args(W.ffn, ws, nullptr, hh, yp, E, d, f, n);
@@ -1256,7 +1404,14 @@ zmoe_status moe_layer_fused(const uint16_t* x, const float* h_in, const float* g
   a.comb_cnt = reinterpret_cast<unsigned int*>(w + W.ffn.comb);
   a.x_ready = L.gbar;                                  // second grid arrival: x_perm complete
   a.x_target = 2u * static_cast<unsigned int>(num_sms());
-  return launch_coop(moe_layer_kernel, "zmoe_moe_layer (fused decode)", s, m.g, m.u, m.dn, m.x, m.h, a, L);
+  a.s_gate = s_gate;
+  a.s_up = s_up;
+  a.s_down = s_down;
+  if (fp8)
+    return launch_coop(moe_layer_kernel<true>, "zmoe_moe_layer_fp8 (fused decode)", s, Lay<true>::THREADS,
+                       Lay<true>::SMEM, m.g, m.u, m.dn, m.x, m.h, a, L);
+  return launch_coop(moe_layer_kernel<false>, "zmoe_moe_layer (fused decode)", s, Lay<false>::THREADS,
+                     Lay<false>::SMEM, m.g, m.u, m.dn, m.x, m.h, a, L);
 }
 
 }  // namespace zmoe

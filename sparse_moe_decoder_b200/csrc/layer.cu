@@ -15,10 +15,10 @@ namespace zmoe {
 bool moe_layer_fused_supported(int T, int E, int d, int f, int k);
 size_t moe_layer_fused_workspace(int T, int E, int d, int f, int k);
 zmoe_status moe_layer_fused(const uint16_t* x, const float* h_in, const float* gamma, float eps, const uint16_t* w_r,
-                            const float* logit_bias, const float* sel_bias, const uint16_t* w_gate,
-                            const uint16_t* w_up, const uint16_t* w_down, int T, int d, int f, int E, int k, float* y,
-                            int32_t* expert_idx, float* gates, float* margin, uint16_t* x_norm_out, void* ws,
-                            cudaStream_t s);
+                            const float* logit_bias, const float* sel_bias, const void* w_gate, const void* w_up,
+                            const void* w_down, int T, int d, int f, int E, int k, float* y, int32_t* expert_idx,
+                            float* gates, float* margin, uint16_t* x_norm_out, void* ws, cudaStream_t s,
+                            const float* s_gate, const float* s_up, const float* s_down);
 
 namespace {
 
@@ -104,9 +104,8 @@ zmoe_status zmoe_moe_layer(const void* x, const float* h, const float* gamma, fl
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (use_fused(T, E, d, f, k, dtype))
     return moe_layer_fused(static_cast<const uint16_t*>(x), h, gamma, eps, static_cast<const uint16_t*>(w_router),
-                           logit_bias, sel_bias, static_cast<const uint16_t*>(w_gate),
-                           static_cast<const uint16_t*>(w_up), static_cast<const uint16_t*>(w_down), T, d, f, E, k, y,
-                           expert_idx, gates, margin, static_cast<uint16_t*>(x_norm), workspace, s);
+                           logit_bias, sel_bias, w_gate, w_up, w_down, T, d, f, E, k, y, expert_idx, gates, margin,
+                           static_cast<uint16_t*>(x_norm), workspace, s, nullptr, nullptr, nullptr);
 
   const SeqWs W = seq_ws(T, E, d, f, k, dtype);
   unsigned char* w = static_cast<unsigned char*>(workspace);
@@ -132,6 +131,45 @@ zmoe_status zmoe_moe_layer(const void* x, const float* h, const float* gamma, fl
   if (st != ZMOE_OK) return st;
   (void)s;
   return zmoe_combine(yp, inv, g, h, T, d, k, y, stream);
+}
+
+size_t zmoe_moe_layer_fp8_workspace_size(int T, int d, int f, int E, int k) {
+  using namespace zmoe;
+  if (T <= 0 || d < 1 || f < 1 || E < 1 || E > 64 || (k != 1 && k != 2) || !moe_layer_fused_supported(T, E, d, f, k))
+    return 0;
+  return moe_layer_fused_workspace(T, E, d, f, k);
+}
+
+zmoe_status zmoe_moe_layer_fp8(const void* x, const float* h, const float* gamma, float eps, const void* w_router,
+                               const float* logit_bias, const float* sel_bias, const uint8_t* q_gate,
+                               const float* s_gate, const uint8_t* q_up, const float* s_up, const uint8_t* q_down,
+                               const float* s_down, int T, int d, int f, int E, int k, float* y, int32_t* expert_idx,
+                               float* gates, float* margin, void* x_norm, void* workspace, size_t ws_bytes,
+                               zmoe_stream_t stream) {
+  using namespace zmoe;
+  ZMOE_REQUIRE(T >= 0, "zmoe_moe_layer_fp8: T must be >= 0");
+  ZMOE_REQUIRE(E >= 1 && E <= 64, "zmoe_moe_layer_fp8: E must be in [1, 64]");
+  ZMOE_REQUIRE((k == 1 || k == 2) && k <= E, "zmoe_moe_layer_fp8: k must be 1 or 2 and <= E");
+  ZMOE_REQUIRE(d % 256 == 0 && f % 256 == 0 && d > 0 && f > 0, "zmoe_moe_layer_fp8: d and f must be multiples of 256");
+  if (T == 0) return ZMOE_OK;
+  ZMOE_REQUIRE((w_router || E == 1) && q_gate && s_gate && q_up && s_up && q_down && s_down && y,
+               "zmoe_moe_layer_fp8: NULL pointer (w_router may be NULL only when E == 1)");
+  ZMOE_REQUIRE(gamma ? h != nullptr : x != nullptr, "zmoe_moe_layer_fp8: needs x, or h with gamma");
+  ZMOE_REQUIRE((!x || aligned16(x)) && (!h || aligned16(h)) && aligned16(y) && (!w_router || aligned16(w_router)) &&
+                   aligned16(q_gate) && aligned16(q_up) && aligned16(q_down) && (!x_norm || aligned16(x_norm)) &&
+                   (!gamma || aligned16(gamma)),
+               "zmoe_moe_layer_fp8: pointers must be 16-byte aligned");
+  if (!moe_layer_fused_supported(T, E, d, f, k) || static_cast<long long>(T) * k >= 64LL * E)
+    return fail(ZMOE_ERR_UNSUPPORTED, "zmoe_moe_layer_fp8: decode sizes only (T * k < 64 E, T * k <= 1024)");
+  const size_t need = zmoe_moe_layer_fp8_workspace_size(T, d, f, E, k);
+  if (!workspace || ws_bytes < need)
+    return fail(ZMOE_ERR_WORKSPACE_TOO_SMALL,
+                "zmoe_moe_layer_fp8: workspace smaller than zmoe_moe_layer_fp8_workspace_size()");
+  clear_error();
+  return moe_layer_fused(static_cast<const uint16_t*>(x), h, gamma, eps, static_cast<const uint16_t*>(w_router),
+                         logit_bias, sel_bias, q_gate, q_up, q_down, T, d, f, E, k, y, expert_idx, gates, margin,
+                         static_cast<uint16_t*>(x_norm), workspace, reinterpret_cast<cudaStream_t>(stream), s_gate,
+                         s_up, s_down);
 }
 
 }  // extern "C"

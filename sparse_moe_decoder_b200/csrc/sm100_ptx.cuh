@@ -189,6 +189,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Two E4M3 values (low byte first) -> two f16 (low half first); exact (every E4M3 value is an f16).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+  return r;
+}
+
 // ---------------------------------------------------------------------------------------------
 // named barriers
 // ---------------------------------------------------------------------------------------------
@@ -258,15 +265,22 @@ inline EncodeTiledFn tensor_map_encoder() {
   return fn;
 }
 
-// bf16 tensor of `rank` dims (dims[0] innermost, element strides 1), 128-byte swizzle, zero fill.
-inline bool encode_bf16_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
-                            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+// Tensor of `rank` dims (dims[0] innermost, element strides 1), zero fill.
+inline bool encode_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int rank, const cuuint64_t* dims,
+                       const cuuint64_t* strides_bytes, const cuuint32_t* box, CUtensorMapSwizzle swz) {
   EncodeTiledFn enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(ptr), dims,
-             strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(ptr), dims, strides_bytes, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 (or any 2-byte type: the copy does not look at the values) tensor, 128-byte swizzle.
+inline bool encode_bf16_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
+                            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  return encode_map(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, dims, strides_bytes, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace zmoe
