@@ -59,13 +59,15 @@ constexpr int STAGES = 5;
 constexpr int W_BYTES = BM * KS * 2;          // 32 KB
 constexpr int X_BYTES = NT * KS * 2;          // 4 KB  x slice
 constexpr int HP_BYTES = NT * KS * 2 * 2;     // 8 KB  h_hi + h_lo slice
-constexpr int STAGE_BYTES = W_BYTES + HP_BYTES;
 constexpr int kThreads = 224;                 // 7 warps (bf16 weights; fp8 adds 4 converter warps)
-constexpr int kWarps = kThreads / 32;
 constexpr int kMaxWarps = 11;
 constexpr int kWarpTok = 6;
 constexpr int kWarpConv = 7;                  // fp8: warps 7..10 expand weight boxes to f16
+constexpr int KS8 = 256;                      // fp8: k per weight stage (two f16 sub-stages of KS)
+constexpr int W8_BYTES = BM * KS8;            // 32 KB of E4M3 codes
 constexpr uint32_t TMEM_COLS = 64;            // 2 accumulator buffers x (gate 16 | up 16)
+constexpr uint32_t TMEM_COLS8 = 256;          // fp8: the accumulators, then 2 f16 A tiles of 64 columns
+constexpr uint32_t kTmemA = 64;               // fp8: first column of A tile 0 (128 k of f16, 2 per column)
 constexpr int kMaxE = 64;
 constexpr int kMaxCtas = 256;
 constexpr int kMaxAssign = 1024;              // T * k of the fused layer
@@ -73,11 +75,13 @@ constexpr unsigned long long kTimeoutNs = 2000000000ull;
 constexpr uint32_t kIdesc = idesc_bf16_f32(BM, NT);
 // kind::f16 with f16 A and B (format field 0): the fp8 path's expanded weights and f16 tokens.
 constexpr uint32_t kIdescF16 = (1u << 4) | (static_cast<uint32_t>(NT >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+constexpr uint32_t kIdesc32 = idesc_bf16_f32(BM, 2 * NT);   // phase B: h_hi and h_lo rows as one operand
+constexpr uint32_t kIdescF16x32 =
+    (1u << 4) | (static_cast<uint32_t>((2 * NT) >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
 // fused layer, phase 0 scratch in the (then idle) ring: ids, ranks, the routed row (f32), the raw
-// token row, gamma, and the router matrix when it fits
-// Phase-0 scratch bound, common to both weight formats (the fp8 ring plus its conversion buffers is the
-// smaller of the two shared-memory ring regions).
-constexpr int kRingBytes = STAGES * (BM * KS + HP_BYTES) + 2 * W_BYTES;
+// token row, gamma, and the router matrix when it fits.  The bound lies within the ring of either
+// weight format (checked in Lay).
+constexpr int kRingBytes = 184 * 1024;
 
 constexpr int kScratch0 = 2 * kMaxAssign * 4;
 
@@ -140,8 +144,9 @@ struct __align__(16) Ctrl {
   uint64_t tempty[2];
   uint64_t drain;
   uint64_t rbar[2];          // fused layer: router matrix (+ gamma), token row
-  uint64_t cfull[2];         // fp8: f16 conversion buffer written
-  uint64_t cempty[2];        // fp8: f16 conversion buffer consumed by the MMAs
+  uint64_t tok_empty[STAGES];  // fp8: token slot consumed by the MMAs (bf16: one slot with the weights);
+                               // its commit also frees the sub-stage's A tile
+  uint64_t afull[2];         // fp8: f16 A tile written to TMEM by the converter warps
   uint32_t tmem_base;
   int abort;
   int bad;
@@ -162,17 +167,23 @@ struct __align__(16) Ctrl {
   float sbias[kMaxE];        // selection bias (0 when absent)
 };
 
-// Shared-memory layout per weight format: the ring of STAGES slots (weight box + token slice), for fp8
-// two f16 conversion buffers (the MMA's A operand), then the control block.
+// Shared-memory layout per weight format.  bf16: a ring of STAGES slots, each a 32 KB weight box
+// (128 rows x 128 k) and the token slice of the same k.  fp8: a ring of STAGES 32 KB E4M3 boxes
+// (128 rows x 256 k) and, apart from it, a ring of STAGES token slices (one per 128 k), so that a
+// weight slot is free again as soon as the converter warps have read it.  The control block follows.
 template <bool FP8>
 struct Lay {
-  static constexpr int W_IN = FP8 ? BM * KS : W_BYTES;       // bytes of one weight box in the ring
-  static constexpr int SLOT = W_IN + HP_BYTES;
-  static constexpr int CBUF = STAGES * SLOT;                 // offset of the conversion buffers
-  static constexpr int RING = CBUF + (FP8 ? 2 * W_BYTES : 0);
+  static constexpr int W_IN = FP8 ? W8_BYTES : W_BYTES;            // bytes of one weight stage
+  static constexpr int W_STRIDE = FP8 ? W8_BYTES : W_BYTES + HP_BYTES;
+  static constexpr int T_BASE = FP8 ? STAGES * W8_BYTES : W_BYTES;  // token slot 0
+  static constexpr int T_STRIDE = FP8 ? HP_BYTES : W_BYTES + HP_BYTES;
+  static constexpr int RING = STAGES * (W_IN + HP_BYTES);
   static constexpr int THREADS = FP8 ? kThreads + 128 : kThreads;
+  static constexpr int KSTAGE = FP8 ? KS8 : KS;                      // k per weight stage
+  static constexpr uint32_t TMEM = FP8 ? TMEM_COLS8 : TMEM_COLS;
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(RING) + sizeof(Ctrl);
-  static_assert(SLOT % 1024 == 0 && W_IN % 1024 == 0, "swizzled operands need 1024-byte alignment");
+  static_assert(W_STRIDE % 1024 == 0 && T_BASE % 1024 == 0 && T_STRIDE % 1024 == 0,
+                "swizzled operands need 1024-byte alignment");
   static_assert(SMEM <= 227 * 1024, "ring + control block exceed the 227 KB a B200 CTA may use");
   static_assert(RING >= kRingBytes, "phase-0 scratch must fit in the ring");
 };
@@ -273,12 +284,16 @@ __device__ __forceinline__ void drain_ring(uint64_t* bars, int armed) {
 // ------------------------------------------------------------------------------------------
 // shared setup: barriers and TMEM; unit and range tables from C.off
 // ------------------------------------------------------------------------------------------
+// empty[]: bf16, the MMAs' commit frees the whole slot; fp8, the four converter warps free the weight
+// box (tok_empty[] takes the MMAs' commit).
+template <bool FP8>
 __device__ __forceinline__ void init_ctrl(Ctrl& C) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&C.full_w[s], 1);
       mbar_init(&C.full_t[s], 1);
-      mbar_init(&C.empty[s], 1);
+      mbar_init(&C.empty[s], FP8 ? 4 : 1);
+      mbar_init(&C.tok_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&C.tfull[b], 1);
@@ -287,16 +302,13 @@ __device__ __forceinline__ void init_ctrl(Ctrl& C) {
     mbar_init(&C.drain, 1);
     mbar_init(&C.rbar[0], 1);
     mbar_init(&C.rbar[1], 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&C.cfull[b], 4);    // one arrival per converter warp
-      mbar_init(&C.cempty[b], 1);   // tcgen05.commit of the stage's MMAs
-    }
+    for (int b = 0; b < 2; ++b) mbar_init(&C.afull[b], 4);   // one arrival per converter warp
     C.abort = 0;
     C.bad = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if ((threadIdx.x >> 5) == 1) tmem_alloc(&C.tmem_base, TMEM_COLS);
+  if ((threadIdx.x >> 5) == 1) tmem_alloc(&C.tmem_base, Lay<FP8>::TMEM);
 }
 
 // Needs C.off; ends with a CTA barrier.  Sets C.bad when the offsets are not a monotone split of
@@ -353,7 +365,11 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
     if (lane == 0) {
       const bool wt = warp == 0;
       uint64_t* full = wt ? C.full_w : C.full_t;
-      int q = 0;            // stages armed on `full`
+      // bf16: one token slice per weight stage, in the weight box's slot; fp8: two (one per 128 k of
+      // the 256-k box), in the token ring, freed by the MMAs while the converters free the box
+      uint64_t* freed = (wt || !FP8) ? C.empty : C.tok_empty;
+      const int per = (FP8 && !wt) ? 2 : 1;
+      int q = 0;            // loads armed on `full`
       bool ok = true;
       int ready_e = -1;     // last expert whose phase-A units were all seen complete
       if (!wt && p.x_ready) {
@@ -372,48 +388,48 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
         for (int i = 0; i < P.n && ok; ++i) {
           const Seg g = seg_at(P, i);
           const Unit U = unit_of(C, ph, E, g.u);
-          for (int j = g.j0; j < g.j1; ++j) {
-            const int slot = q % STAGES;
-            const uint32_t epar = static_cast<uint32_t>((q / STAGES) & 1) ^ 1u;
-            if (!mbar_wait(&C.empty[slot], epar, abort_flag, kTimeoutNs)) {
-              ok = false;
-              break;
-            }
-            unsigned char* dst = base + slot * LY::SLOT;
-            if (wt) {
-              mbar_expect_tx(&full[slot], LY::W_IN);
-              if (FP8) {
-                if (ph == 0)
-                  tma_load_2d(dst, (j & 1) ? mWu : mWg, &full[slot], (j >> 1) * KS, U.e * p.f + U.rb * BM);
-                else
-                  tma_load_2d(dst, mWd, &full[slot], j * KS, U.e * p.d + U.rb * BM);
-              } else if (ph == 0) {
-                tma_load_3d(dst, (j & 1) ? mWu : mWg, &full[slot], 0, U.e * p.f + U.rb * BM, (j >> 1) * CH);
-              } else {
-                tma_load_3d(dst, mWd, &full[slot], 0, U.e * p.d + U.rb * BM, j * CH);
-              }
-            } else if (ph == 0) {
-              mbar_expect_tx(&full[slot], X_BYTES);
-              tma_load_3d(dst + LY::W_IN, mX, &full[slot], 0, U.row0, (j >> 1) * CH);
-            } else {
-              if (U.e != ready_e) {
-                // every phase-A unit of expert e must have stored its h rows
-                const unsigned int target = static_cast<unsigned int>(C.ustart[0][U.e + 1] - C.ustart[0][U.e]);
-                const uint64_t t0 = globaltimer();
-                for (uint32_t it = 0; ld_acquire(p.ready + U.e) < target; ++it) {
-                  if ((it & 15) == 15 && (*abort_flag || globaltimer() - t0 > kTimeoutNs)) {
-                    ok = false;
-                    break;
-                  }
+          for (int j = g.j0; j < g.j1 && ok; ++j) {
+            if (!wt && ph == 1 && U.e != ready_e) {
+              // every phase-A unit of expert e must have stored its h rows
+              const unsigned int target = static_cast<unsigned int>(C.ustart[0][U.e + 1] - C.ustart[0][U.e]);
+              const uint64_t t0 = globaltimer();
+              for (uint32_t it = 0; ld_acquire(p.ready + U.e) < target; ++it) {
+                if ((it & 15) == 15 && (*abort_flag || globaltimer() - t0 > kTimeoutNs)) {
+                  ok = false;
+                  break;
                 }
-                if (!ok) break;
-                ready_e = U.e;
-                asm volatile("fence.proxy.async.global;" ::: "memory");
               }
-              mbar_expect_tx(&full[slot], HP_BYTES);
-              tma_load_4d(dst + LY::W_IN, mH, &full[slot], 0, U.row0, 0, j * CH);
+              if (!ok) break;
+              ready_e = U.e;
+              asm volatile("fence.proxy.async.global;" ::: "memory");
             }
-            ++q;
+            for (int hs = 0; hs < per; ++hs, ++q) {
+              const int slot = q % STAGES;
+              const uint32_t epar = static_cast<uint32_t>((q / STAGES) & 1) ^ 1u;
+              if (!mbar_wait(&freed[slot], epar, abort_flag, kTimeoutNs)) {
+                ok = false;
+                break;
+              }
+              if (wt) {
+                unsigned char* dst = base + slot * LY::W_STRIDE;
+                mbar_expect_tx(&full[slot], LY::W_IN);
+                // bf16: [2 chunks of 64 k][128 rows][128 B]; fp8: [2 chunks of 128 k][128 rows][128 B]
+                const int kc = (ph == 0 ? (j >> 1) : j) * CH;
+                const CUtensorMap* mw = ph == 1 ? mWd : ((j & 1) ? mWu : mWg);
+                tma_load_3d(dst, mw, &full[slot], 0, U.e * (ph == 0 ? p.f : p.d) + U.rb * BM, kc);
+              } else {
+                unsigned char* dst = base + LY::T_BASE + slot * LY::T_STRIDE;
+                // the 128-k block of this slice: the stage's own (bf16), or half hs of the stage (fp8)
+                const int kb = (ph == 0 ? (j >> 1) : j) * per + hs;
+                if (ph == 0) {
+                  mbar_expect_tx(&full[slot], X_BYTES);
+                  tma_load_3d(dst, mX, &full[slot], 0, U.row0, kb * CH);
+                } else {
+                  mbar_expect_tx(&full[slot], HP_BYTES);
+                  tma_load_4d(dst, mH, &full[slot], 0, U.row0, 0, kb * CH);
+                }
+              }
+            }
           }
         }
       }
@@ -422,73 +438,77 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
     }
   } else if (warp == 1) {
     // ===================================== MMA issuer =====================================
-    if (lane == 0) {
-      int q = 0;     // stages consumed
-      int seg = 0;   // segments (accumulator uses)
-      bool ok = true;
-      for (int ph = 0; ph < 2 && ok; ++ph) {
-        const Plan P = make_plan(C.rlo[ph][cta], C.rlo[ph][cta + 1], S[ph]);
-        for (int i = 0; i < P.n && ok; ++i) {
-          const Seg g = seg_at(P, i);
-          const int b = seg & 1;
-          if (!mbar_wait(&C.tempty[b], static_cast<uint32_t>((seg >> 1) & 1) ^ 1u, abort_flag, kTimeoutNs)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          for (int j = g.j0; j < g.j1; ++j, ++q) {
+    // The whole warp walks the schedule, so that its waits and descriptors stay warp-uniform; one elected
+    // lane issues.  An M = 128, N <= 64 MMA costs the issuing thread about as much as it costs the tensor
+    // core, so the instruction count is what is kept low: phase B takes h_hi and h_lo as one N = 32
+    // operand (its two 16-column halves are summed by the epilogue), and a (sub-)stage ends with a
+    // single commit.
+    int q = 0;     // bf16: stages consumed; fp8: 128-k sub-stages consumed (two per stage)
+    int seg = 0;   // segments (accumulator uses)
+    bool ok = true;
+    for (int ph = 0; ph < 2 && ok; ++ph) {
+      const Plan P = make_plan(C.rlo[ph][cta], C.rlo[ph][cta + 1], S[ph]);
+      // token operand: phase A the x slice ([chunk][16 rows][128 B]), phase B the h pair ([chunk][32 rows])
+      const uint32_t bchunk = static_cast<uint32_t>(ph == 0 ? NT * 128 : 2 * NT * 128);
+      const uint32_t idesc = FP8 ? (ph == 0 ? kIdescF16 : kIdescF16x32) : (ph == 0 ? kIdesc : kIdesc32);
+      for (int i = 0; i < P.n && ok; ++i) {
+        const Seg g = seg_at(P, i);
+        const int b = seg & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&C.tempty[b], static_cast<uint32_t>((seg >> 1) & 1) ^ 1u, abort_flag,
+                                               kTimeoutNs));
+        if (!ok) break;
+        tc_fence_after();
+        for (int j = g.j0; j < g.j1 && ok; ++j) {
+          // phase A: gate and up stages alternate; the first stage of each matrix in the segment is one of
+          // the first two, and its first MMA overwrites that accumulator
+          const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * 32 + (ph == 0 ? (j & 1) * 16 : 0));
+          const bool fresh = ph == 0 ? j - g.j0 < 2 : j == g.j0;
+          for (int hs = 0; hs < (FP8 ? 2 : 1); ++hs, ++q) {
             const int slot = q % STAGES;
             const uint32_t par = static_cast<uint32_t>((q / STAGES) & 1);
-            const int cb = q & 1;   // fp8: the conversion buffer holding this stage's f16 weights
-            if (!mbar_wait(FP8 ? &C.cfull[cb] : &C.full_w[slot], FP8 ? static_cast<uint32_t>((q >> 1) & 1) : par,
-                           abort_flag, kTimeoutNs) ||
-                !mbar_wait(&C.full_t[slot], par, abort_flag, kTimeoutNs)) {
-              ok = false;
-              break;
-            }
+            bool got = mbar_wait(FP8 ? &C.afull[q & 1] : &C.full_w[slot], FP8 ? static_cast<uint32_t>((q >> 1) & 1) : par,
+                                 abort_flag, kTimeoutNs);
+            got = got && mbar_wait(&C.full_t[slot], par, abort_flag, kTimeoutNs);
+            ok = __all_sync(0xffffffffu, got);
+            if (!ok) break;
             tc_fence_after();
-            const uint32_t sa = FP8 ? smem_u32(base + LY::CBUF + cb * W_BYTES) : smem_u32(base + slot * LY::SLOT);
-            const uint32_t sb = smem_u32(base + slot * LY::SLOT + LY::W_IN);
-            constexpr uint32_t idesc = FP8 ? kIdescF16 : kIdesc;
-            if (ph == 0) {
-              // gate and up stages alternate: the first stage of each matrix in the segment is one of
-              // the first two, and its first MMA overwrites that accumulator
-              const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * 32 + (j & 1) * 16);
-              const bool fresh = j - g.j0 < 2;
+            const uint64_t db = sw128_desc(smem_u32(base + LY::T_BASE + slot * LY::T_STRIDE));
+            if (elect_one()) {
+              if (FP8) {
+                // 16 k per MMA: 8 TMEM columns of the A tile
+                const uint32_t ta = tmem + kTmemA + static_cast<uint32_t>((q & 1) * 64);
 #pragma unroll
-              for (int c = 0; c < CH; ++c)
+                for (int kk = 0; kk < 8; ++kk)
+                  umma_tmem_a(d_tmem, ta + static_cast<uint32_t>(kk * 8),
+                              db + (((kk >> 2) * bchunk + (kk & 3) * 32) >> 4), idesc,
+                              (fresh && hs == 0 && kk == 0) ? 0u : 1u);
+                umma_commit(&C.tok_empty[slot]);
+              } else {
+                const uint64_t da = sw128_desc(smem_u32(base + slot * LY::W_STRIDE));
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  umma_bf16(d_tmem, sw128_desc(sa + c * (BM * 128) + kk * 32), sw128_desc(sb + c * (NT * 128) + kk * 32),
-                            idesc, (fresh && c == 0 && kk == 0) ? 0u : 1u);
-            } else {
-              // h_hi and h_lo slices of chunk c sit at 2c and 2c + 1 (2 KB each)
-              const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * 32);
-              const bool fresh = j == g.j0;
+                for (int c = 0; c < CH; ++c)
 #pragma unroll
-              for (int c = 0; c < CH; ++c)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const uint64_t ad = sw128_desc(sa + c * (BM * 128) + kk * 32);
-                  umma_bf16(d_tmem, ad, sw128_desc(sb + (2 * c) * (NT * 128) + kk * 32), idesc,
-                            (fresh && c == 0 && kk == 0) ? 0u : 1u);
-                  umma_bf16(d_tmem, ad, sw128_desc(sb + (2 * c + 1) * (NT * 128) + kk * 32), idesc, 1u);
-                }
+                  for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(d_tmem, da + static_cast<uint64_t>((c * (BM * 128) + kk * 32) >> 4),
+                              db + ((c * bchunk + kk * 32) >> 4), idesc, (fresh && c == 0 && kk == 0) ? 0u : 1u);
+                umma_commit(&C.empty[slot]);
+              }
             }
-            umma_commit(&C.empty[slot]);
-            if (FP8) umma_commit(&C.cempty[cb]);
+            __syncwarp();
           }
-          if (!ok) break;
-          umma_commit(&C.tfull[b]);
-          ++seg;
         }
+        if (!ok) break;
+        if (elect_one()) umma_commit(&C.tfull[b]);
+        __syncwarp();
+        ++seg;
       }
-      if (!ok) set_abort(C, p.timeouts);
-      // every MMA this thread issued completes before the drain barrier flips
-      umma_commit(&C.drain);
-      const uint64_t t1 = globaltimer();
-      while (!mbar_try_wait(&C.drain, 0) && globaltimer() - t1 < kTimeoutNs) {
-      }
+    }
+    if (!ok && lane == 0) set_abort(C, p.timeouts);
+    // every MMA this warp issued completes before the drain barrier flips
+    if (elect_one()) umma_commit(&C.drain);
+    __syncwarp();
+    const uint64_t t1 = globaltimer();
+    while (!mbar_try_wait(&C.drain, 0) && globaltimer() - t1 < kTimeoutNs) {
     }
   } else if (warp >= 2 && warp <= 5) {
     // ===================================== epilogue (warps 2..5) =====================================
@@ -512,15 +532,17 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
         {
           uint32_t r0[16], r1[16];
           tmem_ld16(taddr, r0);
-          if (ph == 0) tmem_ld16(taddr + 16, r1);
+          tmem_ld16(taddr + 16, r1);
           tmem_wait_ld();
-          // a segment without gate (up) stages left that accumulator untouched: it contributes 0
+          // phase A: gate in columns 0..15, up in 16..31; a segment without gate (up) stages left that
+          // accumulator untouched: it contributes 0.  Phase B: W h_hi in columns 0..15, W h_lo in 16..31.
           const bool has_g = ph == 1 || sg.j0 < sg.j1 - 1 || (sg.j0 & 1) == 0;
           const bool has_u = ph == 0 && (sg.j0 < sg.j1 - 1 || (sg.j0 & 1) == 1);
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
-            g[t] = has_g ? __uint_as_float(r0[t]) : 0.f;
-            v[t] = has_u ? __uint_as_float(r1[t]) : 0.f;
+            const float a0 = __uint_as_float(r0[t]), a1 = __uint_as_float(r1[t]);
+            g[t] = ph == 1 ? a0 + a1 : (has_g ? a0 : 0.f);
+            v[t] = has_u ? a1 : 0.f;
           }
         }
         tc_fence_before();
@@ -662,49 +684,69 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
     }
     if (!ok) set_abort(C, p.timeouts);
   } else if (FP8 && warp >= kWarpConv) {
-    // ========================= fp8 converters (warps 7..10): E4M3 box -> f16 tile =========================
-    // Each warp expands 4 rows per step (rows 4 cw + 16 i + lane / 8): lane l takes the 16-byte segment
-    // l % 8 of its 128-byte code row (k = 16 (l % 8) .. + 15) and writes the 16 f16 values, two 16-byte
-    // units, into chunk (l % 8) / 4 of the swizzled tile.
-    const int cw = warp - kWarpConv;
-    const int rsub = lane >> 3, sgm = lane & 7;
-    const int c = sgm >> 2, u0 = (sgm & 3) * 2;
-    int q = 0;
+    // ===================== fp8 converters (warps 7..10): E4M3 box -> f16 A tile in TMEM =====================
+    // A thread expands one weight row, row 32 (warp % 4) + lane: the TMEM lane its warp may write.  For
+    // each 128-k half of the 256-k box it reads the row's eight 16-byte units (128-byte swizzle: unit u
+    // of row r at u ^ (r % 8), so a quarter-warp's reads hit distinct banks), converts them to 64 f16
+    // pairs and stores those into A tile q % 2.  Wait outcomes are made warp-uniform: the TMEM stores
+    // are warp-collective.
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kTmemA;
+    int q = 0;   // weight stages
     bool ok = true;
     for (int ph = 0; ph < 2 && ok; ++ph) {
       const Plan P = make_plan(C.rlo[ph][cta], C.rlo[ph][cta + 1], S[ph]);
       for (int i = 0; i < P.n && ok; ++i) {
         const Seg g = seg_at(P, i);
-        for (int j = g.j0; j < g.j1; ++j, ++q) {
-          const int slot = q % STAGES, cb = q & 1;
-          if (!mbar_wait(&C.full_w[slot], static_cast<uint32_t>((q / STAGES) & 1), abort_flag, kTimeoutNs) ||
-              !mbar_wait(&C.cempty[cb], static_cast<uint32_t>((q >> 1) & 1) ^ 1u, abort_flag, kTimeoutNs)) {
-            ok = false;
-            break;
+        for (int j = g.j0; j < g.j1 && ok; ++j, ++q) {
+          const int slot = q % STAGES;
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(&C.full_w[slot], static_cast<uint32_t>((q / STAGES) & 1), abort_flag, kTimeoutNs));
+          if (!ok) break;
+          const unsigned char* box = base + slot * LY::W_STRIDE + r * 128;
+          for (int hs = 0; hs < 2 && ok; ++hs) {
+            const int q2 = 2 * q + hs, ab = q2 & 1;
+            // A tile ab last held sub-stage q2 - 2: its MMAs are done once that sub-stage's commit (on its
+            // token slot) has landed.  That barrier cannot have moved on by a further phase: the next one
+            // needs sub-stage q2 + 3.
+            if (q2 >= 2) {
+              const int prev = q2 - 2;
+              ok = __all_sync(0xffffffffu, mbar_wait(&C.tok_empty[prev % STAGES],
+                                                     static_cast<uint32_t>((prev / STAGES) & 1), abort_flag,
+                                                     kTimeoutNs));
+              if (!ok) break;
+            }
+            tc_fence_after();
+            const unsigned char* row = box + hs * (BM * 128);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint32_t v[32];
+#pragma unroll
+              for (int uu = 0; uu < 4; ++uu) {
+                const int u = half * 4 + uu;
+                const uint4 wv = *reinterpret_cast<const uint4*>(row + ((u ^ (r & 7)) << 4));
+                v[uu * 8 + 0] = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.x));
+                v[uu * 8 + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.x >> 16));
+                v[uu * 8 + 2] = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.y));
+                v[uu * 8 + 3] = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.y >> 16));
+                v[uu * 8 + 4] = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.z));
+                v[uu * 8 + 5] = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.z >> 16));
+                v[uu * 8 + 6] = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.w));
+                v[uu * 8 + 7] = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.w >> 16));
+              }
+              tmem_st32(trow + static_cast<uint32_t>(ab * 64 + half * 32), v);
+            }
+            if (hs == 1) {
+              // the whole box is in registers or TMEM: its slot may refill
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&C.empty[slot]);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&C.afull[ab]);
           }
-          const unsigned char* src = base + slot * LY::SLOT;
-          unsigned char* dst = base + LY::CBUF + cb * W_BYTES;
-#pragma unroll 2
-          for (int r0 = cw * 4; r0 < BM; r0 += 16) {
-            const int r = r0 + rsub;
-            const uint4 wv = *reinterpret_cast<const uint4*>(src + r * 128 + sgm * 16);
-            uint4 o0, o1;
-            o0.x = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.x));
-            o0.y = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.x >> 16));
-            o0.z = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.y));
-            o0.w = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.y >> 16));
-            o1.x = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.z));
-            o1.y = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.z >> 16));
-            o1.z = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.w));
-            o1.w = e4m3x2_to_f16x2(static_cast<uint16_t>(wv.w >> 16));
-            unsigned char* rowp = dst + c * (BM * 128) + r * 128;
-            *reinterpret_cast<uint4*>(rowp + ((u0 ^ (r & 7)) << 4)) = o0;
-            *reinterpret_cast<uint4*>(rowp + (((u0 + 1) ^ (r & 7)) << 4)) = o1;
-          }
-          // generic-proxy writes, read next by the tensor core (async proxy)
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&C.cfull[cb]);
         }
       }
     }
@@ -722,9 +764,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  Ctrl& C = *reinterpret_cast<Ctrl*>(base + STAGES * STAGE_BYTES);
+  Ctrl& C = *reinterpret_cast<Ctrl*>(base + Lay<false>::RING);
   const int S[2] = {2 * (p.d / KS), p.f / KS};   // stages per unit; phase A alternates gate / up along k
-  init_ctrl(C);
+  init_ctrl<false>(C);
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) C.off[i] = p.offsets[i];
   __syncthreads();
   build_tables(C, p, S);
@@ -780,21 +822,6 @@ __device__ __forceinline__ float block_sum(float v, Ctrl& C) {
   }
   __syncthreads();
   return C.red[nwarps()];
-}
-
-// Larger score first, then lower expert index.
-__device__ __forceinline__ bool better(float s, int e, float s2, int e2) { return s > s2 || (s == s2 && e < e2); }
-
-__device__ __forceinline__ void warp_argmax(float& s, int& e) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float so = __shfl_xor_sync(0xffffffffu, s, o);
-    const int eo = __shfl_xor_sync(0xffffffffu, e, o);
-    if (better(so, eo, s, e)) {
-      s = so;
-      e = eo;
-    }
-  }
 }
 
 // Phase 0a scratch in the ring (byte offsets; all multiples of 16).
@@ -1109,8 +1136,9 @@ __global__ void __launch_bounds__(Lay<FP8>::THREADS, 1)
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   Ctrl& C = *reinterpret_cast<Ctrl*>(base + Lay<FP8>::RING);
-  const int S[2] = {2 * (p.d / KS), p.f / KS};
-  init_ctrl(C);
+  // stages per unit (phase A alternates gate / up along k)
+  const int S[2] = {2 * (p.d / Lay<FP8>::KSTAGE), p.f / Lay<FP8>::KSTAGE};
+  init_ctrl<FP8>(C);
   __syncthreads();
   // the ring is idle until the SwiGLU roles start: phase 0 keeps its scratch there
   int* ids = reinterpret_cast<int*>(base);
@@ -1157,7 +1185,7 @@ __global__ void __launch_bounds__(Lay<FP8>::THREADS, 1)
   __syncthreads();
   if ((threadIdx.x >> 5) == 1) {
     tc_fence_after();
-    tmem_dealloc(C.tmem_base, TMEM_COLS);
+    tmem_dealloc(C.tmem_base, Lay<FP8>::TMEM);
   }
 }
 
@@ -1354,15 +1382,16 @@ zmoe_status moe_layer_fused(const uint16_t* x, const float* h_in, const float* g
   bool okm = encode_maps(&m, xp, n, static_cast<const uint16_t*>(w_gate), static_cast<const uint16_t*>(w_up),
                          static_cast<const uint16_t*>(w_down), E, d, f, hh);
   if (okm && fp8) {
-    // E4M3 codes [rows][K]: a 128-row x 128-byte box, unswizzled (the converter warps swizzle)
-    const cuuint64_t dg[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(E) * f};
-    const cuuint64_t sg[1] = {static_cast<cuuint64_t>(d)};
-    const cuuint64_t dd[2] = {static_cast<cuuint64_t>(f), static_cast<cuuint64_t>(E) * d};
-    const cuuint64_t sd[1] = {static_cast<cuuint64_t>(f)};
-    const cuuint32_t box[2] = {KS, BM};
-    okm = encode_map(&m.g, w_gate, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, dg, sg, box, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-          encode_map(&m.u, w_up, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, dg, sg, box, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-          encode_map(&m.dn, w_down, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, dd, sd, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+    // E4M3 codes viewed as [K/128 chunks][rows][128]: a box of 128 rows x 2 chunks (256 k, 32 KB) lands
+    // as [chunk][row][128 B] in the 128-byte swizzle, the layout the converter warps read
+    const cuuint64_t dg[3] = {128, static_cast<cuuint64_t>(E) * f, static_cast<cuuint64_t>(d) / 128};
+    const cuuint64_t sg[2] = {static_cast<cuuint64_t>(d), 128};
+    const cuuint64_t dd[3] = {128, static_cast<cuuint64_t>(E) * d, static_cast<cuuint64_t>(f) / 128};
+    const cuuint64_t sd[2] = {static_cast<cuuint64_t>(f), 128};
+    const cuuint32_t box[3] = {128, BM, KS8 / 128};
+    okm = encode_map(&m.g, w_gate, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, dg, sg, box, CU_TENSOR_MAP_SWIZZLE_128B) &&
+          encode_map(&m.u, w_up, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, dg, sg, box, CU_TENSOR_MAP_SWIZZLE_128B) &&
+          encode_map(&m.dn, w_down, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, dd, sd, box, CU_TENSOR_MAP_SWIZZLE_128B);
   }
   if (!okm) return fail(ZMOE_ERR_CUDA, "zmoe_moe_layer: cuTensorMapEncodeTiled failed");
   if (cudaMemsetAsync(ws, 0, W.ffn.counters_end, s) != cudaSuccess)
