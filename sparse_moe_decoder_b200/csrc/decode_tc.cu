@@ -66,8 +66,11 @@ constexpr int kWarpConv = 7;                  // fp8: warps 7..10 expand weight 
 constexpr int KS8 = 256;                      // fp8: k per weight stage (two f16 sub-stages of KS)
 constexpr int W8_BYTES = BM * KS8;            // 32 KB of E4M3 codes
 constexpr uint32_t TMEM_COLS = 64;            // 2 accumulator buffers x (gate 16 | up 16)
-constexpr uint32_t TMEM_COLS8 = 256;          // fp8: the accumulators, then 2 f16 A tiles of 64 columns
+constexpr int kATiles = 4;                    // fp8: f16 A tiles in TMEM (the converters run this far ahead)
+constexpr uint32_t TMEM_COLS8 = 512;          // fp8: the accumulators, then kATiles A tiles of 64 columns
 constexpr uint32_t kTmemA = 64;               // fp8: first column of A tile 0 (128 k of f16, 2 per column)
+static_assert(kTmemA + 64 * kATiles <= TMEM_COLS8, "A tiles must fit in the TMEM allocation");
+static_assert(kATiles < STAGES, "an A tile's reuse waits on a token-slot barrier that must not run a phase ahead");
 constexpr int kMaxE = 64;
 constexpr int kMaxCtas = 256;
 constexpr int kMaxAssign = 1024;              // T * k of the fused layer
@@ -146,7 +149,7 @@ struct __align__(16) Ctrl {
   uint64_t rbar[2];          // fused layer: router matrix (+ gamma), token row
   uint64_t tok_empty[STAGES];  // fp8: token slot consumed by the MMAs (bf16: one slot with the weights);
                                // its commit also frees the sub-stage's A tile
-  uint64_t afull[2];         // fp8: f16 A tile written to TMEM by the converter warps
+  uint64_t afull[kATiles];   // fp8: f16 A tile written to TMEM by the converter warps
   uint32_t tmem_base;
   int abort;
   int bad;
@@ -302,7 +305,7 @@ __device__ __forceinline__ void init_ctrl(Ctrl& C) {
     mbar_init(&C.drain, 1);
     mbar_init(&C.rbar[0], 1);
     mbar_init(&C.rbar[1], 1);
-    for (int b = 0; b < 2; ++b) mbar_init(&C.afull[b], 4);   // one arrival per converter warp
+    for (int b = 0; b < kATiles; ++b) mbar_init(&C.afull[b], 4);   // one arrival per converter warp
     C.abort = 0;
     C.bad = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -347,9 +350,8 @@ __device__ __forceinline__ void build_tables(Ctrl& C, const DecArgs& p, const in
 // ------------------------------------------------------------------------------------------
 // the SwiGLU roles (both kernels)
 // ------------------------------------------------------------------------------------------
-// FP8: weight boxes arrive as E4M3 codes [128 rows][128 B] (no swizzle); warps 7..10 expand each into
-// an f16 tile in the K-major 128-byte-swizzle layout ([chunk][row][128 B]) that the MMA reads, tokens
-// are f16, and the row scales multiply the finished sums.
+// FP8: weight boxes arrive as E4M3 codes (128 rows x 256 k); warps 7..10 expand each 128-k half into an
+// f16 A tile in TMEM that the MMAs read, tokens are f16, and the row scales multiply the finished sums.
 template <bool FP8>
 __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensorMap* mWu, const CUtensorMap* mWd,
                                           const CUtensorMap* mX, const CUtensorMap* mH, const DecArgs& p, Ctrl& C,
@@ -466,8 +468,8 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
           for (int hs = 0; hs < (FP8 ? 2 : 1); ++hs, ++q) {
             const int slot = q % STAGES;
             const uint32_t par = static_cast<uint32_t>((q / STAGES) & 1);
-            bool got = mbar_wait(FP8 ? &C.afull[q & 1] : &C.full_w[slot], FP8 ? static_cast<uint32_t>((q >> 1) & 1) : par,
-                                 abort_flag, kTimeoutNs);
+            bool got = mbar_wait(FP8 ? &C.afull[q % kATiles] : &C.full_w[slot],
+                                 FP8 ? static_cast<uint32_t>((q / kATiles) & 1) : par, abort_flag, kTimeoutNs);
             got = got && mbar_wait(&C.full_t[slot], par, abort_flag, kTimeoutNs);
             ok = __all_sync(0xffffffffu, got);
             if (!ok) break;
@@ -476,7 +478,7 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
             if (elect_one()) {
               if (FP8) {
                 // 16 k per MMA: 8 TMEM columns of the A tile
-                const uint32_t ta = tmem + kTmemA + static_cast<uint32_t>((q & 1) * 64);
+                const uint32_t ta = tmem + kTmemA + static_cast<uint32_t>((q % kATiles) * 64);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                   umma_tmem_a(d_tmem, ta + static_cast<uint32_t>(kk * 8),
@@ -688,8 +690,8 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
     // A thread expands one weight row, row 32 (warp % 4) + lane: the TMEM lane its warp may write.  For
     // each 128-k half of the 256-k box it reads the row's eight 16-byte units (128-byte swizzle: unit u
     // of row r at u ^ (r % 8), so a quarter-warp's reads hit distinct banks), converts them to 64 f16
-    // pairs and stores those into A tile q % 2.  Wait outcomes are made warp-uniform: the TMEM stores
-    // are warp-collective.
+    // pairs and stores those into the next of the kATiles A tiles.  Wait outcomes are made warp-uniform:
+    // the TMEM stores are warp-collective.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kTmemA;
@@ -706,12 +708,12 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
           if (!ok) break;
           const unsigned char* box = base + slot * LY::W_STRIDE + r * 128;
           for (int hs = 0; hs < 2 && ok; ++hs) {
-            const int q2 = 2 * q + hs, ab = q2 & 1;
-            // A tile ab last held sub-stage q2 - 2: its MMAs are done once that sub-stage's commit (on its
-            // token slot) has landed.  That barrier cannot have moved on by a further phase: the next one
-            // needs sub-stage q2 + 3.
-            if (q2 >= 2) {
-              const int prev = q2 - 2;
+            const int q2 = 2 * q + hs, ab = q2 % kATiles;
+            // A tile ab last held sub-stage q2 - kATiles: its MMAs are done once that sub-stage's commit (on
+            // its token slot) has landed.  That barrier cannot have moved on by a further phase: the next
+            // one needs sub-stage q2 - kATiles + STAGES > q2.
+            if (q2 >= kATiles) {
+              const int prev = q2 - kATiles;
               ok = __all_sync(0xffffffffu, mbar_wait(&C.tok_empty[prev % STAGES],
                                                      static_cast<uint32_t>((prev / STAGES) & 1), abort_flag,
                                                      kTimeoutNs));
@@ -1086,16 +1088,18 @@ __device__ __forceinline__ void permute_all(const LayerArgs& L, const DecArgs& p
   }
   __syncthreads();
   const int rows = C.off[E];
-  if (blockIdx.x == 0) {
+  // the routing outputs: by the last CTA, which holds no x_perm row while rows < grid size
+  if (blockIdx.x == gridDim.x - 1) {
     for (int i = threadIdx.x; i < E; i += nthreads()) L.counts[i] = C.run[i];
     for (int i = threadIdx.x; i <= E; i += nthreads()) L.offsets[i] = C.off[i];
     for (int i = threadIdx.x; i < rows; i += nthreads()) L.perm[i] = C.rowsrc[i];
     for (int i = threadIdx.x; i < n; i += nthreads()) L.inv_perm[i] = C.invp[i];
   }
-  // x_perm rows, one warp per row, spread over the grid
+  // x_perm rows, one warp per row, one row per CTA before any CTA takes a second: a CTA still gathering
+  // when the others start streaming weights sees its loads and stores queue behind theirs
   const uint16_t* xsrc = L.gamma ? L.x_norm : L.x_in;
   const int vecs = p.d / 8;
-  for (int r = blockIdx.x * nwarps() + warp; r < rows; r += gridDim.x * nwarps()) {
+  for (int r = blockIdx.x + gridDim.x * warp; r < rows; r += gridDim.x * nwarps()) {
     const uint4* s = reinterpret_cast<const uint4*>(xsrc + static_cast<size_t>(C.rowsrc[r]) * p.d);
     uint4* dst = reinterpret_cast<uint4*>(L.x_perm + static_cast<size_t>(r) * p.d);
     for (int v0 = 0; v0 < vecs; v0 += 32 * 8) {
