@@ -249,13 +249,13 @@ ZMOE_API zmoe_status zmoe_moe_layer(const void* x, const float* h, const float* 
 ZMOE_API size_t zmoe_moe_layer_fp8_workspace_size(int T, int d, int f, int E, int k);
 
 /*
- * zmoe_moe_layer with fp8 expert weights (the pages' serving stack runs the model in fp8:
- * sglang-omni cookbook, "Hardware / deployment"): each expert weight row is stored as E4M3 codes
- * (bias 7, no infinities) with one fp32 scale, w = code * scale.  The router stays in bf16.
+ * zmoe_moe_layer with fp8 expert weights (the pages' serving stack runs the model in fp8: ZONOS2
+ * page of the sglang-omni cookbook, "Benchmark Results"): each expert weight row is stored as E4M3
+ * codes (bias 7, no infinities) with one fp32 scale, w = code * scale.  The router stays in bf16.
  *   q_gate, q_up: uint8 [E, f, d]; q_down: uint8 [E, d, f]; s_gate, s_up: f32 [E, f]; s_down: f32 [E, d].
  *   Other arguments, outputs and conventions as zmoe_moe_layer with dtype ZMOE_BF16.
  * Decode sizes only (T * k < 64 E, T * k <= 1024, d and f multiples of 256): one cooperative
- * launch streams the codes (half the bf16 bytes), expands them to f16 in shared memory and runs
+ * launch streams the codes (half the bf16 bytes), expands them to f16 in tensor memory and runs
  * f16 x f16 tensor-core contractions with fp32 accumulation, so the layer input and the hidden
  * activations are carried in f16 there: values beyond f16's range (|v| > 65504) count a device
  * error.  Larger sizes return ZMOE_ERR_UNSUPPORTED.

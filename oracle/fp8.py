@@ -1,6 +1,7 @@
 """fp8 expert weights (test infrastructure only: the oracle).
 
-The ZONOS2 serving stack runs the model in fp8 (sglang-omni cookbook page, "Hardware / deployment").
+The ZONOS2 serving stack runs the model in fp8 (ZONOS2 page of the sglang-omni cookbook, "Benchmark
+Results": the measured serving configuration is fp8).
 Reading taken: expert weights stored as E4M3 codes (sign, 4 exponent bits with bias 7, 3 mantissa
 bits; exponent field 0 = subnormals m 2^-9; no infinities; 0x7F / 0xFF are NaN) with one fp32 scale
 per output row, w = decode(code) * scale.  The layer is then the bf16 layer's arithmetic on the
