@@ -560,7 +560,7 @@ def run_fp8(args):
                        "l2": f"fp8 weights rotated over {n_copies} device copies ({n_copies * 0.302:.1f} GB > 126 MB L2)",
                        "experts_touched": touched},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_from_profiles("moe_layer_fp8_cfg7"),
                          "kernel": "moe_layer_kernel<fp8>: router, dispatch, fp8 SwiGLU and combine in one launch",
                          "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"]},
             "cpu_baseline": cpu,
