@@ -24,8 +24,11 @@
 //     5-stage ring (200 KB: 160 KB of weights in flight per SM; boxes of 32 KB or more keep one
 //     SM's TMA near full HBM rate; 5 x 32 KB measured 2% faster than 2 x 64 KB on the decode step),
 //     each completing on its own mbarrier, so weight loads never wait for h; warp 1 allocates TMEM
-//     and issues the MMAs from one thread (tcgen05.commit frees a stage when its MMAs are done);
-//     warps 2..5 read the accumulators with tcgen05.ld and run the epilogues.
+//     and issues the MMAs from one elected lane (tcgen05.commit frees a stage when its MMAs are
+//     done); warps 2..5 read the accumulators with tcgen05.ld and run the epilogues.
+//   * fp8 weights (E4M3 codes, one fp32 scale per row): 32 KB boxes of 128 rows x 256 k in a ring of
+//     their own; warps 7..10 expand each 128-k half into an f16 A tile in TMEM, the MMAs read A from
+//     TMEM, the tokens and the h pair are f16, and the row scales multiply the finished sums.
 //   * Phase-A units of expert e release-increment ready[e]; the token producer acquires ready[e]
 //     before loading h rows of expert e (cross-proxy fence before the TMA).
 //   * Every wait is bounded (time limit): on expiry the CTA counts a device timeout, aborts,

@@ -75,6 +75,30 @@ def test_bad_arguments_rejected_on_host(L, call):
     assert len(L.zmoe_last_error()) > 0
 
 
+def _fp8_layer(L, T=4, d=256, f=256, E=16, k=1, x=0x1000, h=NULL, gamma=NULL, w_router=0x2000, q_gate=0x3000,
+               y=0x4000):
+    """zmoe_moe_layer_fp8 with placeholder (never dereferenced) 16-byte-aligned pointers by default."""
+    s = 0x5000
+    return L.zmoe_moe_layer_fp8(x, h, gamma, 1e-6, w_router, NULL, NULL, q_gate, s, 0x6000, s, 0x7000, s, T, d, f, E,
+                                k, y, NULL, NULL, NULL, NULL, NULL, 0, NULL)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(T=-1), dict(E=65), dict(E=0), dict(k=3), dict(k=2, E=1), dict(d=384), dict(f=128),
+    dict(q_gate=NULL), dict(y=NULL), dict(w_router=NULL),          # no router with E = 16
+    dict(x=NULL), dict(gamma=0x8000),                              # neither x nor h with gamma
+])
+def test_fp8_layer_bad_arguments_rejected_on_host(L, kw):
+    assert _fp8_layer(L, **kw) == 1   # ZMOE_ERR_INVALID_ARG, nothing launched
+    assert len(L.zmoe_last_error()) > 0
+
+
+def test_fp8_layer_unaligned_and_empty(L):
+    assert _fp8_layer(L, q_gate=0x3000 + 8) == 1
+    assert b"aligned" in L.zmoe_last_error()
+    assert _fp8_layer(L, T=0) == 0     # nothing to do: OK without touching the device
+
+
 def test_unaligned_pointers_rejected(L):
     # 16-byte alignment is checked on the host before any launch (pointer values are never dereferenced)
     p = ctypes.c_void_p(0x1000 + 4)
