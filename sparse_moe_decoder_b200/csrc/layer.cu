@@ -4,10 +4,11 @@
 // ZONOS2 digest items 5-6 (sparse MoE FFN, top-1 / top-2 routing, RMSNorm), the telknet.cc article
 // on ZONOS2, section 2.1 (router, gate-weighted sum of the chosen experts).
 //
-// Decode sizes (bf16, T * k < 64 E and T * k <= 1024) run as ONE cooperative launch
-// (decode_tc.cu: pre-norm + router, grid barrier, dispatch, grid barrier, stream-K SwiGLU with the
-// combine in its epilogue).  Every other size runs the separate entry points in order:
-// zmoe_rmsnorm, zmoe_route, zmoe_permute, zmoe_grouped_swiglu, zmoe_combine.
+// A few tokens (bf16, T * k <= 4) run as one cooperative launch of CUDA-core matrix-vector products
+// without split-k (tiny_layer.cu).  Decode sizes (bf16, T * k < 64 E and T * k <= 1024) run as ONE
+// cooperative launch (decode_tc.cu: pre-norm + router, grid barrier, dispatch, grid barrier,
+// stream-K SwiGLU with the combine in its epilogue).  Every other size runs the separate entry points
+// in order: zmoe_rmsnorm, zmoe_route, zmoe_permute, zmoe_grouped_swiglu, zmoe_combine.
 #include "common.cuh"
 
 namespace zmoe {
@@ -20,7 +21,18 @@ zmoe_status moe_layer_fused(const uint16_t* x, const float* h_in, const float* g
                             float* gates, float* margin, uint16_t* x_norm_out, void* ws, cudaStream_t s,
                             const float* s_gate, const float* s_up, const float* s_down);
 
+bool moe_layer_tiny_supported(int T, int E, int d, int f, int k);
+size_t moe_layer_tiny_workspace(int T, int f, int k);
+zmoe_status moe_layer_tiny(const uint16_t* x, const float* h_in, const float* gamma, float eps, const uint16_t* w_r,
+                           const float* logit_bias, const float* sel_bias, const uint16_t* w_gate, const uint16_t* w_up,
+                           const uint16_t* w_down, int T, int d, int f, int E, int k, float* y, int32_t* expert_idx,
+                           float* gates, float* margin, uint16_t* x_norm, void* ws, cudaStream_t s);
+
 namespace {
+
+bool use_tiny(int T, int E, int d, int f, int k, zmoe_dtype dtype) {
+  return dtype == ZMOE_BF16 && moe_layer_tiny_supported(T, E, d, f, k);
+}
 
 // Rows per expert below which the fused decode launch is used (the grouped SwiGLU's own
 // decode / prefill threshold).
@@ -74,6 +86,7 @@ size_t zmoe_moe_layer_workspace_size(int T, int d, int f, int E, int k, zmoe_dty
   using namespace zmoe;
   if (T < 0 || d < 1 || f < 1 || E < 1 || E > 64 || (k != 1 && k != 2) || !dtype_ok(dtype)) return 0;
   if (T == 0) return 0;
+  if (use_tiny(T, E, d, f, k, dtype)) return moe_layer_tiny_workspace(T, f, k);
   if (use_fused(T, E, d, f, k, dtype)) return moe_layer_fused_workspace(T, E, d, f, k);
   return seq_ws(T, E, d, f, k, dtype).total;
 }
@@ -102,6 +115,11 @@ zmoe_status zmoe_moe_layer(const void* x, const float* h, const float* gamma, fl
     return fail(ZMOE_ERR_WORKSPACE_TOO_SMALL, "zmoe_moe_layer: workspace smaller than zmoe_moe_layer_workspace_size()");
   clear_error();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (use_tiny(T, E, d, f, k, dtype))
+    return moe_layer_tiny(static_cast<const uint16_t*>(x), h, gamma, eps, static_cast<const uint16_t*>(w_router),
+                          logit_bias, sel_bias, static_cast<const uint16_t*>(w_gate), static_cast<const uint16_t*>(w_up),
+                          static_cast<const uint16_t*>(w_down), T, d, f, E, k, y, expert_idx, gates, margin,
+                          static_cast<uint16_t*>(x_norm), workspace, s);
   if (use_fused(T, E, d, f, k, dtype))
     return moe_layer_fused(static_cast<const uint16_t*>(x), h, gamma, eps, static_cast<const uint16_t*>(w_router),
                            logit_bias, sel_bias, w_gate, w_up, w_down, T, d, f, E, k, y, expert_idx, gates, margin,
