@@ -9,7 +9,7 @@ permutation, the SwiGLU and the combine.  Each case is checked on every token:
     of the method, and the oracle consumes the same bf16 values);
   * with the pre-norm, x itself against the fp64 RMSNorm, and the result in place (y aliasing h).
 Shapes span one and several 16-row token blocks per expert, top-1 and top-2, E = 1, an empty
-expert, batch 1, and the full decode-step size.
+expert, batch 1, the tiny-batch launch (T * k <= 4) and its boundary, and the full decode-step size.
 """
 import numpy as np
 import pytest
@@ -140,6 +140,19 @@ def test_fused_repeatable_bitwise():
     first = host(R.run(x, W)).copy()
     for _ in range(3):
         assert np.array_equal(host(R.run(x, W)), first)
+
+
+@pytest.mark.parametrize("T,k", [(2, 2), (4, 1), (2, 1), (5, 1)])
+def test_tiny_batch_layer(T, k):
+    """A few tokens (T * k <= 4 runs the tiny-batch launch, T = 5 the stream-K one): the decode
+    stack's pre-norm layer in place, at the model's dimensions, against the oracle."""
+    require_gpu()
+    L = make_moe_layer(T, 2048, 3072, 16, k, seed=70 + T + k, sel_bias_var=0.1, with_gamma=True, draw_x=False)
+    h = (2.0 * np.random.default_rng(T).standard_normal((T, 2048))).astype(np.float32)
+    R, y, xn = run_fused(L, h_host=h, gamma=L.gamma, in_place=True)
+    assert_close(xn, oracle.rmsnorm(h.astype(np.float64), L.gamma.astype(np.float64), EPS), "bf16", "pre-norm output")
+    r, ex = check_layer(L, h.astype(np.float64), y, host(R.idx), host(R.gates), xn, f"tiny T={T} k={k}")
+    print(f"tiny T={T} k={k}: y-h max err {r:.2e} x RMS, {ex} low-margin tokens")
 
 
 @pytest.mark.parametrize("T", [1, 40, 300])
