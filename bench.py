@@ -437,8 +437,8 @@ def run_stack(args):
                        "experts_touched_per_token": touched, "cuda_graph": used_graph},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                         "kernel": f"whole decode step (embed + {spec.total_layers} x moe_layer_kernel: pre-norm, "
-                                   "router, dispatch, SwiGLU and combine in one launch per layer)",
+                         "kernel": f"whole decode step (embed + {spec.total_layers} x tiny_layer_kernel: pre-norm, "
+                                   "router, SwiGLU and combine in one launch per layer)",
                          "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peaks["source"]},
             "cpu_baseline": cpu,
             "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
