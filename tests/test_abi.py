@@ -127,3 +127,16 @@ def test_workspace_queries(L):
     assert L.zmoe_permute_workspace_size(16384, 16, 2) >= (32768 // 256) * 16 * 4
     assert L.zmoe_permute_workspace_size(-1, 16, 1) == 0
     assert L.zmoe_grouped_swiglu_workspace_size(64, 16, 2048, 3072, 1) >= 0
+
+
+def test_layer_dispatch_by_batch_size(L):
+    """zmoe_moe_layer's launch choice, visible in its workspace query (host logic, no device call made
+    beyond the attribute queries): T * k <= 4 takes the tiny-batch launch, whose workspace is one
+    256-byte counter block plus h in fp32 for the T k assignments; larger decode batches take the
+    stream-K launch, with its per-SM partial slots."""
+    BF16 = 1   # ZMOE_BF16
+    for T, k in [(1, 1), (1, 2), (2, 2), (4, 1)]:
+        assert L.zmoe_moe_layer_workspace_size(T, 2048, 3072, 16, k, BF16) == 256 + T * k * 3072 * 4
+    big = L.zmoe_moe_layer_workspace_size(5, 2048, 3072, 16, 1, BF16)
+    assert big > 256 + 5 * 3072 * 4 + 148 * 2 * 2 * 16 * 128 * 4
+
