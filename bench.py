@@ -2,9 +2,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
 
-A step is one pass of the whole MoE layer over one batch of synthetic tokens:
-zmoe_route -> zmoe_permute -> zmoe_grouped_swiglu -> zmoe_combine, all through libzmoe's
-C-ABI.  The default workload is the decode step (T = 64 tokens, d_model 2048, d_ff 3072,
+A step is one pass of the whole MoE layer over one batch of synthetic tokens, through libzmoe's
+C-ABI: at decode sizes one zmoe_moe_layer call (router, dispatch, SwiGLU and combine in one
+launch); at prefill sizes zmoe_route -> zmoe_permute -> zmoe_grouped_swiglu -> zmoe_combine.
+The default workload is the decode step (T = 64 tokens, d_model 2048, d_ff 3072,
 16 experts, top-1, bf16 weights with fp32 accumulation): memory-bound, every touched
 expert's weights are streamed from HBM once.  Four copies of the layer's weights (2.4 GB,
 far above the 126 MB L2) are used in rotation so that no step finds its weights in L2.
@@ -31,6 +32,8 @@ import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
+
+from sparse_moe_decoder_b200.dp import job_rate, max_over_ranks, rank_token_seed  # noqa: E402
 
 METRIC = "MoE-layer tokens/sec on 1 B200 and % of roofline (HBM GB/s or tensor TFLOP/s)"
 FALLBACK_HBM_GBS = 6650.0
@@ -332,7 +335,7 @@ def run_stack(args):
     n = args.warmup + args.steps
     codes = spec.codes(n + 1)
     if rank > 0:
-        codes = np.random.default_rng(1000 + rank).integers(0, 1024, size=codes.shape).astype(np.int32)
+        codes = np.random.default_rng(rank_token_seed(rank)).integers(0, 1024, size=codes.shape).astype(np.int32)
     codes_dev = torch.from_numpy(codes).cuda()
     stream = torch.cuda.current_stream()
 
@@ -386,12 +389,9 @@ def run_stack(args):
         ev1.record(stream)
         torch.cuda.synchronize()
     elapsed_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t[0])
+    elapsed_ms, = max_over_ranks([elapsed_ms], "cuda")
     ms_per_step = elapsed_ms / args.steps
-    value = world * args.steps / (elapsed_ms / 1e3)
+    value = job_rate(1, world, args.steps, elapsed_ms)
 
     # e2e: codes from pinned host memory each step, the final residual stream read back
     codes_host = torch.from_numpy(codes).pin_memory()
@@ -470,7 +470,7 @@ def run_fp8(args):
     L = make_config(2)
     if rank > 0:
         from moe_inputs import round_to_bf16
-        L.x = round_to_bf16(np.random.default_rng(1000 + rank).standard_normal(L.x.shape, dtype=np.float32))
+        L.x = round_to_bf16(np.random.default_rng(rank_token_seed(rank)).standard_normal(L.x.shape, dtype=np.float32))
     Q = [quantize_e4m3_rows(w) for w in (L.w_gate, L.w_up, L.w_down)]
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     n_copies = args.weight_copies if args.weight_copies > 0 else 8     # 8 x 302 MB of codes > L2
@@ -510,11 +510,8 @@ def run_fp8(args):
         torch.cuda.synchronize()
     elapsed = e0.elapsed_time(e1)
     k_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    if world > 1:
-        t = torch.tensor([elapsed, k_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed, k_ms = float(t[0]), float(t[1])
-    value = T * world * args.steps / (elapsed / 1e3)
+    elapsed, k_ms = max_over_ranks([elapsed, k_ms], "cuda")
+    value = job_rate(T, world, args.steps, elapsed)
     # e2e from pinned host memory
     xh = torch.from_numpy(L.x).to(torch.bfloat16).pin_memory()
     yh = torch.empty((T, L.d), dtype=torch.float32).pin_memory()
@@ -529,10 +526,7 @@ def run_fp8(args):
     a1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = a0.elapsed_time(a1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms, = max_over_ranks([e2e_ms], "cuda")
     errs = zmoe_get_device_errors()
     peaks = load_peaks()
     M = T
@@ -603,7 +597,7 @@ def main(argv=None):
     if rank > 0:
         # each rank its own tokens, replicated weights
         from moe_inputs import round_to_bf16
-        rng = np.random.default_rng(1000 + rank)
+        rng = np.random.default_rng(rank_token_seed(rank))
         L.x = round_to_bf16(rng.standard_normal(L.x.shape, dtype=np.float32))
     dt = torch.bfloat16
     W0 = MoEWeights.from_host(L)
@@ -655,13 +649,9 @@ def main(argv=None):
         dist.barrier()
     elapsed_ms = ev0.elapsed_time(ev1)
     ffn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_ffn)
-    if world > 1:
-        t = torch.tensor([elapsed_ms, ffn_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, ffn_ms = float(t[0]), float(t[1])
+    elapsed_ms, ffn_ms = max_over_ranks([elapsed_ms, ffn_ms], "cuda")
     ms_per_step = elapsed_ms / args.steps
-    tokens_total = L.T * world * args.steps
-    value = tokens_total / (elapsed_ms / 1e3)
+    value = job_rate(L.T, world, args.steps, elapsed_ms)
 
     # launches of libzmoe kernels per step
     n_assign = L.T * L.k
@@ -687,11 +677,8 @@ def main(argv=None):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e_value = tokens_total / (e2e_ms / 1e3)
+    e2e_ms, = max_over_ranks([e2e_ms], "cuda")
+    e2e_value = job_rate(L.T, world, args.steps, e2e_ms)
     h2d = x_host.numel() * x_host.element_size()
     d2h = y_host.numel() * y_host.element_size()
 
