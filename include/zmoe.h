@@ -224,8 +224,10 @@ ZMOE_API size_t zmoe_moe_layer_workspace_size(int T, int d, int f, int E, int k,
  *   y[t] = h[t] + sum_{i < k} gates[t, i] * FFN_{expert_idx[t, i]}(x[t])   (h == NULL: no residual)
  * with the router, dispatch, SwiGLU and combine of zmoe_route, zmoe_permute,
  * zmoe_grouped_swiglu and zmoe_combine (same conventions, same results up to fp32 summation
- * order).  Decode sizes (bf16, T * k < 64 E, T * k <= 1024, d and f multiples of 256) run as
- * one cooperative launch; other sizes run those entry points in order.
+ * order).  A few tokens (bf16, T * k <= 4) run as one cooperative launch that contracts every
+ * weight row whole on one SM (the hidden activations kept in fp32, not as a bf16 pair); decode
+ * sizes (bf16, T * k < 64 E, T * k <= 1024, d and f multiples of 256) run as one cooperative
+ * stream-K launch; other sizes run those entry points in order.
  *   x: [T, d] of `dtype` (or NULL with gamma); h: f32 [T, d] or NULL (required with gamma);
  *   gamma: f32 [d] or NULL; w_router [E, d], w_gate, w_up [E, f, d], w_down [E, d, f] of
  *   `dtype`; logit_bias, sel_bias: f32 [E] or NULL.

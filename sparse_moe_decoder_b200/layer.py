@@ -1,8 +1,8 @@
 """The MoE layer and the batch-1 decode stack, chained through libzmoe's C entry points.
 
 Buffers are allocated once (torch is used for device memory only); every step runs in
-libzmoe's kernels.  A layer is one call of ``zmoe_moe_layer`` (one cooperative launch at
-decode sizes); ``MoELayerRunner.run_steps`` chains the separate entry points instead:
+libzmoe's kernels.  A layer is one call of ``zmoe_moe_layer`` (one cooperative launch for a few
+tokens and at decode sizes); ``MoELayerRunner.run_steps`` chains the separate entry points instead:
 
     zmoe_route -> zmoe_permute -> zmoe_grouped_swiglu -> zmoe_combine
 
