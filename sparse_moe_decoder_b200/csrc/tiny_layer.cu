@@ -18,8 +18,6 @@
 //   * phase B: CTA c owns the d-rows [c d / C, (c + 1) d / C); it bulk-loads all of h and contracts
 //     its W_down rows, then writes y for its rows, summing the chosen experts in slot order.
 // Every sum is fp32 and in a fixed order (no atomics): the result does not depend on timing.
-#include <cooperative_groups.h>
-
 #include "sm100_ptx.cuh"
 
 namespace zmoe {
