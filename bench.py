@@ -5,10 +5,12 @@
 A step is one pass of the whole MoE layer over one batch of synthetic tokens, through libzmoe's
 C-ABI: at decode sizes one zmoe_moe_layer call (router, dispatch, SwiGLU and combine in one
 launch); at prefill sizes zmoe_route -> zmoe_permute -> zmoe_grouped_swiglu -> zmoe_combine.
-The default workload is the decode step (T = 64 tokens, d_model 2048, d_ff 3072,
-16 experts, top-1, bf16 weights with fp32 accumulation): memory-bound, every touched
-expert's weights are streamed from HBM once.  Four copies of the layer's weights (2.4 GB,
-far above the 126 MB L2) are used in rotation so that no step finds its weights in L2.
+The default (headline) workload is the largest single-GPU layer: T = 16384 tokens, d_model 2048,
+d_ff 3072, 16 experts, top-2 with renormalised gates and a Zipf(1.2) logit skew, bf16 weights with
+fp32 accumulation; the grouped SwiGLU is tensor-bound and is reported against the bf16 tensor
+peak.  The same run also measures, and reports under "also", the decode step (T = 64, top-1:
+HBM-bound; four copies of the weights, 2.4 GB, rotate so that no step finds them in L2), the
+top-1 prefill layer with uneven loads, and the batch-1 24-layer decode stack (us/token).
 
 Multi-GPU (torchrun, one rank per GPU): tokens are independent, so every rank runs its own
 batch against replicated weights with no data-path collective (weak scaling); the time is
@@ -45,7 +47,9 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4, 5, 6, 7])
+    ap.add_argument("--config", type=int, default=None, choices=[2, 3, 4, 5, 6, 7],
+                    help="one workload alone; default: the headline workload (4) with workloads 2, 3 and 5 "
+                         "measured in the same run and reported under 'also'")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle timing leg")
@@ -188,6 +192,8 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
+    if args.config is None:
+        args.config = HEADLINE
     if args.config in (5, 6):
         return run_reference_stack(args)
     from moe_inputs import make_config
@@ -312,16 +318,10 @@ def oracle_stack_layers(spec, expert):
 
 def run_stack(args):
     """Configuration 5: tokens/s (= 1 / s per token) of the 24-layer batch-1 stack; 6: the full 28-layer
-    FFN stack (3 dense + 24 MoE + 1 dense)."""
+    FFN stack (3 dense + 24 MoE + 1 dense).  Returns rank 0's JSON line (None on other ranks)."""
     import torch
-    import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local_rank)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=torch.device("cuda", local_rank))
+    world, rank, local_rank = args.world, args.rank, args.local_rank
     from moe_inputs import StackSpec, bf16_bits, stack_expert_bits
     from sparse_moe_decoder_b200 import zmoe_get_device_errors
     from sparse_moe_decoder_b200.layer import stack_from_bits
@@ -447,24 +447,15 @@ def run_stack(args):
             "clocks": clk.summary(),
             "device_errors": dev_errors,
         }
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    return 0
+        return line
+    return None
 
 
 def run_fp8(args):
     """Workload 7: the decode step (configuration 2's tokens and weights) with the expert weights stored
     as E4M3 codes + row scales, one zmoe_moe_layer_fp8 call per step."""
     import torch
-    import torch.distributed as dist
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local_rank)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+    world, rank, local_rank = args.world, args.rank, args.local_rank
     from moe_inputs import make_config, quantize_e4m3_rows
     from sparse_moe_decoder_b200 import zmoe_get_device_errors, zmoe_moe_layer_fp8
     L = make_config(2)
@@ -545,7 +536,7 @@ def run_fp8(args):
         cpu = {"value": T * n / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"oracle.moe_layer_fp8 (numpy float64) on the 64-token layer, {n} step(s), {el:.1f} s"}
     if rank == 0:
-        print(json.dumps({
+        return {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp8", "data": "synthetic",
@@ -561,35 +552,16 @@ def run_fp8(args):
             "e2e": {"value": T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * L.d * 2, "d2h_bytes_per_step": T * L.d * 4},
             "gpu_launches": args.steps, "clocks": clk.summary(), "layer_ms_per_step": k_ms, "device_errors": errs,
-        }), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    return 0
+        }
+    return None
 
 
-def main(argv=None):
-    args = parse_args(argv)
-    if args.impl == "reference":
-        return run_reference(args)
-    if args.config == 7:
-        return run_fp8(args)
-    if args.config >= 5:
-        return run_stack(args)
-
+def run_layer(args):
+    """Workloads 2-4: one MoE layer per step.  Returns rank 0's JSON line (None on other ranks)."""
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA GPU")
-    torch.cuda.set_device(local_rank)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
-
+    world, rank, local_rank = args.world, args.rank, args.local_rank
     from moe_inputs import make_config
     from sparse_moe_decoder_b200 import MoELayerRunner, MoEWeights, zmoe_get_device_errors
 
@@ -657,7 +629,8 @@ def main(argv=None):
     n_assign = L.T * L.k
     launches_per_step = 1 if fused else 1 + (1 if n_assign <= 1024 else 4) + 2 + 1
 
-    # e2e: the same steps through the public API from pinned host memory, result read back
+    # e2e: the same layer through the public API (one zmoe_moe_layer call) from pinned host memory,
+    # result read back
     x_host = torch.from_numpy(L.x).to(dt).pin_memory()
     y_host = torch.empty((L.T, L.d), dtype=torch.float32).pin_memory()
     x_dev = torch.empty_like(x)
@@ -684,12 +657,12 @@ def main(argv=None):
 
     dev_errors = zmoe_get_device_errors()
 
-    # roofline of the dominant kernels (the grouped-SwiGLU launches: gate/up then down)
+    # roofline of the dominant kernels (decode: the one layer launch; prefill: the grouped-SwiGLU
+    # launches, gate/up then down)
     peaks = load_peaks()
     bpe = 2
-    counts_all = counts
-    touched = int((counts_all > 0).sum())
-    M = int(counts_all.sum())
+    touched = int((counts > 0).sum())
+    M = int(counts.sum())
     weight_bytes = touched * 3 * L.f * L.d * bpe
     act_bytes = M * L.d * bpe + 2 * (M * 2 * L.f * bpe) + M * L.d * 4   # x_perm in, h pair out + in, y_perm out
     if fused:
@@ -697,47 +670,120 @@ def main(argv=None):
         act_bytes += L.T * L.d * bpe + L.E * L.d * bpe + M * L.d * bpe + L.T * L.d * 4
     alg_bytes = weight_bytes + act_bytes
     flops = 2.0 * M * 3 * L.d * L.f
-    if args.config == 2:
+    if fused:
         achieved = alg_bytes / (ffn_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_from_profiles("grouped_swiglu_cfg2"),
-                "kernel": ("moe_layer_kernel: router, dispatch, SwiGLU and combine in one launch" if fused else
-                           "zmoe_grouped_swiglu (dec_tc_kernel)"),
+                "kernel": "moe_layer_kernel: router, dispatch, SwiGLU and combine in one launch",
                 "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peaks["source"]}
     else:
         achieved = flops / (ffn_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"],
                 "traffic": traffic_from_profiles(f"grouped_swiglu_cfg{args.config}"),
-                "kernel": "zmoe_grouped_swiglu", "algorithmic_flops_per_launch": flops,
-                "peak_source": peaks["source"]}
+                "kernel": "zmoe_grouped_swiglu (tc_ffn_kernel: gate/up, then down)",
+                "algorithmic_flops_per_launch": flops, "peak_source": peaks["source"],
+                "peak_kind": "burst (the SwiGLU is timed alone, between the other calls of the step)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, steps, el, sample = oracle_leg(L, args.cpu_seconds)
         cpu = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle", "sample": sample}
 
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOADS[args.config], "T": L.T, "d_model": L.d, "d_ff": L.f, "E": L.E,
-                       "k": L.k, "tokens_per_rank": L.T, "parallelism": f"dp{world} (replicated weights, no "
-                       "data-path collective)",
-                       "l2": (f"weights rotated over {n_copies} device copies ({n_copies * 0.604:.1f} GB > 126 MB L2)"
-                              if n_copies > 1 else "inputs larger than L2 (one layer's weights: 604 MB)"),
-                       "experts_touched": experts_touched},
-            "roofline": roof,
-            "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk.summary(),
-            "ffn_ms_per_step": ffn_ms,
-            "device_errors": dev_errors,
-        }
+    if rank != 0:
+        return None
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOADS[args.config], "T": L.T, "d_model": L.d, "d_ff": L.f, "E": L.E,
+                   "k": L.k, "tokens_per_rank": L.T, "parallelism": f"dp{world} (replicated weights, no "
+                   "data-path collective)",
+                   "l2": (f"weights rotated over {n_copies} device copies ({n_copies * 0.604:.1f} GB > 126 MB L2)"
+                          if n_copies > 1 else "inputs larger than L2 (one layer's weights: 604 MB, x and the "
+                          "permuted rows another 0.2-0.3 GB)"),
+                   "experts_touched": experts_touched,
+                   "expert_loads": counts.tolist()},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "call": "zmoe_moe_layer"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "ffn_ms_per_step": ffn_ms,
+        "device_errors": dev_errors,
+    }
+
+
+def summary_of(line):
+    """The keys of another workload's line that the headline line carries under 'also'."""
+    if line is None:
+        return None
+    out = {"workload": line["config"]["workload"], "value": line["value"], "unit": line["unit"],
+           "steps": line["steps"], "warmup": line["warmup"], "ms_per_step": line["ms_per_step"]}
+    if "us_per_token" in line["config"]:
+        out["us_per_token"] = line["config"]["us_per_token"]
+    r = line.get("roofline") or {}
+    for k in ("bound", "achieved", "peak", "unit", "frac", "kernel"):
+        if k in r:
+            out[f"roofline_{k}"] = r[k]
+    out["e2e_value"] = (line.get("e2e") or {}).get("value")
+    out["clocks"] = line.get("clocks")
+    out["gpu_launches"] = line.get("gpu_launches")
+    out["device_errors"] = line.get("device_errors")
+    return out
+
+
+def run_one(args):
+    if args.config == 7:
+        return run_fp8(args)
+    if args.config >= 5:
+        return run_stack(args)
+    return run_layer(args)
+
+
+HEADLINE = 4
+ALSO = ((2, 200, 20), (3, None, None), (5, 100, 10))    # (workload, min steps, min warm-up)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    args.world = int(os.environ.get("WORLD_SIZE", "1"))
+    args.rank = int(os.environ.get("RANK", "0"))
+    args.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(args.local_rank)
+    if args.world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                device_id=torch.device("cuda", args.local_rank))
+    if args.config is not None:
+        line = run_one(args)
+    else:
+        # the headline workload, then the others in the same run (same ranks, same collective steps)
+        args.config = HEADLINE
+        line = run_one(args)
+        also = {}
+        for cfg, min_steps, min_warm in ALSO:
+            sub = argparse.Namespace(**vars(args))
+            sub.config = cfg
+            sub.no_cpu_baseline = True
+            if min_steps:
+                sub.steps = max(args.steps, min_steps)
+                sub.warmup = max(args.warmup, min_warm)
+            torch.cuda.empty_cache()
+            also[f"workload_{cfg}"] = summary_of(run_one(sub))
+        if line is not None:
+            line["also"] = also
+    if line is not None:
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if args.world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0

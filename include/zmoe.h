@@ -153,21 +153,22 @@ ZMOE_API zmoe_status zmoe_permute(const int32_t* expert_idx, const void* x, zmoe
                          void* workspace, size_t ws_bytes, zmoe_stream_t stream);
 
 /*
- * zmoe_permute without any device allocation, for callers that cannot allocate: code
- * whose device memory is wholly owned by a host framework's pool allocator (a cudaMalloc
- * behind its back can fail for lack of memory, or stall the device while it waits),
- * code that must not synchronise the device on its hot path, and code recording into a
- * CUDA graph in a capture mode that forbids allocation.  The ZONOS2 pages have no
- * counterpart: this is an interface convenience, not a step of the method.
+ * zmoe_permute without any device allocation, for callers that cannot allocate: code whose
+ * device memory is wholly owned by a host framework's pool allocator (a cudaMalloc behind the
+ * pool's back can fail for lack of memory, or stall every stream while the driver maps the
+ * pages), and code on a latency-critical path that must never synchronise the device.  The
+ * ZONOS2 pages have no counterpart: this is an interface convenience, not a step of the method.
  *   Same arguments, outputs and results as zmoe_permute, without workspace/ws_bytes.
  *   Its scratch (per-tile expert counts, 64 KB) is a static device array inside the
  *   library, held by every GPU that loads it until the process exits.  Limit: T * k <=
- *   65536; larger problems return ZMOE_ERR_INVALID_ARG with a message naming the limit.
- *   The first call on a device looks up that array's device address (once per device,
- *   with the device current) and caches it; make that first call before capturing a
- *   stream into a CUDA graph.  All calls share the array: calls that overlap on the GPU
- *   (different streams without ordering between them) race and give wrong results.  It
- *   calls no cudaMalloc, cudaFree or allocating library routine.
+ *   65536; larger problems return ZMOE_ERR_INVALID_ARG with a message naming the limit and
+ *   launch nothing.  The first call on a device looks up that array's device address (once
+ *   per device, with the device current) and caches it for the life of the process, so a
+ *   device reset after that first call is not supported; make the first call before any
+ *   stream capture.  All calls share the array and it keeps the last call's contents (the
+ *   call rewrites every entry it reads, so nothing needs clearing between calls); calls that
+ *   overlap on the GPU (different streams without ordering between them) race on it and give
+ *   wrong results.  It calls no cudaMalloc, cudaFree or allocating library routine.
  */
 ZMOE_API zmoe_status zmoe_permute_noalloc(const int32_t* expert_idx, const void* x, zmoe_dtype dtype, int T, int d,
                                           int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
@@ -308,6 +309,19 @@ ZMOE_API zmoe_status zmoe_speaker_prefix(const float* e, const void* w_spk, zmoe
  * else ZMOE_OK.
  */
 ZMOE_API zmoe_status zmoe_get_device_errors(zmoe_stream_t stream, uint32_t* count);
+
+/*
+ * Fault injection for tests of the timeout path (no counterpart on the pages; failure detection of
+ * the library itself).  With extra > 0, every later launch of the stream-K decode kernels
+ * (zmoe_moe_layer and zmoe_moe_layer_fp8 at decode sizes, zmoe_grouped_swiglu below 64 rows per
+ * expert) makes its phase-A -> phase-B hand-off wait for `extra` more finished phase-A units than
+ * exist, giving up after limit_ns (in [1 us, 2 s]) instead of the usual 2 s.  The wait then runs
+ * out: each CTA counts a timeout, stops, waits (bounded) for its own copies and MMAs, frees its
+ * tensor memory and returns, and zmoe_get_device_errors() reports ZMOE_ERR_TIMEOUT.  The outputs of
+ * such a launch are undefined.  zmoe_debug_inject_timeout(0, 0) restores normal operation.  The
+ * setting is process-wide and read when a call launches; for tests only.
+ */
+ZMOE_API zmoe_status zmoe_debug_inject_timeout(uint32_t extra, uint64_t limit_ns);
 
 #ifdef __cplusplus
 }

@@ -50,6 +50,7 @@ __global__ void combine_kernel(const float4* __restrict__ y_perm, const int32_t*
 
 extern "C" zmoe_status zmoe_combine(const float* y_perm, const int32_t* inv_perm, const float* gates,
                                     const float* residual, int T, int d, int k, float* y, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_combine");
   using namespace zmoe;
   ZMOE_REQUIRE(T >= 0, "zmoe_combine: T must be >= 0");
   ZMOE_REQUIRE(k == 1 || k == 2, "zmoe_combine: k must be 1 or 2");

@@ -8,6 +8,8 @@
 
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "zmoe.h"
 
 namespace zmoe {
@@ -39,6 +41,16 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t dtype_size(zmoe_dtype dt) { return dt == ZMOE_BF16 ? 2 : 4; }
 
 inline bool dtype_ok(int dt) { return dt == ZMOE_F32 || dt == ZMOE_BF16; }
+
+// An NVTX range around one entry point, so that a profiler timeline shows each zmoe_* call
+// (header-only NVTX v3: without a tool attached a push/pop costs a few nanoseconds).
+struct TraceRange {
+  explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
+#define ZMOE_TRACE(name) ::zmoe::TraceRange zmoe_trace_range_(name)
 
 #define ZMOE_REQUIRE(cond, msg)                                      \
   do {                                                               \

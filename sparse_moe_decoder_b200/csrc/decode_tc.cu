@@ -44,6 +44,8 @@
 //   and, after a second barrier, fuses the gate-weighted combine into the down projection's
 //   epilogue: y[t] = residual[t] + sum_i gate[t, i] * y_perm[row(t, i)], formed in slot order (for
 //   k = 2 by the later of the token's two units, from both rows, so the sum is deterministic).
+#include <atomic>
+
 #include "sm100_ptx.cuh"
 
 namespace zmoe {
@@ -117,6 +119,10 @@ struct DecArgs {
   // fused layer: x_perm is complete once this counter reaches x_target (grid-wide arrivals)
   const unsigned int* x_ready;
   unsigned int x_target;
+  // the phase-A -> phase-B hand-off waits for ready[e] >= (phase-A units of e) + hand_extra, at most
+  // hand_limit_ns; hand_extra is 0 except under zmoe_debug_inject_timeout
+  unsigned int hand_extra;
+  unsigned long long hand_limit_ns;
 };
 
 struct LayerArgs {
@@ -396,10 +402,11 @@ __device__ __forceinline__ void ffn_roles(const CUtensorMap* mWg, const CUtensor
           for (int j = g.j0; j < g.j1 && ok; ++j) {
             if (!wt && ph == 1 && U.e != ready_e) {
               // every phase-A unit of expert e must have stored its h rows
-              const unsigned int target = static_cast<unsigned int>(C.ustart[0][U.e + 1] - C.ustart[0][U.e]);
+              const unsigned int target =
+                  static_cast<unsigned int>(C.ustart[0][U.e + 1] - C.ustart[0][U.e]) + p.hand_extra;
               const uint64_t t0 = globaltimer();
               for (uint32_t it = 0; ld_acquire(p.ready + U.e) < target; ++it) {
-                if ((it & 15) == 15 && (*abort_flag || globaltimer() - t0 > kTimeoutNs)) {
+                if ((it & 15) == 15 && (*abort_flag || globaltimer() - t0 > p.hand_limit_ns)) {
                   ok = false;
                   break;
                 }
@@ -1280,6 +1287,11 @@ zmoe_status launch_coop(K kernel, const char* what, cudaStream_t s, int threads,
   return check_launch(what);
 }
 
+// Fault injection for tests of the timeout path (zmoe_debug_inject_timeout): host-side settings that
+// every launch copies into its arguments.
+std::atomic<unsigned int> g_inject_extra{0};
+std::atomic<unsigned long long> g_inject_limit_ns{0};
+
 DecArgs dec_args(const Layout& Lo, void* ws, const int32_t* offsets, uint16_t* h, float* y_perm, int E, int d, int f,
                  int M_total) {
   unsigned char* w = static_cast<unsigned char*>(ws);
@@ -1300,6 +1312,8 @@ DecArgs dec_args(const Layout& Lo, void* ws, const int32_t* offsets, uint16_t* h
   a.M_total = M_total;
   a.ua_cap = Lo.ua;
   a.ub_cap = Lo.ub;
+  a.hand_extra = g_inject_extra.load();
+  a.hand_limit_ns = a.hand_extra ? g_inject_limit_ns.load() : kTimeoutNs;
   return a;
 }
 
@@ -1451,3 +1465,12 @@ zmoe_status moe_layer_fused(const uint16_t* x, const float* h_in, const float* g
 }
 
 }  // namespace zmoe
+
+extern "C" zmoe_status zmoe_debug_inject_timeout(uint32_t extra, uint64_t limit_ns) {
+  ZMOE_REQUIRE(extra == 0 || (limit_ns >= 1000ull && limit_ns <= 2000000000ull),
+               "zmoe_debug_inject_timeout: limit_ns must be in [1 us, 2 s] when extra > 0");
+  zmoe::clear_error();
+  zmoe::g_inject_limit_ns.store(extra ? limit_ns : 0ull);
+  zmoe::g_inject_extra.store(extra);
+  return ZMOE_OK;
+}

@@ -51,6 +51,7 @@ extern "C" {
 
 zmoe_status zmoe_delay_shear(const int32_t* X, int32_t* Y, int B, int T, int N, int32_t pad,
                              zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_delay_shear");
   using namespace zmoe;
   ZMOE_REQUIRE(B >= 0 && T >= 0, "zmoe_delay_shear: B and T must be >= 0");
   ZMOE_REQUIRE(N >= 1 && N <= 64, "zmoe_delay_shear: N must be in [1, 64]");
@@ -64,6 +65,7 @@ zmoe_status zmoe_delay_shear(const int32_t* X, int32_t* Y, int B, int T, int N, 
 }
 
 zmoe_status zmoe_delay_unshear(const int32_t* Y, int32_t* X, int B, int Ty, int N, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_delay_unshear");
   using namespace zmoe;
   ZMOE_REQUIRE(B >= 0, "zmoe_delay_unshear: B must be >= 0");
   ZMOE_REQUIRE(N >= 1 && N <= 64, "zmoe_delay_unshear: N must be in [1, 64]");

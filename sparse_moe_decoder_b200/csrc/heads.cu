@@ -309,6 +309,7 @@ size_t zmoe_output_heads_workspace_size(int T, int N) {
 zmoe_status zmoe_output_heads(const float* h, const float* gamma, float eps, const void* w_heads, zmoe_dtype dtype,
                               int T, int N, int V, int d, int32_t* ids, float* logits, void* x_out, void* workspace,
                               size_t ws_bytes, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_output_heads");
   using namespace zmoe;
   ZMOE_REQUIRE(dtype_ok(dtype), "zmoe_output_heads: bad dtype");
   ZMOE_REQUIRE(T >= 0 && N >= 1 && V >= 1, "zmoe_output_heads: T >= 0, N >= 1, V >= 1");

@@ -96,6 +96,7 @@ zmoe_status zmoe_moe_layer(const void* x, const float* h, const float* gamma, fl
                            const void* w_down, zmoe_dtype dtype, int T, int d, int f, int E, int k, float* y,
                            int32_t* expert_idx, float* gates, float* margin, void* x_norm, void* workspace,
                            size_t ws_bytes, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_moe_layer");
   using namespace zmoe;
   ZMOE_REQUIRE(dtype_ok(dtype), "zmoe_moe_layer: bad dtype");
   ZMOE_REQUIRE(T >= 0, "zmoe_moe_layer: T must be >= 0");
@@ -164,6 +165,7 @@ zmoe_status zmoe_moe_layer_fp8(const void* x, const float* h, const float* gamma
                                const float* s_down, int T, int d, int f, int E, int k, float* y, int32_t* expert_idx,
                                float* gates, float* margin, void* x_norm, void* workspace, size_t ws_bytes,
                                zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_moe_layer_fp8");
   using namespace zmoe;
   ZMOE_REQUIRE(T >= 0, "zmoe_moe_layer_fp8: T must be >= 0");
   ZMOE_REQUIRE(E >= 1 && E <= 64, "zmoe_moe_layer_fp8: E must be in [1, 64]");

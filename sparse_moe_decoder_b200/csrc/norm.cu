@@ -151,6 +151,7 @@ extern "C" {
 zmoe_status zmoe_embed_sum_rmsnorm(const int32_t* ids, const void* tables, zmoe_dtype table_dtype,
                                    const float* gamma, float eps, int T, int N, int V, int d, void* out,
                                    zmoe_dtype out_dtype, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_embed_sum_rmsnorm");
   using namespace zmoe;
   ZMOE_REQUIRE(dtype_ok(table_dtype) && dtype_ok(out_dtype), "zmoe_embed_sum_rmsnorm: bad dtype");
   ZMOE_REQUIRE(T >= 0 && N >= 1 && N <= 64 && V >= 1, "zmoe_embed_sum_rmsnorm: bad T, N or V");
@@ -182,6 +183,7 @@ zmoe_status zmoe_embed_sum_rmsnorm(const int32_t* ids, const void* tables, zmoe_
 
 zmoe_status zmoe_rmsnorm(const void* h, zmoe_dtype in_dtype, const float* gamma, float eps, int T, int d, void* out,
                          zmoe_dtype out_dtype, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_rmsnorm");
   using namespace zmoe;
   ZMOE_REQUIRE(dtype_ok(in_dtype) && dtype_ok(out_dtype), "zmoe_rmsnorm: bad dtype");
   ZMOE_REQUIRE(T >= 0, "zmoe_rmsnorm: T must be >= 0");

@@ -206,6 +206,7 @@ size_t zmoe_permute_workspace_size(int T, int E, int k) {
 zmoe_status zmoe_permute(const int32_t* expert_idx, const void* x, zmoe_dtype dtype, int T, int d, int E, int k,
                          int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* x_perm,
                          void* workspace, size_t ws_bytes, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_permute");
   using namespace zmoe;
   ZMOE_REQUIRE(dtype_ok(dtype), "zmoe_permute: bad dtype");
   ZMOE_REQUIRE(T >= 0, "zmoe_permute: T must be >= 0");
@@ -255,9 +256,10 @@ zmoe_status zmoe_permute(const int32_t* expert_idx, const void* x, zmoe_dtype dt
 // holds the array (64 KB) until the process exits.  In host code `g_noalloc_tile_counts` is
 // only a host-side stand-in for the symbol, never a device address; its device address is
 // fetched with cudaGetSymbolAddress once per device, with that device current, on the first
-// call made on that device, and cached.  Every call shares the array and it keeps the last
-// call's contents: the count pass writes every entry the later passes read, so nothing needs
-// clearing, but two calls that overlap on the GPU (different streams, no ordering) race on it.
+// call made on that device, and cached for the life of the process (a device reset after that
+// first call is not supported).  Every call shares the array and it keeps the last call's
+// contents: the count pass writes every entry the later passes read, so nothing needs clearing,
+// but two calls that overlap on the GPU (different streams, no ordering) race on it.
 // ---------------------------------------------------------------------------------------------
 namespace zmoe {
 namespace {
@@ -278,9 +280,11 @@ zmoe_status noalloc_scratch(int32_t** out) {
   if (!g_noalloc_addr[dev]) {
     int32_t* ptr = nullptr;
     e = cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_noalloc_tile_counts);
-    if (e != cudaSuccess || ptr == nullptr)
+    if (e != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();   // consume the error so that a later call's launch check does not report it
       return fail(ZMOE_ERR_CUDA, std::string("zmoe_permute_noalloc: cudaGetSymbolAddress failed: ") +
                                      cudaGetErrorString(e));
+    }
     g_noalloc_addr[dev] = ptr;
   }
   *out = g_noalloc_addr[dev];
@@ -293,6 +297,7 @@ zmoe_status noalloc_scratch(int32_t** out) {
 extern "C" zmoe_status zmoe_permute_noalloc(const int32_t* expert_idx, const void* x, zmoe_dtype dtype, int T, int d,
                                             int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
                                             int32_t* inv_perm, void* x_perm, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_permute_noalloc");
   using namespace zmoe;
   ZMOE_REQUIRE(dtype_ok(dtype), "zmoe_permute_noalloc: bad dtype");
   ZMOE_REQUIRE(T >= 0, "zmoe_permute_noalloc: T must be >= 0");

@@ -244,6 +244,7 @@ __global__ void single_expert_kernel(int T, int32_t* __restrict__ expert_idx, fl
 extern "C" zmoe_status zmoe_route(const void* x, const void* w_router, zmoe_dtype dtype, const float* logit_bias,
                                   const float* sel_bias, int T, int d, int E, int k, int32_t* expert_idx,
                                   float* gates, float* margin, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_route");
   using namespace zmoe;
   ZMOE_REQUIRE(dtype_ok(dtype), "zmoe_route: bad dtype");
   ZMOE_REQUIRE(T >= 0, "zmoe_route: T must be >= 0");

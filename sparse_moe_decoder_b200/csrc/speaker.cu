@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(kThreads) speaker_kernel(const float* __restri
 
 extern "C" zmoe_status zmoe_speaker_prefix(const float* e, const void* w_spk, zmoe_dtype dtype, const float* b_spk,
                                            int B, int d, int n_in, float* out, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_speaker_prefix");
   using namespace zmoe;
   ZMOE_REQUIRE(dtype_ok(dtype), "zmoe_speaker_prefix: bad dtype");
   ZMOE_REQUIRE(B >= 0 && d >= 1 && n_in >= 8 && n_in % 8 == 0, "zmoe_speaker_prefix: B >= 0, d >= 1, n_in % 8 == 0");

@@ -103,6 +103,7 @@ size_t zmoe_grouped_swiglu_workspace_size(int M_total, int E, int d, int f, zmoe
 zmoe_status zmoe_grouped_swiglu(const void* x_perm, const int32_t* offsets, int M_total, const void* w_gate,
                                 const void* w_up, const void* w_down, zmoe_dtype dtype, int E, int d, int f, void* h,
                                 float* y_perm, void* workspace, size_t ws_bytes, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_grouped_swiglu");
   using namespace zmoe;
   ZMOE_REQUIRE(dtype_ok(dtype), "zmoe_grouped_swiglu: bad dtype");
   ZMOE_REQUIRE(M_total >= 0, "zmoe_grouped_swiglu: M_total must be >= 0");

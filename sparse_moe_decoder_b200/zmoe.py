@@ -53,6 +53,7 @@ SIGNATURES = {
     "zmoe_moe_layer": (_I, [_P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                             _P, _S, _P]),
     "zmoe_get_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "zmoe_debug_inject_timeout": (_I, [ctypes.c_uint32, ctypes.c_uint64]),
 }
 
 

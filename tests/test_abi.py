@@ -140,3 +140,10 @@ def test_layer_dispatch_by_batch_size(L):
     big = L.zmoe_moe_layer_workspace_size(5, 2048, 3072, 16, 1, BF16)
     assert big > 256 + 5 * 3072 * 4 + 148 * 2 * 2 * 16 * 128 * 4
 
+
+
+def test_timeout_injection_checks_its_limit(L):
+    """The test hook of the timeout path only sets host-side state: no GPU needed."""
+    assert L.zmoe_debug_inject_timeout(1, 10) == 1                  # below 1 us: ZMOE_ERR_INVALID_ARG
+    assert L.zmoe_debug_inject_timeout(1, 3_000_000_000) == 1       # above 2 s
+    assert L.zmoe_debug_inject_timeout(0, 0) == 0

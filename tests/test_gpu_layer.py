@@ -1,9 +1,9 @@
 """The whole MoE layer through the C-ABI vs the oracle: zmoe_moe_layer (one call) and the four separate
 entry points (route -> permute -> grouped SwiGLU -> combine).
 
-Configurations 1 and 2 are compared on every token (configuration 2, T = 64, is the decode step the
-benchmark times, in the same launch configuration).  Configurations 3 and 4 (T = 16384) compare all
-routing decisions and a sample of output rows the oracle computes one by one.
+Every configuration is compared on every token: 1 and 2 (the decode step), and the T = 16384 prefill
+layers 3 and 4 (the headline workload the benchmark times, in the same launch configuration), whose
+grouped SwiGLU runs many tiles per CTA.
 """
 import numpy as np
 import pytest
@@ -43,27 +43,23 @@ def test_layer_every_token(cfg, steps):
 
 
 @pytest.mark.parametrize("cfg", [3, 4])
-def test_layer_prefill_sampled(cfg):
+def test_layer_prefill_every_token(cfg):
+    """The T = 16384 prefill layers (top-1 with uneven loads; top-2 with the Zipf skew) on every token:
+    ids bit-exact outside the margin exemption, y element by element within the bf16 bar."""
     require_gpu()
     L = make_config(cfg)
     R, y = run_layer(L)
-    sel, gates, margin, _ = oracle.route(L.x, L.w_router, L.k, L.sel_bias, L.logit_bias)
+    ref = oracle.moe_layer(L.x, L.w_router, L.w_gate, L.w_up, L.w_down, L.k, L.sel_bias, L.logit_bias)
     idx = host(R.idx)
-    ok = margin >= MARGIN_EXEMPT
-    assert np.array_equal(idx[ok], sel[ok]), "routing differs on a token with margin >= 1e-4"
-    counts = np.bincount(sel.ravel(), minlength=L.E)
+    ok = ref["margin"] >= MARGIN_EXEMPT
+    assert np.array_equal(idx[ok], ref["expert_idx"][ok]), "routing differs on a token with margin >= 1e-4"
+    counts = ref["counts"]
     print(f"config {cfg}: expert loads {counts.tolist()}, expert-0 share {counts[0] / counts.sum():.3f}, "
           f"{int((~ok).sum())} low-margin tokens")
-    rng = np.random.default_rng(cfg)
-    sample = np.unique(np.concatenate([[0, L.T - 1], rng.integers(0, L.T, size=192)]))
-    sample = sample[(idx[sample] == sel[sample]).all(1)]
-    want = np.zeros((len(sample), L.d))
-    for n, t in enumerate(sample):
-        for i in range(L.k):
-            e = sel[t, i]
-            want[n] += gates[t, i] * oracle.swiglu_ffn(L.x[t:t + 1], L.w_gate[e], L.w_up[e], L.w_down[e])[0]
-    r = assert_close(y[sample], want, "bf16", f"config {cfg} sampled y")
-    print(f"config {cfg}: sampled y max err {r:.2e} x RMS over {len(sample)} tokens")
+    same = (idx == ref["expert_idx"]).all(1)
+    assert same.sum() >= L.T - int((~ok).sum())
+    r = assert_close(y[same], ref["y"][same], "bf16", f"config {cfg} y (all {int(same.sum())} tokens)")
+    print(f"config {cfg}: y max err {r:.2e} x RMS over {int(same.sum())} of {L.T} tokens")
 
 
 def test_layer_token_permutation_invariance():

@@ -1,12 +1,14 @@
-"""zmoe_permute_noalloc through the C-ABI against zmoe_permute (the entry point with a workspace).
+"""zmoe_permute_noalloc through the C-ABI: against zmoe_permute (the entry point with a workspace) and
+against the oracle's permutation.
 
-Some callers cannot allocate device memory at all: their framework's pool owns it, a cudaMalloc
-would stall the device on a latency-critical path, or they record into a CUDA graph in a capture
-mode that forbids allocation.  zmoe_permute_noalloc serves them with scratch held in a static
-device array of the library.  The permutation is integer work, so its outputs must equal
-zmoe_permute's bit for bit, on two calls in a row (the second call finds the array holding the
-first call's contents).  This file is collected last so that a failure here leaves every other
-test already run.
+Some callers cannot allocate device memory: a host framework whose pool allocator owns all of it (a
+cudaMalloc behind its back can fail for lack of memory, or stall every stream while the driver maps
+pages), or code on a latency-critical path that must never synchronise the device.  For them
+zmoe_permute_noalloc keeps its scratch in a static device array of the library.  The permutation is
+integer work and a bf16 row copy, so its outputs must equal zmoe_permute's and the oracle's bit for
+bit, on two calls in a row (the second call finds the array holding the first call's contents).
+Sizes up to the array's limit (T * k = 65536 assignments) are accepted, one past it is rejected.
+This file is collected last so that a failure here leaves every other test already run.
 """
 import ctypes
 
@@ -14,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from sparse_moe_decoder_b200 import zmoe_permute
 from sparse_moe_decoder_b200.zmoe import ZMOE_BF16, lib
 from tests.gpu_util import require_gpu
@@ -21,6 +24,7 @@ from tests.gpu_util import require_gpu
 pytestmark = pytest.mark.gpu
 
 OUT_KEYS = ("counts", "offsets", "perm", "inv_perm", "x_perm")
+LIMIT = 65536                                     # assignments the static scratch holds
 
 
 def noalloc_permute(idx: torch.Tensor, x: torch.Tensor, E: int):
@@ -44,31 +48,50 @@ def case(T, E, k, seed):
     if k == 1:
         idx = rng.integers(0, E, size=(T, 1))
     else:
-        idx = np.stack([rng.permutation(E)[:2] for _ in range(T)])
-    x = torch.from_numpy(rng.standard_normal((T, 256), dtype=np.float32)).to("cuda", torch.bfloat16)
-    return torch.from_numpy(idx.astype(np.int32)).cuda(), x
+        idx = np.argsort(rng.random((T, E)), axis=1)[:, :2]      # two distinct experts per token
+    x = rng.standard_normal((T, 256), dtype=np.float32)
+    return idx.astype(np.int32), x
 
 
-@pytest.mark.parametrize("T,E,k", [(16384, 16, 2), (64, 16, 1), (30000, 64, 2)])
-def test_noalloc_matches_workspace_entry_point_twice(T, E, k):
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy()
+
+
+@pytest.mark.parametrize("T,E,k", [(16384, 16, 2), (64, 16, 1), (30000, 64, 2), (32768, 16, 2), (65536, 4, 1)])
+def test_noalloc_matches_workspace_entry_point_and_oracle_twice(T, E, k):
     require_gpu()
     for call in range(2):                         # two calls in a row share the static scratch
-        idx, x = case(T, E, k, seed=100 * call + T)
+        idx_h, x_h = case(T, E, k, seed=100 * call + T)
+        idx = torch.from_numpy(idx_h).cuda()
+        x = torch.from_numpy(x_h).to("cuda", torch.bfloat16)
         want = zmoe_permute(idx, x, E)
         st, got = noalloc_permute(idx, x, E)
         assert st == 0, lib().zmoe_last_error()
         torch.cuda.synchronize()
         for key in OUT_KEYS:
-            a, b = want[key].cpu(), got[key].cpu()
+            a, b = want[key], got[key]
             if key == "x_perm":
-                a, b = a.view(torch.int16), b.view(torch.int16)
-            assert torch.equal(a, b), f"call {call}: {key} differs"
+                assert np.array_equal(bf16_bits(a), bf16_bits(b)), f"call {call}: {key} differs from zmoe_permute"
+            else:
+                assert torch.equal(a.cpu(), b.cpu()), f"call {call}: {key} differs from zmoe_permute"
+        ref = oracle.permute(idx_h, E, x.float().cpu().numpy())
+        for key in ("counts", "offsets", "perm", "inv_perm"):
+            assert np.array_equal(got[key].cpu().numpy(), ref[key]), f"call {call}: {key} differs from the oracle"
+        x_ref = torch.from_numpy(np.ascontiguousarray(ref["x_perm"], np.float32)).to(torch.bfloat16)
+        assert np.array_equal(bf16_bits(got["x_perm"]), x_ref.view(torch.int16).numpy()), \
+            f"call {call}: x_perm differs from the oracle"
 
 
-def test_noalloc_rejects_sizes_beyond_its_scratch():
+@pytest.mark.parametrize("T,k", [(32769, 2), (LIMIT + 1, 1)])
+def test_noalloc_rejects_sizes_beyond_its_scratch(T, k):
     require_gpu()
-    T, E, k = 40000, 16, 2                        # 80000 assignments > 65536
-    idx, x = case(T, E, k, seed=1)
-    st, _ = noalloc_permute(idx, x, E)
+    E = 16
+    assert T * k == LIMIT + 1 or T * k == LIMIT + 2
+    idx_h, x_h = case(T, E, k, seed=1)
+    idx = torch.from_numpy(idx_h).cuda()
+    x = torch.from_numpy(x_h).to("cuda", torch.bfloat16)
+    st, out = noalloc_permute(idx, x, E)
     assert st == 1                                # ZMOE_ERR_INVALID_ARG, nothing launched
     assert b"65536" in lib().zmoe_last_error()
+    torch.cuda.synchronize()
+    assert int(out["counts"][0]) == -7            # outputs untouched
