@@ -437,13 +437,16 @@ def run_stack(args):
                        "experts_touched_per_token": touched, "cuda_graph": used_graph},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                         "kernel": f"whole decode step (embed + {spec.total_layers} x tiny_layer_kernel: pre-norm, "
-                                   "router, SwiGLU and combine in one launch per layer)",
+                         "kernel": (f"whole decode step: one stack_kernel launch (embedding + RMSNorm, then "
+                                    f"{spec.total_layers} pre-norm layers: router, SwiGLU, residual)"
+                                    + (" + heads_kernel" if full else "")) if st.persistent else
+                                   (f"whole decode step (embed + {spec.total_layers} x tiny_layer_kernel: pre-norm, "
+                                    "router, SwiGLU and combine in one launch per layer)"),
                          "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peaks["source"]},
             "cpu_baseline": cpu,
             "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": spec.n_codebooks * 4, "d2h_bytes_per_step": spec.d * 4},
-            "gpu_launches": (1 + spec.total_layers + (1 if full else 0)) * args.steps,
+            "gpu_launches": ((1 if st.persistent else 1 + spec.total_layers) + (1 if full else 0)) * args.steps,
             "clocks": clk.summary(),
             "device_errors": dev_errors,
         }

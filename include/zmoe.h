@@ -301,6 +301,51 @@ ZMOE_API zmoe_status zmoe_output_heads(const float* h, const float* gamma, float
 ZMOE_API zmoe_status zmoe_speaker_prefix(const float* e, const void* w_spk, zmoe_dtype dtype, const float* b_spk,
                                          int B, int d, int n_in, float* out, zmoe_stream_t stream);
 
+/* One layer of zmoe_decode_stack (bf16 weights, the layouts of zmoe_moe_layer). */
+typedef struct zmoe_stack_layer {
+  const void* w_router;     /* bf16 [E, d]; NULL only for a dense FFN layer (E == 1, k == 1: gate 1) */
+  const float* logit_bias;  /* [E] or NULL: enters the gates and the selection */
+  const float* sel_bias;    /* [E] or NULL: selection only */
+  const float* gamma;       /* [d] the layer's pre-norm gain */
+  const void* w_gate;       /* bf16 [E, f, d] */
+  const void* w_up;         /* bf16 [E, f, d] */
+  const void* w_down;       /* bf16 [E, d, f] */
+  int E;                    /* experts, 1..64 */
+  int k;                    /* experts per token, 1 or 2, <= E */
+} zmoe_stack_layer;
+
+/* Bytes of workspace zmoe_decode_stack needs for layers of at most E_max experts; 0 when these
+ * sizes are not supported (see the limits below). */
+ZMOE_API size_t zmoe_decode_stack_workspace_size(int n_layers, int d, int f, int E_max);
+
+/*
+ * The batch-1 decode stack in one call ([DIGEST] item 5: the decoder input is the RMSNorm of the
+ * summed embeddings of the codebook frame; the FFN side of the decoder is a stack of pre-norm
+ * residual blocks, dense or MoE, top-1 and top-2 in the last MoE layer; [ROUTING] section 2.1).
+ * One token (T = 1):
+ *   if ids:  h = RMSNorm(sum_j tables[j, ids[j]]) * gamma0     (fp32 sum, as zmoe_embed_sum_rmsnorm)
+ *   for l < n_layers:  x = bf16(RMSNorm(h) * layers[l].gamma)
+ *                      h = h + sum_{i<k} gate_i * FFN_{e_i}(x)  (router, top-k and gates as zmoe_route;
+ *                                                                a dense layer: expert 0, gate 1)
+ *   ids: int32 [N] or NULL (then h holds the stack input on entry); tables: bf16 [N, V, d]; gamma0:
+ *   f32 [d]; h: f32 [d], in place (the final residual stream on return).
+ *   Optional outputs (NULL to skip): layer_idx int32 [n_layers, 2] and layer_gates f32 [n_layers, 2]
+ *   (the chosen experts and gates of each layer in slot order; -1 / 0 past k), layer_h f32
+ *   [n_layers, d] (h entering each layer), layer_x bf16 [n_layers, d] (each layer's routed input).
+ *   One persistent cooperative launch over all SMs (plus a 256-byte memset of the workspace): every
+ *   CTA repeats the pre-norm and routing, the weights stream through shared memory, two grid
+ *   barriers per layer.  Same arithmetic as n_layers zmoe_moe_layer calls with T = 1 (fp32 sums in a
+ *   fixed order; the router's summation order differs, so ids can differ only on near-ties).
+ *   Limits: n_layers <= 32, d % 8 == 0, d <= 4096, f % 8 == 0, N <= 32, and the per-CTA buffers
+ *   must fit one SM (14 ring slots of max(4 d, 2 f) bytes, the largest router E d 2 bytes, 8 d +
+ *   8 f bytes): d = 2048, f = 3072, E = 16 fits; larger sizes return ZMOE_ERR_UNSUPPORTED.  Ids
+ *   outside [0, V) count a device error and contribute nothing.
+ */
+ZMOE_API zmoe_status zmoe_decode_stack(const zmoe_stack_layer* layers, int n_layers, int d, int f, float eps,
+                                       const int32_t* ids, const void* tables, const float* gamma0, int N, int V,
+                                       float* h, int32_t* layer_idx, float* layer_gates, float* layer_h,
+                                       void* layer_x, void* workspace, size_t ws_bytes, zmoe_stream_t stream);
+
 /*
  * Reads and clears the device error counters of the current device.  Synchronises
  * `stream` (and the device) first.  *count = data errors (ids or indices out of range)

@@ -121,7 +121,8 @@ class DecodeStack:
     weights, also the codebook heads and the greedy next frame (``next_ids``)."""
 
     def __init__(self, tables: torch.Tensor, gamma0: torch.Tensor, layers: List[MoEWeights], eps: float = 1e-6,
-                 T: int = 1, w_heads: Optional[torch.Tensor] = None, gamma_out: Optional[torch.Tensor] = None):
+                 T: int = 1, w_heads: Optional[torch.Tensor] = None, gamma_out: Optional[torch.Tensor] = None,
+                 persistent: Optional[bool] = None):
         self.tables, self.gamma0, self.layers, self.eps, self.T = tables, gamma0, layers, eps, T
         L0 = layers[0]
         dev = tables.device
@@ -139,11 +140,36 @@ class DecodeStack:
         self.layer_inputs: List[torch.Tensor] = []
         self.layer_h: List[torch.Tensor] = []
         self.layer_idx: List[torch.Tensor] = []
+        # One token per step: the whole stack (embedding included) is one zmoe_decode_stack call when
+        # its sizes are supported; otherwise (or with persistent=False) one zmoe_moe_layer call per layer.
+        nL, d, f = len(layers), L0.d, L0.f
+        ws = Z.zmoe_decode_stack_workspace_size(nL, d, f, max(L.E for L in layers)) if T == 1 else 0
+        if persistent and ws == 0:
+            raise ValueError("zmoe_decode_stack does not support these sizes")
+        self.persistent = ws > 0 and persistent is not False and L0.dtype == torch.bfloat16
+        if self.persistent:
+            self.stack_ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+            self.stack_arr = Z.stack_layers(layers)
+            self.rec = dict(layer_idx=torch.empty((nL, 2), dtype=torch.int32, device=dev),
+                            layer_gates=torch.empty((nL, 2), dtype=torch.float32, device=dev),
+                            layer_h=torch.empty((nL, d), dtype=torch.float32, device=dev),
+                            layer_x=torch.empty((nL, d), dtype=L0.dtype, device=dev))
 
     def step(self, ids: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         """One decode step; returns the final fp32 residual stream h [T, d]."""
         if ids is not None:
             self.ids.copy_(ids)
+        if self.persistent:
+            Z.zmoe_decode_stack(self.layers, self.h, self.eps, ids=self.ids, tables=self.tables, gamma0=self.gamma0,
+                                outs=self.rec if self.record_inputs else None, workspace=self.stack_ws, stream=stream,
+                                layer_array=self.stack_arr)
+            if self.record_inputs:
+                r = self.rec
+                self.layer_h = [r["layer_h"][l:l + 1] for l in range(len(self.layers))]
+                self.layer_inputs = [r["layer_x"][l:l + 1] for l in range(len(self.layers))]
+                self.layer_idx = [r["layer_idx"][l:l + 1, :L.k] for l, L in enumerate(self.layers)]
+            self._heads(stream)
+            return self.h
         Z.zmoe_embed_sum_rmsnorm(self.ids, self.tables, self.gamma0, self.eps, out=self.h, stream=stream)
         if self.record_inputs:
             self.layer_inputs, self.layer_h, self.layer_idx = [], [], []
@@ -157,16 +183,19 @@ class DecodeStack:
             if self.record_inputs:
                 self.layer_inputs.append(self.x.clone())
                 self.layer_idx.append(R.idx.clone())
+        self._heads(stream)
+        return self.h
+
+    def _heads(self, stream=None):
         if self.w_heads is not None:
             outs = dict(ids=self.next_ids, x=self.head_x) if self.record_inputs else dict(ids=self.next_ids)
             Z.zmoe_output_heads(self.h, self.w_heads, self.gamma_out, self.eps, outs=outs, workspace=self.head_ws,
                                 stream=stream)
-        return self.h
 
 
 def stack_from_bits(tables_bits, gamma0, layer_small, expert_bits, n_layers: int, E: int, d: int, f: int,
                     k_of, eps: float = 1e-6, T: int = 1, device="cuda", E_of=None, heads_bits=None,
-                    gamma_out=None) -> DecodeStack:
+                    gamma_out=None, persistent: Optional[bool] = None) -> DecodeStack:
     """Builds a DecodeStack on the device from host arrays.
 
     tables_bits: uint16 [N, V, d] bf16 bit patterns; gamma0: f32 [d]; layer_small(l) -> (W_r f32 [E, d]
@@ -197,4 +226,4 @@ def stack_from_bits(tables_bits, gamma0, layer_small, expert_bits, n_layers: int
     tables = bits_to_dev(tables_bits)
     heads = bits_to_dev(heads_bits) if heads_bits is not None else None
     g_out = torch.from_numpy(gamma_out).to(device) if gamma_out is not None else None
-    return DecodeStack(tables, torch.from_numpy(gamma0).to(device), layers, eps, T, heads, g_out)
+    return DecodeStack(tables, torch.from_numpy(gamma0).to(device), layers, eps, T, heads, g_out, persistent)

@@ -54,7 +54,15 @@ SIGNATURES = {
                             _P, _S, _P]),
     "zmoe_get_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "zmoe_debug_inject_timeout": (_I, [ctypes.c_uint32, ctypes.c_uint64]),
+    "zmoe_decode_stack_workspace_size": (_S, [_I, _I, _I, _I]),
+    "zmoe_decode_stack": (_I, [_P, _I, _I, _I, _F, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P]),
 }
+
+
+class StackLayer(ctypes.Structure):
+    """zmoe_stack_layer (include/zmoe.h)."""
+    _fields_ = [("w_router", _P), ("logit_bias", _P), ("sel_bias", _P), ("gamma", _P), ("w_gate", _P),
+                ("w_up", _P), ("w_down", _P), ("E", _I), ("k", _I)]
 
 
 class ZmoeError(RuntimeError):
@@ -392,6 +400,58 @@ def zmoe_speaker_prefix(e: torch.Tensor, w_spk: torch.Tensor, b_spk: Optional[to
     _check(lib().zmoe_speaker_prefix(_ptr(e), _ptr(w_spk), _dtype_code(w_spk.dtype), _ptr(b_spk), B, d, n_in, _ptr(y),
                                      _stream(stream)), "zmoe_speaker_prefix")
     return y
+
+
+def zmoe_decode_stack_workspace_size(n_layers: int, d: int, f: int, E_max: int) -> int:
+    """Bytes of workspace for zmoe_decode_stack; 0 when these sizes are not supported."""
+    return int(lib().zmoe_decode_stack_workspace_size(n_layers, d, f, E_max))
+
+
+def stack_layers(layers) -> ctypes.Array:
+    """The zmoe_stack_layer array of a list of MoEWeights-like objects (w_router, logit_bias, sel_bias,
+    gamma, w_gate, w_up, w_down, k).  The tensors must stay alive while the array is used."""
+    arr = (StackLayer * len(layers))()
+    for i, L in enumerate(layers):
+        for name in ("w_gate", "w_up", "w_down"):
+            _need(getattr(L, name), name, torch.bfloat16, 3)
+        _need(L.gamma, "gamma", torch.float32, 1)
+        arr[i] = StackLayer(_ptr(L.w_router), _ptr(L.logit_bias), _ptr(L.sel_bias), _ptr(L.gamma), _ptr(L.w_gate),
+                            _ptr(L.w_up), _ptr(L.w_down), L.w_gate.shape[0], L.k)
+    return arr
+
+
+def zmoe_decode_stack(layers, h: torch.Tensor, eps: float = 1e-6, ids: Optional[torch.Tensor] = None,
+                      tables: Optional[torch.Tensor] = None, gamma0: Optional[torch.Tensor] = None,
+                      outs: Optional[dict] = None, workspace: Optional[torch.Tensor] = None, stream=None,
+                      layer_array: Optional[ctypes.Array] = None) -> torch.Tensor:
+    """The batch-1 stack in one call: h [1, d] (or [d]) f32 in place; with ``ids`` [N] / [1, N] the
+    stack input is the embedding sum + RMSNorm of ``tables`` [N, V, d] with ``gamma0``.
+
+    ``outs`` may hold ``layer_idx`` int32 [L, 2], ``layer_gates`` f32 [L, 2], ``layer_h`` f32 [L, d] and
+    ``layer_x`` bf16 [L, d].  ``layer_array`` (from ``stack_layers``) skips rebuilding the descriptors.
+    """
+    _need(h, "h", torch.float32)
+    d = h.shape[-1]
+    n = len(layers)
+    f = layers[0].w_gate.shape[1]
+    outs = outs or {}
+    arr = layer_array if layer_array is not None else stack_layers(layers)
+    N = V = 0
+    if ids is not None:
+        _need(ids, "ids", torch.int32)
+        _need(tables, "tables", torch.bfloat16, 3)
+        N, V = tables.shape[0], tables.shape[1]
+    ws_bytes = zmoe_decode_stack_workspace_size(n, d, f, max(L.w_gate.shape[0] for L in layers))
+    if ws_bytes == 0:
+        raise ZmoeError(2, "zmoe_decode_stack", "these sizes are not supported")
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=h.device)
+    _check(lib().zmoe_decode_stack(ctypes.cast(arr, _P), n, d, f, float(eps), _ptr(ids), _ptr(tables), _ptr(gamma0),
+                                   N, V, _ptr(h), _ptr(outs.get("layer_idx")), _ptr(outs.get("layer_gates")),
+                                   _ptr(outs.get("layer_h")), _ptr(outs.get("layer_x")), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "zmoe_decode_stack")
+    return h
 
 
 def zmoe_get_device_errors(stream=None) -> int:

@@ -1,6 +1,7 @@
 """The batch-1 decode stack (embedding sum + RMSNorm, 24 pre-norm MoE layers, top-2 in the last) on the
 GPU vs the oracle; and the decoder's full 28-layer FFN stack (3 dense layers, the 24 MoE layers, 1 dense
-layer), each layer one zmoe_moe_layer call.
+layer).  Both run as one zmoe_decode_stack launch (the path the benchmark times); the 24-layer stack is
+also checked as one zmoe_moe_layer call per layer.
 
 Full size: 24 layers x 16 experts of d_model 2048, d_ff 3072 (14.5 GB of bf16 weights), in the launch
 configuration the benchmark times (T = 1 per step).  Layer by layer the oracle is teacher-forced: it
@@ -16,7 +17,8 @@ import torch
 
 import oracle
 from moe_inputs import StackSpec, bf16_bits, stack_expert_bits
-from sparse_moe_decoder_b200.layer import stack_from_bits
+from sparse_moe_decoder_b200 import zmoe_get_device_errors
+from sparse_moe_decoder_b200.layer import DecodeStack, stack_from_bits
 from tests.gpu_util import MARGIN_EXEMPT, assert_close, host, require_gpu
 
 pytestmark = pytest.mark.gpu
@@ -44,7 +46,43 @@ def stack28():
 
 
 def test_stack_teacher_forced_layers(stack):
-    check_teacher_forced(*stack, STEPS)
+    spec, st = stack
+    assert st.persistent, "T = 1 at d = 2048, f = 3072, E = 16 runs as one zmoe_decode_stack launch"
+    check_teacher_forced(spec, st, STEPS)
+
+
+def test_stack_per_layer_calls_teacher_forced(stack):
+    """The same weights, one zmoe_moe_layer call (tiny-batch launch) per layer."""
+    spec, st = stack
+    st2 = DecodeStack(st.tables, st.gamma0, st.layers, st.eps, 1, persistent=False)
+    assert not st2.persistent
+    check_teacher_forced(spec, st2, 1)
+
+
+def test_stack_one_launch_matches_per_layer_calls(stack):
+    """Both paths from the same codes: the same routes (unless a near-tie flips) and the same final stream
+    within the bf16 bar."""
+    spec, st = stack
+    st2 = DecodeStack(st.tables, st.gamma0, st.layers, st.eps, 1, persistent=False)
+    codes = torch.from_numpy(spec.codes(3)[2:3]).cuda()
+    st.record_inputs = st2.record_inputs = True
+    a = host(st.step(codes)).astype(np.float64)
+    b = host(st2.step(codes)).astype(np.float64)
+    same = all(np.array_equal(host(st.layer_idx[l]), host(st2.layer_idx[l])) for l in range(spec.n_layers))
+    if same:
+        assert_close(a, b, "bf16", "one launch vs per-layer calls")
+    assert zmoe_get_device_errors() == 0
+
+
+def test_stack_bad_code_is_counted(stack):
+    """An id outside [0, V) counts a device error and contributes nothing (no out-of-range read)."""
+    spec, st = stack
+    codes = spec.codes(1).copy()
+    codes[0, 3] = 5000
+    st.record_inputs = False
+    st.step(torch.from_numpy(codes).cuda())
+    assert zmoe_get_device_errors() >= 1
+    assert zmoe_get_device_errors() == 0
 
 
 def test_full_ffn_stack_teacher_forced(stack28):
