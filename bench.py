@@ -53,6 +53,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle timing leg")
+    ap.add_argument("--h-pair", action="store_true",
+                    help="prefill: carry h as the bf16 pair with the bf16 down weights instead of f16 h with the "
+                         "prepared f16 down weights")
     ap.add_argument("--weight-copies", type=int, default=0,
                     help="device copies of the layer weights used in rotation (0: 4 for the decode step, else 1)")
     return ap.parse_args(argv)
@@ -583,14 +586,29 @@ def run_layer(args):
     x = torch.from_numpy(L.x).to("cuda", dt)
     stream = torch.cuda.current_stream()
 
+    # decode sizes: the whole layer is one zmoe_moe_layer call (one cooperative launch); prefill sizes
+    # time the four entry points separately, with events around the grouped SwiGLU.  Prefill carries h in
+    # f16 with the f16 down weights, prepared once here (a load-time conversion, outside the timing).
+    fused = L.T * L.k < 64 * L.E
+    f16h = not fused and not args.h_pair
+    if f16h:
+        for W in Ws:
+            W.prepare_f16()
+        torch.cuda.synchronize()
+
     def step(i):
         return R.run(x, Ws[i % n_copies])
 
-    # decode sizes: the whole layer is one zmoe_moe_layer call (one cooperative launch); prefill sizes
-    # time the four entry points separately, with events around the grouped SwiGLU
-    fused = L.T * L.k < 64 * L.E
+    def layer_call(xin, W):
+        return R.run_f16h(xin, W) if f16h else R.run(xin, W)
+
     for i in range(args.warmup):
-        step(i) if fused else R.run_steps(x, Ws[i % n_copies])
+        if fused:
+            step(i)
+        elif f16h:
+            R.run_steps_f16h(x, Ws[i % n_copies])
+        else:
+            R.run_steps(x, Ws[i % n_copies])
     torch.cuda.synchronize()
     counts = np.bincount(R.idx.cpu().numpy().ravel(), minlength=L.E)
     experts_touched = int((counts > 0).sum())
@@ -614,8 +632,12 @@ def run_layer(args):
             Z.zmoe_route(x, W.w_router, W.k, W.logit_bias, W.sel_bias, outs=(R.idx, R.gates, R.margin))
             Z.zmoe_permute(R.idx, x, W.E, outs=R.perm_outs, workspace=R.perm_ws)
             ev_ffn[i][0].record(stream)
-            Z.zmoe_grouped_swiglu(R.perm_outs["x_perm"], R.perm_outs["offsets"], W.w_gate, W.w_up, W.w_down,
-                                  h=R.h, y_perm=R.y_perm, workspace=R.ffn_ws)
+            if f16h:
+                Z.zmoe_grouped_swiglu_f16h(R.perm_outs["x_perm"], R.perm_outs["offsets"], W.w_gate, W.w_up,
+                                           W.w_down_f16, W.down_scale, h=R.h16, y_perm=R.y_perm)
+            else:
+                Z.zmoe_grouped_swiglu(R.perm_outs["x_perm"], R.perm_outs["offsets"], W.w_gate, W.w_up, W.w_down,
+                                      h=R.h, y_perm=R.y_perm, workspace=R.ffn_ws)
             ev_ffn[i][1].record(stream)
             Z.zmoe_combine(R.y_perm, R.perm_outs["inv_perm"], R.gates, None, out=R.y)
         ev1.record(stream)
@@ -639,7 +661,7 @@ def run_layer(args):
     x_dev = torch.empty_like(x)
     for i in range(min(3, args.warmup)):
         x_dev.copy_(x_host, non_blocking=True)
-        R.run(x_dev, Ws[i % n_copies])
+        layer_call(x_dev, Ws[i % n_copies])
         y_host.copy_(R.y, non_blocking=True)
     torch.cuda.synchronize()
     if world > 1:
@@ -648,7 +670,7 @@ def run_layer(args):
     e0.record(stream)
     for i in range(args.steps):
         x_dev.copy_(x_host, non_blocking=True)
-        R.run(x_dev, Ws[i % n_copies])
+        layer_call(x_dev, Ws[i % n_copies])
         y_host.copy_(R.y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -667,7 +689,8 @@ def run_layer(args):
     touched = int((counts > 0).sum())
     M = int(counts.sum())
     weight_bytes = touched * 3 * L.f * L.d * bpe
-    act_bytes = M * L.d * bpe + 2 * (M * 2 * L.f * bpe) + M * L.d * 4   # x_perm in, h pair out + in, y_perm out
+    h_cols = L.f if f16h else 2 * L.f
+    act_bytes = M * L.d * bpe + 2 * (M * h_cols * bpe) + M * L.d * 4   # x_perm in, h out + in, y_perm out
     if fused:
         # the launch also reads x and W_r, writes and re-reads x_perm, and writes y
         act_bytes += L.T * L.d * bpe + L.E * L.d * bpe + M * L.d * bpe + L.T * L.d * 4
@@ -684,7 +707,9 @@ def run_layer(args):
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"],
                 "traffic": traffic_from_profiles(f"grouped_swiglu_cfg{args.config}"),
-                "kernel": "zmoe_grouped_swiglu (tc_ffn_kernel: gate/up, then down)",
+                "kernel": ("zmoe_grouped_swiglu_f16h (tc_ffn_kernel on CTA pairs: gate/up, then down over f16 h)"
+                           if f16h else "zmoe_grouped_swiglu (tc_ffn_kernel on CTA pairs: gate/up, then down over "
+                                        "the bf16 h pair)"),
                 "algorithmic_flops_per_launch": flops, "peak_source": peaks["source"],
                 "peak_kind": "burst (the SwiGLU is timed alone, between the other calls of the step)"}
 
@@ -706,11 +731,13 @@ def run_layer(args):
                           if n_copies > 1 else "inputs larger than L2 (one layer's weights: 604 MB, x and the "
                           "permuted rows another 0.2-0.3 GB)"),
                    "experts_touched": experts_touched,
-                   "expert_loads": counts.tolist()},
+                   "expert_loads": counts.tolist(),
+                   "h": ("f16 (down weights converted once to f16 with a power-of-two scale per expert)" if f16h
+                         else "bf16 pair (h_hi + h_lo)" if not fused else "bf16 pair")},
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "call": "zmoe_moe_layer"},
+                "call": "zmoe_moe_layer_f16h" if f16h else "zmoe_moe_layer"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "ffn_ms_per_step": ffn_ms,

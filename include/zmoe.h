@@ -174,6 +174,37 @@ ZMOE_API zmoe_status zmoe_permute_noalloc(const int32_t* expert_idx, const void*
                                           int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm,
                                           int32_t* inv_perm, void* x_perm, zmoe_stream_t stream);
 
+/*
+ * One-time preparation of the down-projection weights for the f16 prefill path (no counterpart on
+ * the pages: a storage format of the weights).  Both operands of a tensor-core MMA share one 16-bit
+ * format, and the prefill down GEMM carries h in f16 (11 significant bits; one bf16 h costs up to 3%
+ * of the output RMS), so W_down is converted once to f16, each expert scaled by a power of two that
+ * puts its largest |w| in [2^14, 2^15):
+ *   w_down_f16[e] = f16(w_down[e] * 2^s_e),   down_scale[e] = 2^-s_e
+ * exact for every weight within 2^28 of the expert's largest (smaller ones round with an absolute
+ * error below 2^-39 of the largest).  w_down: bf16 [E, d, f]; w_down_f16: f16 [E, d, f] (caller
+ * memory, 16-byte aligned); down_scale: f32 [E]; workspace: >= 4 E bytes of device scratch.
+ */
+ZMOE_API zmoe_status zmoe_prepare_w_down_f16(const void* w_down, int E, int d, int f, void* w_down_f16,
+                                             float* down_scale, void* workspace, size_t ws_bytes,
+                                             zmoe_stream_t stream);
+
+/*
+ * The grouped SwiGLU of zmoe_grouped_swiglu for prefill-size batches with h carried in f16 and the
+ * prepared down weights (zmoe_prepare_w_down_f16):
+ *   h[r]      = f16(silu(W_gate[e] x_perm[r]) * (W_up[e] x_perm[r]))             [f] f16
+ *   y_perm[r] = down_scale[e] * (W_down_f16[e] h[r])                              [d] f32
+ * x_perm, w_gate, w_up: bf16 as zmoe_grouped_swiglu; w_down_f16: f16 [E, d, f]; down_scale: f32 [E];
+ * h: f16 [M_total, f] (caller scratch that also exposes the hidden activations); offsets on the device.
+ * An |h| beyond f16's range (65504) counts a device error (zmoe_get_device_errors).  Runs the CTA-pair
+ * tcgen05 kernels at any M_total (built for >= 64 rows per expert on average); d % 256 == 0,
+ * f % 256 == 0, 16-byte aligned.  No workspace.
+ */
+ZMOE_API zmoe_status zmoe_grouped_swiglu_f16h(const void* x_perm, const int32_t* offsets, int M_total,
+                                              const void* w_gate, const void* w_up, const void* w_down_f16,
+                                              const float* down_scale, int E, int d, int f, void* h, float* y_perm,
+                                              zmoe_stream_t stream);
+
 /* Bytes of workspace zmoe_grouped_swiglu needs for these sizes. */
 ZMOE_API size_t zmoe_grouped_swiglu_workspace_size(int M_total, int E, int d, int f, zmoe_dtype dtype);
 
@@ -300,6 +331,23 @@ ZMOE_API zmoe_status zmoe_output_heads(const float* h, const float* gamma, float
  */
 ZMOE_API zmoe_status zmoe_speaker_prefix(const float* e, const void* w_spk, zmoe_dtype dtype, const float* b_spk,
                                          int B, int d, int n_in, float* out, zmoe_stream_t stream);
+
+/* Bytes of workspace zmoe_moe_layer_f16h needs. */
+ZMOE_API size_t zmoe_moe_layer_f16h_workspace_size(int T, int d, int f, int E, int k);
+
+/*
+ * zmoe_moe_layer (same arguments, bf16) with the prepared f16 down weights (zmoe_prepare_w_down_f16) in
+ * place of w_down, for prefill-size batches: pre-norm (with gamma), zmoe_route, zmoe_permute,
+ * zmoe_grouped_swiglu_f16h, zmoe_combine, in order on `stream`.  The same layer as zmoe_moe_layer up to
+ * h's rounding to f16 (~3e-3 of the output RMS at most on the skewed prefill layers).
+ * d % 256 == 0, f % 256 == 0.
+ */
+ZMOE_API zmoe_status zmoe_moe_layer_f16h(const void* x, const float* h, const float* gamma, float eps,
+                                         const void* w_router, const float* logit_bias, const float* sel_bias,
+                                         const void* w_gate, const void* w_up, const void* w_down_f16,
+                                         const float* down_scale, int T, int d, int f, int E, int k, float* y,
+                                         int32_t* expert_idx, float* gates, float* margin, void* x_norm,
+                                         void* workspace, size_t ws_bytes, zmoe_stream_t stream);
 
 /* One layer of zmoe_decode_stack (bf16 weights, the layouts of zmoe_moe_layer). */
 typedef struct zmoe_stack_layer {

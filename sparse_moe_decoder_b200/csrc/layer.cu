@@ -192,4 +192,60 @@ zmoe_status zmoe_moe_layer_fp8(const void* x, const float* h, const float* gamma
                          s_up, s_down);
 }
 
+size_t zmoe_moe_layer_f16h_workspace_size(int T, int d, int f, int E, int k) {
+  using namespace zmoe;
+  if (T <= 0 || d < 1 || f < 1 || E < 1 || E > 64 || (k != 1 && k != 2)) return 0;
+  return seq_ws(T, E, d, f, k, ZMOE_BF16).total;
+}
+
+zmoe_status zmoe_moe_layer_f16h(const void* x, const float* h, const float* gamma, float eps, const void* w_router,
+                                const float* logit_bias, const float* sel_bias, const void* w_gate, const void* w_up,
+                                const void* w_down_f16, const float* down_scale, int T, int d, int f, int E, int k,
+                                float* y, int32_t* expert_idx, float* gates, float* margin, void* x_norm,
+                                void* workspace, size_t ws_bytes, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_moe_layer_f16h");
+  using namespace zmoe;
+  ZMOE_REQUIRE(T >= 0, "zmoe_moe_layer_f16h: T must be >= 0");
+  ZMOE_REQUIRE(E >= 1 && E <= 64, "zmoe_moe_layer_f16h: E must be in [1, 64]");
+  ZMOE_REQUIRE((k == 1 || k == 2) && k <= E, "zmoe_moe_layer_f16h: k must be 1 or 2 and <= E");
+  ZMOE_REQUIRE(d >= 256 && d % 256 == 0 && f >= 256 && f % 256 == 0,
+               "zmoe_moe_layer_f16h: d and f must be multiples of 256");
+  if (T == 0) return ZMOE_OK;
+  ZMOE_REQUIRE((w_router || E == 1) && w_gate && w_up && w_down_f16 && down_scale && y,
+               "zmoe_moe_layer_f16h: NULL pointer (w_router may be NULL only when E == 1)");
+  ZMOE_REQUIRE(gamma ? h != nullptr : x != nullptr, "zmoe_moe_layer_f16h: needs x, or h with gamma");
+  ZMOE_REQUIRE((!x || aligned16(x)) && (!h || aligned16(h)) && aligned16(y) && (!w_router || aligned16(w_router)) &&
+                   aligned16(w_gate) && aligned16(w_up) && aligned16(w_down_f16) && (!x_norm || aligned16(x_norm)) &&
+                   (!gamma || aligned16(gamma)),
+               "zmoe_moe_layer_f16h: pointers must be 16-byte aligned");
+  const size_t need = zmoe_moe_layer_f16h_workspace_size(T, d, f, E, k);
+  if (!workspace || ws_bytes < need)
+    return fail(ZMOE_ERR_WORKSPACE_TOO_SMALL,
+                "zmoe_moe_layer_f16h: workspace smaller than zmoe_moe_layer_f16h_workspace_size()");
+  clear_error();
+  const SeqWs W = seq_ws(T, E, d, f, k, ZMOE_BF16);
+  unsigned char* w = static_cast<unsigned char*>(workspace);
+  const void* xin = x;
+  if (gamma) {
+    void* xn = x_norm ? x_norm : static_cast<void*>(w + W.x_norm);
+    zmoe_status st = zmoe_rmsnorm(h, ZMOE_F32, gamma, eps, T, d, xn, ZMOE_BF16, stream);
+    if (st != ZMOE_OK) return st;
+    xin = xn;
+  }
+  int32_t* idx = expert_idx ? expert_idx : reinterpret_cast<int32_t*>(w + W.idx);
+  float* g = gates ? gates : reinterpret_cast<float*>(w + W.gates);
+  zmoe_status st = zmoe_route(xin, w_router, ZMOE_BF16, logit_bias, sel_bias, T, d, E, k, idx, g, margin, stream);
+  if (st != ZMOE_OK) return st;
+  int32_t* inv = reinterpret_cast<int32_t*>(w + W.inv_perm);
+  st = zmoe_permute(idx, xin, ZMOE_BF16, T, d, E, k, reinterpret_cast<int32_t*>(w + W.counts),
+                    reinterpret_cast<int32_t*>(w + W.offsets), reinterpret_cast<int32_t*>(w + W.perm), inv,
+                    w + W.x_perm, w + W.perm_ws, W.perm_ws_bytes, stream);
+  if (st != ZMOE_OK) return st;
+  float* yp = reinterpret_cast<float*>(w + W.y_perm);
+  st = zmoe_grouped_swiglu_f16h(w + W.x_perm, reinterpret_cast<int32_t*>(w + W.offsets), T * k, w_gate, w_up,
+                                w_down_f16, down_scale, E, d, f, w + W.h, yp, stream);
+  if (st != ZMOE_OK) return st;
+  return zmoe_combine(yp, inv, g, h, T, d, k, y, stream);
+}
+
 }  // extern "C"

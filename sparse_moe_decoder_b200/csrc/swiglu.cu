@@ -23,6 +23,9 @@ bool grouped_swiglu_dec_tc_supported(int d, int f);
 zmoe_status grouped_swiglu_tc(const uint16_t* x_perm, const int32_t* offsets, int M_total, const uint16_t* w_gate,
                               const uint16_t* w_up, const uint16_t* w_down, int E, int d, int f, uint16_t* h,
                               float* y_perm, void* ws, size_t ws_bytes, cudaStream_t s);
+zmoe_status grouped_swiglu_tc_f16h(const uint16_t* x_perm, const int32_t* offsets, int M_total, const uint16_t* w_gate,
+                                   const uint16_t* w_up, const uint16_t* w_down_f16, const float* down_scale, int E,
+                                   int d, int f, uint16_t* h, float* y_perm, cudaStream_t s);
 size_t grouped_swiglu_tc_workspace(int M_total, int E, int d, int f);
 bool grouped_swiglu_tc_supported(int d, int f);
 
@@ -150,6 +153,31 @@ zmoe_status zmoe_grouped_swiglu(const void* x_perm, const int32_t* offsets, int 
     return fail(ZMOE_ERR_WORKSPACE_TOO_SMALL,
                 "zmoe_grouped_swiglu: workspace smaller than zmoe_grouped_swiglu_workspace_size()");
   return grouped_swiglu_dec_tc(xp, offsets, M_total, wg, wu, wd, E, d, f, hh, y_perm, workspace, s);
+}
+
+zmoe_status zmoe_grouped_swiglu_f16h(const void* x_perm, const int32_t* offsets, int M_total, const void* w_gate,
+                                     const void* w_up, const void* w_down_f16, const float* down_scale, int E, int d,
+                                     int f, void* h, float* y_perm, zmoe_stream_t stream) {
+  ZMOE_TRACE("zmoe_grouped_swiglu_f16h");
+  using namespace zmoe;
+  ZMOE_REQUIRE(M_total >= 0, "zmoe_grouped_swiglu_f16h: M_total must be >= 0");
+  ZMOE_REQUIRE(E >= 1 && E <= 64, "zmoe_grouped_swiglu_f16h: E must be in [1, 64]");
+  ZMOE_REQUIRE(d >= 256 && f >= 256 && d % 256 == 0 && f % 256 == 0,
+               "zmoe_grouped_swiglu_f16h: d and f must be multiples of 256");
+  ZMOE_REQUIRE(offsets != nullptr, "zmoe_grouped_swiglu_f16h: offsets is NULL");
+  if (M_total == 0) return ZMOE_OK;
+  ZMOE_REQUIRE(x_perm && w_gate && w_up && w_down_f16 && down_scale && h && y_perm,
+               "zmoe_grouped_swiglu_f16h: NULL pointer");
+  ZMOE_REQUIRE(aligned16(x_perm) && aligned16(w_gate) && aligned16(w_up) && aligned16(w_down_f16) && aligned16(h) &&
+                   aligned16(y_perm),
+               "zmoe_grouped_swiglu_f16h: pointers must be 16-byte aligned");
+  ZMOE_REQUIRE(static_cast<long long>(M_total) * (d > f ? d : f) <= 0x7fffffffLL,
+               "zmoe_grouped_swiglu_f16h: M_total * max(d, f) overflows int32");
+  clear_error();
+  return grouped_swiglu_tc_f16h(static_cast<const uint16_t*>(x_perm), offsets, M_total,
+                                static_cast<const uint16_t*>(w_gate), static_cast<const uint16_t*>(w_up),
+                                static_cast<const uint16_t*>(w_down_f16), down_scale, E, d, f, static_cast<uint16_t*>(h),
+                                y_perm, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

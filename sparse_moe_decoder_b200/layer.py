@@ -36,6 +36,14 @@ class MoEWeights:
     logit_bias: Optional[torch.Tensor] = None   # f32 [E]
     gamma: Optional[torch.Tensor] = None        # f32 [d], pre-norm gain (stack only)
     k: int = 1
+    w_down_f16: Optional[torch.Tensor] = None   # f16 [E, d, f], prepared by prepare_f16()
+    down_scale: Optional[torch.Tensor] = None   # f32 [E]
+
+    def prepare_f16(self) -> "MoEWeights":
+        """The prefill path's f16 copy of W_down (zmoe_prepare_w_down_f16), made once."""
+        if self.w_down_f16 is None:
+            self.w_down_f16, self.down_scale = Z.zmoe_prepare_w_down_f16(self.w_down)
+        return self
 
     @property
     def E(self) -> int:
@@ -87,6 +95,7 @@ class MoELayerRunner:
         self.ffn_ws = torch.empty(max(Z.zmoe_grouped_swiglu_workspace_size(M, E, d, f, dtype), 16),
                                   dtype=torch.uint8, device=dev)
         self.y = torch.empty((T, d), dtype=torch.float32, device=dev)
+        self.h16 = torch.empty((M, f), dtype=torch.float16, device=dev) if dtype == torch.bfloat16 else None
         self.layer_ws = torch.empty(max(Z.zmoe_moe_layer_workspace_size(T, d, f, E, k, dtype), 16), dtype=torch.uint8,
                                     device=dev)
 
@@ -103,6 +112,34 @@ class MoELayerRunner:
                                 logit_bias=W.logit_bias, sel_bias=W.sel_bias,
                                 out=self.y if out is None else out, outs=outs, workspace=self.layer_ws,
                                 stream=stream)
+
+    def run_f16h(self, x: Optional[torch.Tensor], W: MoEWeights, residual: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None, stream=None, gamma: Optional[torch.Tensor] = None,
+                 eps: float = 1e-6) -> torch.Tensor:
+        """The layer in one zmoe_moe_layer_f16h call (prefill sizes; W needs prepare_f16())."""
+        outs = dict(expert_idx=self.idx, gates=self.gates, margin=self.margin)
+        return Z.zmoe_moe_layer_f16h(W.w_router, W.w_gate, W.w_up, W.w_down_f16, W.down_scale, W.k, x=x, h=residual,
+                                     gamma=gamma, eps=eps, logit_bias=W.logit_bias, sel_bias=W.sel_bias,
+                                     out=self.y if out is None else out, outs=outs, workspace=self.layer_ws16,
+                                     stream=stream)
+
+    @property
+    def layer_ws16(self) -> torch.Tensor:
+        if not hasattr(self, "_layer_ws16"):
+            n = int(Z.lib().zmoe_moe_layer_f16h_workspace_size(self.T, self.d, self.f, self.E, self.k))
+            self._layer_ws16 = torch.empty(max(n, 16), dtype=torch.uint8, device=self.y.device)
+        return self._layer_ws16
+
+    def run_steps_f16h(self, x: torch.Tensor, W: MoEWeights, residual: Optional[torch.Tensor] = None,
+                       out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """route -> permute -> grouped SwiGLU (f16 h) -> combine through the separate entry points."""
+        Z.zmoe_route(x, W.w_router, W.k, W.logit_bias, W.sel_bias, outs=(self.idx, self.gates, self.margin),
+                     stream=stream)
+        Z.zmoe_permute(self.idx, x, W.E, outs=self.perm_outs, workspace=self.perm_ws, stream=stream)
+        Z.zmoe_grouped_swiglu_f16h(self.perm_outs["x_perm"], self.perm_outs["offsets"], W.w_gate, W.w_up,
+                                   W.w_down_f16, W.down_scale, h=self.h16, y_perm=self.y_perm, stream=stream)
+        return Z.zmoe_combine(self.y_perm, self.perm_outs["inv_perm"], self.gates, residual,
+                              out=self.y if out is None else out, stream=stream)
 
     def run_steps(self, x: torch.Tensor, W: MoEWeights, residual: Optional[torch.Tensor] = None,
                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

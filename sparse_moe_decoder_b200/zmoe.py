@@ -55,6 +55,11 @@ SIGNATURES = {
     "zmoe_get_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "zmoe_debug_inject_timeout": (_I, [ctypes.c_uint32, ctypes.c_uint64]),
     "zmoe_decode_stack_workspace_size": (_S, [_I, _I, _I, _I]),
+    "zmoe_prepare_w_down_f16": (_I, [_P, _I, _I, _I, _P, _P, _P, _S, _P]),
+    "zmoe_grouped_swiglu_f16h": (_I, [_P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P]),
+    "zmoe_moe_layer_f16h_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "zmoe_moe_layer_f16h": (_I, [_P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                                 _P, _S, _P]),
     "zmoe_decode_stack": (_I, [_P, _I, _I, _I, _F, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P]),
 }
 
@@ -399,6 +404,64 @@ def zmoe_speaker_prefix(e: torch.Tensor, w_spk: torch.Tensor, b_spk: Optional[to
     y = out if out is not None else torch.empty((B, d), dtype=torch.float32, device=e.device)
     _check(lib().zmoe_speaker_prefix(_ptr(e), _ptr(w_spk), _dtype_code(w_spk.dtype), _ptr(b_spk), B, d, n_in, _ptr(y),
                                      _stream(stream)), "zmoe_speaker_prefix")
+    return y
+
+
+def zmoe_prepare_w_down_f16(w_down: torch.Tensor, out: Optional[torch.Tensor] = None,
+                            scale: Optional[torch.Tensor] = None, stream=None):
+    """The f16 copy of bf16 W_down [E, d, f] (each expert scaled by a power of two) and its per-expert
+    factors down_scale [E] f32 (w_down = w_down_f16 * down_scale, exact)."""
+    _need(w_down, "w_down", torch.bfloat16, 3)
+    E, d, f = w_down.shape
+    out = out if out is not None else torch.empty((E, d, f), dtype=torch.float16, device=w_down.device)
+    scale = scale if scale is not None else torch.empty((E,), dtype=torch.float32, device=w_down.device)
+    ws = torch.empty(max(4 * E, 16), dtype=torch.uint8, device=w_down.device)
+    _check(lib().zmoe_prepare_w_down_f16(_ptr(w_down), E, d, f, _ptr(out), _ptr(scale), _ptr(ws), ws.numel(),
+                                         _stream(stream)), "zmoe_prepare_w_down_f16")
+    return out, scale
+
+
+def zmoe_grouped_swiglu_f16h(x_perm: torch.Tensor, offsets: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
+                             w_down_f16: torch.Tensor, down_scale: torch.Tensor, h: Optional[torch.Tensor] = None,
+                             y_perm: Optional[torch.Tensor] = None, stream=None):
+    """Prefill grouped SwiGLU with h in f16 and the prepared down weights.  Returns (h f16 [M, f], y_perm f32)."""
+    _need(x_perm, "x_perm", torch.bfloat16, 2)
+    _need(w_down_f16, "w_down_f16", torch.float16, 3)
+    M, d = x_perm.shape
+    E, f = w_gate.shape[0], w_gate.shape[1]
+    h = h if h is not None else torch.empty((M, f), dtype=torch.float16, device=x_perm.device)
+    y_perm = y_perm if y_perm is not None else torch.empty((M, d), dtype=torch.float32, device=x_perm.device)
+    _check(lib().zmoe_grouped_swiglu_f16h(_ptr(x_perm), _ptr(offsets), M, _ptr(w_gate), _ptr(w_up), _ptr(w_down_f16),
+                                          _ptr(down_scale), E, d, f, _ptr(h), _ptr(y_perm), _stream(stream)),
+           "zmoe_grouped_swiglu_f16h")
+    return h, y_perm
+
+
+def zmoe_moe_layer_f16h(w_router: Optional[torch.Tensor], w_gate: torch.Tensor, w_up: torch.Tensor,
+                        w_down_f16: torch.Tensor, down_scale: torch.Tensor, k: int, x: Optional[torch.Tensor] = None,
+                        h: Optional[torch.Tensor] = None, gamma: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                        logit_bias: Optional[torch.Tensor] = None, sel_bias: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, outs: Optional[dict] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """zmoe_moe_layer with the prepared f16 down weights (prefill sizes); f32 [T, d]."""
+    src = h if gamma is not None else x
+    if src is None:
+        raise ValueError("zmoe_moe_layer_f16h: needs x, or h with gamma")
+    T, d = src.shape
+    E, f = w_gate.shape[0], w_gate.shape[1]
+    if x is not None:
+        _need(x, "x", torch.bfloat16, 2)
+    outs = outs or {}
+    y = out if out is not None else torch.empty((T, d), dtype=torch.float32, device=src.device)
+    ws_bytes = int(lib().zmoe_moe_layer_f16h_workspace_size(T, d, f, E, k))
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=src.device)
+    _check(lib().zmoe_moe_layer_f16h(_ptr(x), _ptr(h), _ptr(gamma), float(eps), _ptr(w_router), _ptr(logit_bias),
+                                     _ptr(sel_bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down_f16), _ptr(down_scale), T,
+                                     d, f, E, k, _ptr(y), _ptr(outs.get("expert_idx")), _ptr(outs.get("gates")),
+                                     _ptr(outs.get("margin")), _ptr(outs.get("x_norm")), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)),
+           "zmoe_moe_layer_f16h")
     return y
 
 
