@@ -13,15 +13,19 @@
 // launch per layer pays the launch, the staging of the router rows and the first weight bytes every
 // time; here one launch runs all layers and per layer only two grid barriers separate the phases:
 //   * every CTA repeats the pre-norm, the router logits and the selection (no barrier before the
-//     weights); the router rows and gain of layer l + 1 are bulk-copied into shared memory while layer
-//     l streams its weights, so routing starts from shared memory;
-//   * phase A: CTA c owns the f-rows [c f / C, (c + 1) f / C) of each chosen expert; one producer thread
-//     streams a gate row and an up row per slot of a 14-slot ring (bulk copies), 7 consumer warps
-//     (slot s always belongs to warp 1 + s % 7) contract them on the CUDA cores; h goes to global
-//     memory in fp32;
-//   * grid barrier 1 (consumers only: the producer keeps streaming W_down rows), a bulk copy of h;
-//   * phase B: CTA c owns the d-rows [c d / C, (c + 1) d / C), contracts them and adds the chosen
-//     experts, in slot order, to its rows of the residual stream h (in global memory, in place);
+//     weights); the router rows and gain of layer l + 1 are bulk-copied into shared memory at the end of
+//     layer l (while its grid barrier runs), so routing starts from shared memory;
+//   * phase A: CTA c owns the f-rows [c f / C, (c + 1) f / C) of each chosen expert.  These rows are
+//     contiguous in W_gate and W_up, so one producer thread streams them as blocks of up to 7 rows,
+//     one bulk copy per ring slot (~28 KB: one SM's streaming rate grows with the copy size, 4 KB copies
+//     reach well under half of it); gate and up blocks alternate, 7 consumer warps take every slot in
+//     order, warp w row w of the block (the gate value waits in shared memory for the up row); h goes
+//     to global memory in fp32;
+//   * grid barrier 1 (consumers only: the producer keeps streaming W_down blocks), a bulk copy of h
+//     into the router rows' area;
+//   * phase B: CTA c owns the d-rows [c d / C, (c + 1) d / C) (blocks of up to 5 rows of W_down, ~30 KB),
+//     contracts them and adds the chosen experts, in slot order, to its rows of the residual stream h
+//     (in global memory, in place);
 //   * grid barrier 2 (all of h updated) before the next layer's pre-norm.
 // Every sum is fp32 in a fixed order (no atomics on data): results do not depend on timing.  Every
 // wait is bounded; on expiry the CTA counts a timeout, stops, waits (bounded) for its own copies in
@@ -38,8 +42,8 @@ using namespace ptx;
 
 constexpr int kThreads = 256;            // warp 0: producer; warps 1..7: consumers
 constexpr int kConsumers = 7;
-constexpr int kSlots = 2 * kConsumers;   // slot s is consumed by warp 1 + s % kConsumers only
-static_assert(kSlots % kConsumers == 0, "a slot must belong to one consumer warp");
+constexpr int kSlots = 4;                // every consumer warp takes every slot, in order
+constexpr uint32_t kSlotTarget = 32768;  // bytes of weights per slot (at most)
 constexpr int kMaxK = 2;
 constexpr int kMaxE = 64;
 constexpr int kMaxLayers = 32;
@@ -75,8 +79,9 @@ struct StackArgs {
   float* layer_gates;        // [n_layers, 2] or null (0 past k)
   float* layer_h;            // [n_layers, d] or null: h entering each layer
   uint16_t* layer_x;         // [n_layers, d] or null: each layer's input as routed (bf16)
-  uint32_t slot_bytes;       // max(4 d, 2 f)
-  uint32_t wr_bytes;         // max over layers of E d 2, a multiple of 16
+  uint32_t slot_bytes;       // max(ra 2 d, rb 2 f), a multiple of 128
+  uint32_t r1_bytes;         // max(E d 2 over layers, kMaxK f 4), a multiple of 16
+  int ra, rb;                // rows per phase-A block (<= 7) and per phase-B block (<= 7)
 };
 
 struct __align__(16) StackCtrl {
@@ -84,6 +89,7 @@ struct __align__(16) StackCtrl {
   uint64_t empty[kSlots];
   uint64_t st;               // staging of a layer's router rows and gain: one phase per layer
   uint64_t hb;               // the layer's h, after grid barrier 1: one phase per layer
+  uint64_t r1free;           // phase B has read h: the area may take the next router rows (one per layer)
   int abort;
   int nu;                    // chosen experts (= k): slot i holds expert uexp[i] with gate gsel[i]
   int uexp[kMaxK];
@@ -91,24 +97,45 @@ struct __align__(16) StackCtrl {
   int ids[kMaxN];
   float red[kThreads / 32];
   float logit[kMaxE];
+  float gv[kConsumers];      // gate value of warp w's row of the current block
   float ypart[kMaxK][kMaxRowsB];
 };
 
-// Shared memory: ring | router rows | gamma | x (f32) | h of the chosen experts (f32) | control.
+// Shared memory: ring | R1 (router rows, then h of the chosen experts in phase B) | gamma | x (f32) |
+// control.
 struct StackSmem {
-  size_t ring, wr, gam, xs, hs, ctrl, total;
+  size_t ring, r1, gam, xs, ctrl, total;
 };
 
-__host__ __device__ inline StackSmem stack_smem(int d, int f, uint32_t slot_bytes, uint32_t wr_bytes) {
+__host__ __device__ inline StackSmem stack_smem(int d, uint32_t slot_bytes, uint32_t r1_bytes) {
   StackSmem S{};
   S.ring = 0;
-  S.wr = static_cast<size_t>(kSlots) * slot_bytes;
-  S.gam = S.wr + wr_bytes;
+  S.r1 = static_cast<size_t>(kSlots) * slot_bytes;
+  S.gam = S.r1 + r1_bytes;
   S.xs = S.gam + static_cast<size_t>(d) * 4;
-  S.hs = S.xs + static_cast<size_t>(d) * 4;
-  S.ctrl = S.hs + static_cast<size_t>(kMaxK) * f * 4;
+  S.ctrl = S.xs + static_cast<size_t>(d) * 4;
   S.total = S.ctrl + sizeof(StackCtrl);
   return S;
+}
+
+// Rows per block: as many as fit kSlotTarget bytes, 1..7.
+__host__ __device__ inline int rows_per_block(int row_bytes) {
+  const int r = static_cast<int>(kSlotTarget) / row_bytes;
+  return r < 1 ? 1 : (r > kConsumers ? kConsumers : r);
+}
+
+// A ring slot holds a phase-A block (ra rows of 2 d bytes) or a phase-B block (rb rows of 2 f bytes).
+inline uint32_t slot_bytes_for(int d, int f) {
+  const uint32_t a = static_cast<uint32_t>(rows_per_block(2 * d)) * 2u * d;
+  const uint32_t b = static_cast<uint32_t>(rows_per_block(2 * f)) * 2u * f;
+  return ((a > b ? a : b) + 127u) & ~127u;
+}
+
+// R1 holds a layer's router rows (E d bf16) during routing and h of the chosen experts (kMaxK f f32) in
+// phase B.
+inline uint32_t r1_bytes_for(int E_max, int d, int f) {
+  const uint32_t wr = static_cast<uint32_t>(E_max) * d * 2u, hb = static_cast<uint32_t>(kMaxK) * f * 4u;
+  return ((wr > hb ? wr : hb) + 15u) & ~15u;
 }
 
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort) {
@@ -184,13 +211,13 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int d = a.d, f = a.f;
-  const StackSmem S = stack_smem(d, f, a.slot_bytes, a.wr_bytes);
+  const StackSmem S = stack_smem(d, a.slot_bytes, a.r1_bytes);
   StackCtrl& C = *reinterpret_cast<StackCtrl*>(base + S.ctrl);
-  unsigned char* wr_s = base + S.wr;
+  unsigned char* wr_s = base + S.r1;                    // router rows (routing) ...
+  float* hs = reinterpret_cast<float*>(base + S.r1);    // ... then h of the chosen experts (phase B)
   unsigned char* gam_s = base + S.gam;
   const float* gam = reinterpret_cast<const float*>(gam_s);
   float* xs = reinterpret_cast<float*>(base + S.xs);
-  float* hs = reinterpret_cast<float*>(base + S.hs);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nC = gridDim.x, c = blockIdx.x;
   volatile int* abort_flag = &C.abort;
@@ -201,15 +228,18 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
   const int n0 = static_cast<int>(static_cast<long long>(d) * c / nC);
   const int n1 = static_cast<int>(static_cast<long long>(d) * (c + 1) / nC);
   const int nRA = f1 - f0, nRB = n1 - n0;
+  const int RA = a.ra, RB = a.rb;
+  const int GA = (nRA + RA - 1) / RA, GB = (nRB + RB - 1) / RB;   // blocks per chosen expert
   const int nvec = d / 8;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&C.full[s], 1);
-      mbar_init(&C.empty[s], 1);
+      mbar_init(&C.empty[s], kConsumers);   // one arrival per consumer warp
     }
     mbar_init(&C.st, 1);
     mbar_init(&C.hb, 1);
+    mbar_init(&C.r1free, 1);
     C.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     stage_layer(a, 0, C, wr_s, gam_s);
@@ -366,51 +396,70 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
     const int nu = C.nu;
-    const int nA = nu * nRA, nIt = nA + nu * nRB;
+    // items of this layer: phase A, per chosen expert u and block g, a gate block then an up block
+    // (i = 2 (u GA + g) + {0, 1}); phase B, per u and g, a W_down block (i = nA + u GB + g)
+    const int nA = 2 * nu * GA, nIt = nA + nu * GB;
 
     if (warp == 0) {
       // ================================ producer ================================
       if (lane == 0) {
-        if (l + 1 < L) {
-          stage_layer(a, l + 1, C, wr_s, gam_s);   // routing of this layer is done: the area is free
-          ++staged;
-        }
         int i = 0;
         for (; i < nIt; ++i) {
           const int qq = q + i, slot = qq % kSlots;
           if (!wait_bounded(&C.empty[slot], static_cast<uint32_t>((qq / kSlots) & 1) ^ 1u, abort_flag)) break;
           unsigned char* dst = base + static_cast<size_t>(slot) * a.slot_bytes;
+          const uint16_t* src;
+          uint32_t bytes;
           if (i < nA) {
-            const int u = i / nRA, r = f0 + i % nRA;
-            const size_t off = (static_cast<size_t>(C.uexp[u]) * f + r) * d;
-            mbar_expect_tx(&C.full[slot], static_cast<uint32_t>(4 * d));
-            bulk_load(dst, Ly.w_gate + off, static_cast<uint32_t>(2 * d), &C.full[slot]);
-            bulk_load(dst + 2 * d, Ly.w_up + off, static_cast<uint32_t>(2 * d), &C.full[slot]);
+            const int blk = i >> 1, u = blk / GA, r0 = f0 + (blk % GA) * RA;
+            const int nr = (f1 - r0) < RA ? (f1 - r0) : RA;
+            src = ((i & 1) ? Ly.w_up : Ly.w_gate) + (static_cast<size_t>(C.uexp[u]) * f + r0) * d;
+            bytes = static_cast<uint32_t>(nr) * d * 2u;
           } else {
-            const int j = i - nA;
-            const int u = j / nRB, n = n0 + j % nRB;
-            mbar_expect_tx(&C.full[slot], static_cast<uint32_t>(2 * f));
-            bulk_load(dst, Ly.w_down + (static_cast<size_t>(C.uexp[u]) * d + n) * f, static_cast<uint32_t>(2 * f),
-                      &C.full[slot]);
+            const int j = i - nA, u = j / GB, m0 = n0 + (j % GB) * RB;
+            const int nr = (n1 - m0) < RB ? (n1 - m0) : RB;
+            src = Ly.w_down + (static_cast<size_t>(C.uexp[u]) * d + m0) * f;
+            bytes = static_cast<uint32_t>(nr) * f * 2u;
           }
+          mbar_expect_tx(&C.full[slot], bytes);
+          bulk_load(dst, src, bytes, &C.full[slot]);
         }
         issued = q + i;
-        if (i < nIt) abort_cta(C, a.timeouts);
+        if (i < nIt) {
+          abort_cta(C, a.timeouts);
+        } else if (l + 1 < L) {
+          // the next layer's router rows go where phase B reads h: wait until it has
+          if (wait_bounded(&C.r1free, static_cast<uint32_t>(l & 1), abort_flag)) {
+            stage_layer(a, l + 1, C, wr_s, gam_s);
+            ++staged;
+          } else {
+            abort_cta(C, a.timeouts);
+          }
+        }
       }
       __syncwarp();
     } else {
       // ================================ consumers (warps 1..7) ================================
+      // every consumer warp takes every item in order; warp cw contracts row cw of the block
       const int cw = warp - 1;
-      // phase A: h of the owned f-rows of each chosen expert (item i is consumed by warp 1 + (q + i) % 7)
-      for (int i = ((cw - q) % kConsumers + kConsumers) % kConsumers; i < nA && ok; i += kConsumers) {
+      // phase A: h of the owned f-rows of each chosen expert
+      for (int i = 0; i < nA && ok; ++i) {
         const int qq = q + i, slot = qq % kSlots;
         ok = __all_sync(0xffffffffu, wait_bounded(&C.full[slot], static_cast<uint32_t>((qq / kSlots) & 1), abort_flag));
         if (!ok) break;
-        const int u = i / nRA, r = f0 + i % nRA;
-        const uint16_t* gr = reinterpret_cast<const uint16_t*>(base + static_cast<size_t>(slot) * a.slot_bytes);
-        const float gv = warp_dot(gr, xs, d, lane);
-        const float uv = warp_dot(gr + d, xs, d, lane);
-        if (lane == 0) a.hbuf[static_cast<size_t>(u) * f + r] = gv / (1.f + expf(-gv)) * uv;
+        const int blk = i >> 1, u = blk / GA, r0 = f0 + (blk % GA) * RA;
+        const int nr = (f1 - r0) < RA ? (f1 - r0) : RA;
+        if (cw < nr) {
+          const uint16_t* row = reinterpret_cast<const uint16_t*>(base + static_cast<size_t>(slot) * a.slot_bytes) +
+                                static_cast<size_t>(cw) * d;
+          const float v = warp_dot(row, xs, d, lane);
+          if ((i & 1) == 0) {
+            if (lane == 0) C.gv[cw] = v;                     // the gate value waits for the up block
+          } else if (lane == 0) {
+            const float gv = C.gv[cw];
+            a.hbuf[static_cast<size_t>(u) * f + r0 + cw] = gv / (1.f + expf(-gv)) * v;
+          }
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&C.empty[slot]);
       }
@@ -434,19 +483,25 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       ok = bar_and(1, kConsumers * 32, ok && !*abort_flag);
       if (ok) ok = __all_sync(0xffffffffu, wait_bounded(&C.hb, static_cast<uint32_t>(l & 1), abort_flag));
       // phase B: the owned d-rows of each chosen expert
-      for (int i = nA + ((cw - (q + nA)) % kConsumers + kConsumers) % kConsumers; i < nIt && ok; i += kConsumers) {
+      for (int i = nA; i < nIt && ok; ++i) {
         const int qq = q + i, slot = qq % kSlots;
         ok = __all_sync(0xffffffffu, wait_bounded(&C.full[slot], static_cast<uint32_t>((qq / kSlots) & 1), abort_flag));
         if (!ok) break;
-        const int j = i - nA;
-        const int u = j / nRB, n = j % nRB;
-        const uint16_t* dr = reinterpret_cast<const uint16_t*>(base + static_cast<size_t>(slot) * a.slot_bytes);
-        const float v = warp_dot(dr, hs + static_cast<size_t>(u) * f, f, lane);
-        if (lane == 0) C.ypart[u][n] = v;
+        const int j = i - nA, u = j / GB, m = (j % GB) * RB;        // m: first row, relative to n0
+        const int nr = (nRB - m) < RB ? (nRB - m) : RB;
+        if (cw < nr) {
+          const uint16_t* row = reinterpret_cast<const uint16_t*>(base + static_cast<size_t>(slot) * a.slot_bytes) +
+                                static_cast<size_t>(cw) * f;
+          const float v = warp_dot(row, hs + static_cast<size_t>(u) * f, f, lane);
+          if (lane == 0) C.ypart[u][m + cw] = v;
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&C.empty[slot]);
       }
+      // h (in the router rows' area) has been read: the producer may stage the next layer there
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       ok = bar_and(1, kConsumers * 32, ok);
+      if (threadIdx.x == 32 && ok) mbar_arrive(&C.r1free);
       // the owned rows of the residual stream: h + the chosen experts in slot order
       if (ok) {
         for (int n = threadIdx.x - 32; n < nRB; n += kConsumers * 32) {
@@ -508,10 +563,9 @@ size_t zmoe_decode_stack_workspace_size(int n_layers, int d, int f, int E_max) {
       f % 8 != 0 || E_max < 1 || E_max > kMaxE)
     return 0;
   const int nC = num_sms();
-  const uint32_t slot = static_cast<uint32_t>(4 * d > 2 * f ? 4 * d : 2 * f);
-  const uint32_t wr = (static_cast<uint32_t>(E_max) * d * 2u + 15u) & ~15u;
   if (nC < 1 || (d + nC - 1) / nC > kMaxRowsB ||
-      stack_smem(d, f, slot, wr).total + 1024 > static_cast<size_t>(max_smem_optin()))
+      stack_smem(d, slot_bytes_for(d, f), r1_bytes_for(E_max, d, f)).total + 1024 >
+          static_cast<size_t>(max_smem_optin()))
     return 0;
   return 256 + static_cast<size_t>(kMaxK) * f * 4;
 }
@@ -533,7 +587,7 @@ zmoe_status zmoe_decode_stack(const zmoe_stack_layer* layers, int n_layers, int 
   }
   ZMOE_REQUIRE(!layer_x || aligned16(layer_x), "zmoe_decode_stack: layer_x must be 16-byte aligned");
   StackArgs a{};
-  uint32_t wr_bytes = 16;
+  int E_max = 1;
   for (int l = 0; l < n_layers; ++l) {
     const zmoe_stack_layer& Ly = layers[l];
     ZMOE_REQUIRE(Ly.E >= 1 && Ly.E <= kMaxE, "zmoe_decode_stack: a layer's E must be in [1, 64]");
@@ -554,15 +608,12 @@ zmoe_status zmoe_decode_stack(const zmoe_stack_layer* layers, int n_layers, int 
     D.w_down = static_cast<const uint16_t*>(Ly.w_down);
     D.E = Ly.E;
     D.k = Ly.k;
-    if (Ly.w_router) {
-      const uint32_t b = static_cast<uint32_t>(Ly.E) * d * 2u;
-      if (b > wr_bytes) wr_bytes = b;
-    }
+    if (Ly.w_router && Ly.E > E_max) E_max = Ly.E;
   }
-  wr_bytes = (wr_bytes + 15u) & ~15u;
+  const uint32_t r1 = r1_bytes_for(E_max, d, f);
   const int nC = num_sms();
-  const uint32_t slot = static_cast<uint32_t>(4 * d > 2 * f ? 4 * d : 2 * f);
-  const StackSmem S = stack_smem(d, f, slot, wr_bytes);
+  const uint32_t slot = slot_bytes_for(d, f);
+  const StackSmem S = stack_smem(d, slot, r1);
   const size_t smem = S.total + 1024;
   if (nC < 1 || (d + nC - 1) / nC > kMaxRowsB || smem > static_cast<size_t>(max_smem_optin()))
     return fail(ZMOE_ERR_UNSUPPORTED, "zmoe_decode_stack: these sizes do not fit one SM's shared memory");
@@ -591,7 +642,9 @@ zmoe_status zmoe_decode_stack(const zmoe_stack_layer* layers, int n_layers, int 
   a.layer_h = layer_h;
   a.layer_x = static_cast<uint16_t*>(layer_x);
   a.slot_bytes = slot;
-  a.wr_bytes = wr_bytes;
+  a.r1_bytes = r1;
+  a.ra = rows_per_block(2 * d);
+  a.rb = rows_per_block(2 * f);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(workspace, 0, 256, s) != cudaSuccess)
     return check_launch("zmoe_decode_stack: clearing the barrier");

@@ -3,9 +3,10 @@
 zmoe_prepare_w_down_f16 is checked against its definition: w_down = w_down_f16 * down_scale exactly for
 every weight within 2^28 of its expert's largest (bit-exact as doubles), with a power-of-two scale per
 expert.  The grouped SwiGLU and the whole layer are checked against the fp64 oracle on every row and
-token: y_perm and y within the bf16 bar (2e-2 x RMS), h within 1e-3 x RMS (f16 keeps 11 significant bits:
-~2.4e-4 relative per element, plus the fp32 accumulation over K = d), routing ids bit-exact outside the
-margin exemption.  An h beyond f16's range is counted as a device error.
+token: y_perm and y within the bf16 bar (2e-2 x RMS), routing ids bit-exact outside the margin exemption.
+h is checked against f16's own rounding bound: |h_gpu - h| <= 2^-11 |h| (half an f16 ulp, relative to each
+element: h has tails ~30x its RMS) plus 1e-3 x RMS(h) for the fp32 accumulation of bf16 products over
+K = d (~1.5e-4 x RMS measured).  An h beyond f16's range is counted as a device error.
 """
 import numpy as np
 import pytest
@@ -20,6 +21,15 @@ from tests.gpu_util import MARGIN_EXEMPT, assert_close, host, rel_err, require_g
 pytestmark = pytest.mark.gpu
 
 H16_TOL = 1e-3
+
+
+def check_h16(h, h_ref):
+    """max(|h - h_ref| - 2^-11 |h_ref|) <= 1e-3 x RMS(h_ref); returns that excess / RMS."""
+    h_ref = np.asarray(h_ref, np.float64)
+    rms = float(np.sqrt(np.mean(h_ref * h_ref)))
+    excess = float(np.max(np.abs(np.asarray(h, np.float64) - h_ref) - 2.0 ** -11 * np.abs(h_ref))) / rms
+    assert excess <= H16_TOL, f"h (f16): error beyond half an f16 ulp = {excess:.3e} x RMS"
+    return excess
 
 
 def _offsets(counts):
@@ -74,7 +84,7 @@ def test_f16h_ragged_rows(counts):
     h, y = run_f16h(L, L.x, off)
     y_ref, h_ref = oracle.grouped_swiglu(L.x, off, L.w_gate, L.w_up, L.w_down)
     assert_close(y, y_ref, "bf16", "ragged y_perm (f16 h)")
-    assert rel_err(h, h_ref) <= H16_TOL
+    check_h16(h, h_ref)
 
 
 @pytest.mark.parametrize("E,d,f,counts", [
@@ -90,7 +100,7 @@ def test_f16h_tensor_core_shapes(E, d, f, counts):
     h, y = run_f16h(L, L.x, off)
     y_ref, h_ref = oracle.grouped_swiglu(L.x, off, L.w_gate, L.w_up, L.w_down)
     r = assert_close(y, y_ref, "bf16", "f16h y_perm")
-    assert rel_err(h, h_ref) <= H16_TOL
+    check_h16(h, h_ref)
     print(f"f16h E={E} d={d} f={f}: y_perm max err {r:.2e} x RMS")
 
 
@@ -111,9 +121,8 @@ def test_f16h_prefill_every_row(cfg):
     h, y = run_f16h(L, p["x_perm"], p["offsets"])
     y_ref, h_ref = oracle.grouped_swiglu(p["x_perm"], p["offsets"], L.w_gate, L.w_up, L.w_down)
     r = assert_close(y, y_ref, "bf16", f"config {cfg} y_perm (f16 h, every row)")
-    rh = rel_err(h, h_ref)
-    assert rh <= H16_TOL
-    print(f"config {cfg}: f16h y_perm max err {r:.2e} x RMS, h {rh:.2e} x RMS over {y.shape[0]} rows")
+    rh = check_h16(h, h_ref)
+    print(f"config {cfg}: f16h y_perm max err {r:.2e} x RMS, h excess over half an ulp {rh:.2e} x RMS over {y.shape[0]} rows")
 
 
 @pytest.mark.parametrize("cfg", [3, 4])
