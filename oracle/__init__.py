@@ -25,12 +25,14 @@ from .layer import combine, moe_layer, moe_layer_bruteforce, decode_stack_step
 from .params import param_counts
 from .heads import head_logits, greedy, output_heads
 from .speaker import speaker_prefix
-from .fp8 import e4m3_decode, dequantize_rows, moe_layer_fp8
+from .fp8 import (e4m3_decode, e4m3_encode, dequantize_rows, moe_layer_fp8, moe_layer_w8a8,
+                  quantize_rows_dynamic)
 
 __all__ = [
     "delay_shear", "delay_unshear", "embed_sum", "rmsnorm", "embed_sum_rmsnorm",
     "router_logits", "softmax", "select_topk", "route", "permute", "silu", "swiglu_ffn",
     "grouped_swiglu", "combine", "moe_layer", "moe_layer_bruteforce", "decode_stack_step",
     "param_counts", "head_logits", "greedy", "output_heads", "speaker_prefix",
-    "e4m3_decode", "dequantize_rows", "moe_layer_fp8",
+    "e4m3_decode", "e4m3_encode", "dequantize_rows", "moe_layer_fp8", "moe_layer_w8a8",
+    "quantize_rows_dynamic",
 ]

@@ -97,6 +97,8 @@ struct __align__(16) StackCtrl {
   int ids[kMaxN];
   float red[kThreads / 32];
   float logit[kMaxE];
+  float qb[kMaxE];           // the layer's logit bias (0 when none)
+  float sb[kMaxE];           // the layer's selection bias (0 when none)
   float gv[kConsumers];      // gate value of warp w's row of the current block
   float ypart[kMaxK][kMaxRowsB];
 };
@@ -305,6 +307,11 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       if (threadIdx.x == 0) abort_cta(C, a.timeouts);
       break;
     }
+    // the layer's biases, loaded alongside the residual stream (read after the norm's CTA barriers)
+    if (threadIdx.x < E) {
+      C.qb[threadIdx.x] = Ly.logit_bias ? Ly.logit_bias[threadIdx.x] : 0.f;
+      C.sb[threadIdx.x] = Ly.sel_bias ? Ly.sel_bias[threadIdx.x] : 0.f;
+    }
     // ---- pre-norm: x = bf16(RMSNorm(h) * gamma), kept as f32 in xs ----
     if (l > 0 || !a.ids) {
 #pragma unroll
@@ -348,44 +355,75 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       }
     }
     __syncthreads();
-    // ---- top-k (larger score first, ties to the lower index) and gates ----
-    if (threadIdx.x == 0) {
+    // ---- top-k (larger score first, ties to the lower index) and gates, by warp 0: lane l holds experts
+    // l and l + 32; maxima, arg-maxima and the softmax sum by butterflies ----
+    if (warp == 0) {
       if (!Ly.w_r) {
-        C.uexp[0] = 0;
-        C.gsel[0] = 1.f;
-        C.nu = 1;
+        if (lane == 0) {
+          C.uexp[0] = 0;
+          C.gsel[0] = 1.f;
+          C.nu = 1;
+        }
       } else {
-        const float NEG = -INFINITY;
-        float s1 = NEG, s2 = NEG, q1 = NEG, q2 = NEG, m = NEG;
-        int e1 = -1, e2 = -1;
-        for (int e = 0; e < E; ++e) {
-          const float qv = C.logit[e] + (Ly.logit_bias ? Ly.logit_bias[e] : 0.f);
-          const float sc = qv + (Ly.sel_bias ? Ly.sel_bias[e] : 0.f);
-          m = fmaxf(m, qv);
-          if (e1 < 0 || sc > s1) {
-            s2 = s1; e2 = e1; q2 = q1;
-            s1 = sc; e1 = e; q1 = qv;
-          } else if (e2 < 0 || sc > s2) {
-            s2 = sc; e2 = e; q2 = qv;
+        float qv[2], sv[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int e = lane + 32 * j;
+          qv[j] = e < E ? C.logit[e] + C.qb[e] : -INFINITY;
+          sv[j] = e < E ? qv[j] + C.sb[e] : -INFINITY;
+        }
+        float m = fmaxf(qv[0], qv[1]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float z = (lane < E ? expf(qv[0] - m) : 0.f) + (lane + 32 < E ? expf(qv[1] - m) : 0.f);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        int sel[kMaxK];
+        float qsel[kMaxK];
+#pragma unroll
+        for (int i = 0; i < kMaxK; ++i) {
+          if (i >= k) break;
+          // the lane's best candidate not chosen yet, then the warp's (larger score, else lower index)
+          float bs = -INFINITY;
+          int be = 0x7fffffff;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E && (i == 0 || e != sel[0]) && (sv[j] > bs || (sv[j] == bs && e < be))) {
+              bs = sv[j];
+              be = e;
+            }
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (os > bs || (os == bs && oe < be)) {
+              bs = os;
+              be = oe;
+            }
+          }
+          sel[i] = be;
+          qsel[i] = __shfl_sync(0xffffffffu, (be >> 5) ? qv[1] : qv[0], be & 31);
+        }
+        if (lane == 0) {
+          if (k == 1) {
+            C.uexp[0] = sel[0];
+            C.gsel[0] = expf(qsel[0] - m) / z;
+            C.nu = 1;
+          } else {
+            const float z1 = expf(qsel[0] - m), z2 = expf(qsel[1] - m);
+            const float iz = 1.f / (z1 + z2);
+            C.uexp[0] = sel[0];
+            C.gsel[0] = z1 * iz;
+            C.uexp[1] = sel[1];
+            C.gsel[1] = z2 * iz;
+            C.nu = 2;
           }
         }
-        float z = 0.f;
-        for (int e = 0; e < E; ++e) z += expf(C.logit[e] + (Ly.logit_bias ? Ly.logit_bias[e] : 0.f) - m);
-        if (k == 1) {
-          C.uexp[0] = e1;
-          C.gsel[0] = expf(q1 - m) / z;
-          C.nu = 1;
-        } else {
-          const float z1 = expf(q1 - m), z2 = expf(q2 - m);
-          const float iz = 1.f / (z1 + z2);
-          C.uexp[0] = e1;
-          C.gsel[0] = z1 * iz;
-          C.uexp[1] = e2;
-          C.gsel[1] = z2 * iz;
-          C.nu = 2;
-        }
       }
-      if (c == 0) {
+      __syncwarp();
+      if (c == 0 && lane == 0) {
         for (int i = 0; i < kMaxK; ++i) {
           if (a.layer_idx) a.layer_idx[l * kMaxK + i] = i < C.nu ? C.uexp[i] : -1;
           if (a.layer_gates) a.layer_gates[l * kMaxK + i] = i < C.nu ? C.gsel[i] : 0.f;

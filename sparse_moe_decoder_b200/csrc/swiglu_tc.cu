@@ -23,7 +23,9 @@
 //               CTA), waits for both CTAs' stage bytes and issues the MMAs from one lane; a commit
 //               multicast to both CTAs frees a stage and, per tile, hands the accumulator to both
 //               epilogues; odd CTA: allocates with the even CTA and forwards the completion of each
-//               of its stages to the even CTA's barrier;
+//               of its stages to the even CTA's barrier.  Barriers that the other CTA arrives on are
+//               polled without suspending the thread (a suspended waiter wakes ~0.5 us late on a
+//               remote arrival, which starved the MMAs);
 //   warps 2..5  epilogue: tcgen05.ld of this CTA's 128 accumulator rows (a 32-lane quarter per warp),
 //               SiLU * up -> h (gate/up) or the scaled fp32 result (down); masked stores of valid rows;
 //               then an arrival on the even CTA's accumulator-free barrier.
@@ -185,7 +187,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < nkb; ++kb, ++kbt) {
           const int s = kbt % STAGES;
           const uint32_t ph = static_cast<uint32_t>(kbt / STAGES) & 1u;
-          if (!mbar_wait(&C.empty[s], ph ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_cluster(&C.empty[s], ph ^ 1u, abort_flag, kTimeoutNs)) {
             set_abort(C, p.timeouts, peer);
             ok = false;
             break;

@@ -438,5 +438,52 @@ def pin_fp8(e4m3_decode, dequantize_rows, moe_layer_fp8):
     assert np.array_equal(dequantize_rows(qg, sg), e4m3_decode(qg) * sg[..., None])
 
 
+def pin_w8a8(e4m3_encode, quantize_rows_dynamic, moe_layer_w8a8):
+    """E4M3 encoding against torch's float8_e4m3fn conversion on the whole grid, every midpoint (ties to
+    the even code) and random values, with closed-form ties and saturation; the per-token dynamic scale in
+    closed form; a 1-expert W8A8 layer against the same steps written with torch (its float8 and float16
+    conversions, F.linear, F.silu)."""
+    import torch
+    import torch.nn.functional as F
+    from oracle import e4m3_decode
+    grid = e4m3_decode(np.arange(127, dtype=np.uint8))
+    mids = (grid[:-1] + grid[1:]) / 2
+    rng = np.random.default_rng(9)
+    v = np.concatenate([grid, -grid, mids, -mids, rng.standard_normal(20000) * 40, rng.random(5000) * 2.0 ** -6])
+    v32 = v.astype(np.float32)
+    ref = torch.from_numpy(v32).to(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(e4m3_decode(e4m3_encode(v32)), ref)
+    assert e4m3_encode(np.array([1.0625]))[0] == 0x38        # tie between 1 (even code) and 1.125
+    assert e4m3_encode(np.array([1.1875]))[0] == 0x3A        # tie between 1.125 and 1.25 (even code)
+    assert e4m3_encode(np.array([3.0 * 2.0 ** -10]))[0] == 0x02   # subnormal tie 1.5 x 2^-9 -> 2 x 2^-9
+    assert list(e4m3_encode(np.array([1000.0, -1000.0, 448.0, 0.0]))) == [0x7E, 0xFE, 0x7E, 0x00]
+    row = np.array([[448.0 * 2 ** -3, -2.0 ** -3, 0.5 * 2 ** -3, 0.0]], np.float32)
+    q, s = quantize_rows_dynamic(row)
+    assert s[0] == np.float32(2 ** -3) and list(q[0]) == [0x7E, 0xB8, 0x30, 0x00]
+    q0, s0 = quantize_rows_dynamic(np.zeros((1, 8), np.float32))
+    assert s0[0] == 1.0 and not q0.any()
+    # one expert, W8A8, against torch
+    d, f, T = 32, 96, 35     # 3360 hidden values: the f16 step moves ~0.4% of them across an E4M3 midpoint
+    qg, qu, qd = (rng.integers(0, 0x7E, size=sh).astype(np.uint8) | (rng.integers(0, 2, size=sh) << 7).astype(np.uint8)
+                  for sh in ((1, f, d), (1, f, d), (1, d, f)))
+    # row scales of weights whose largest magnitude is ~0.2-0.6 (a 448-code row), tokens of varied size
+    sg, su, sd = (((rng.random(sh) + 0.5) * 1e-3).astype(np.float32) for sh in ((1, f), (1, f), (1, d)))
+    x = (rng.standard_normal((T, d)) * np.tile([[1.0], [3.0], [0.1], [1e-3], [5.0], [1.0], [2.0]], (5, 1))).astype(np.float32)
+    out = moe_layer_w8a8(x, rng.standard_normal((1, d)), qg, sg, qu, su, qd, sd, 1)
+
+    def tq(a32):   # per-row dynamic quantization with torch's conversion, dequantized
+        a32 = torch.from_numpy(np.asarray(a32, np.float32))
+        s_ = a32.abs().amax(dim=1) / torch.tensor(448.0, dtype=torch.float32)
+        s_ = torch.where(s_ > 0, s_, torch.ones_like(s_))
+        return (a32 / s_[:, None]).to(torch.float8_e4m3fn).double() * s_.double()[:, None]
+
+    W = lambda q_, s_: torch.from_numpy(q_[0]).view(torch.float8_e4m3fn).double() * torch.from_numpy(s_[0]).double()[:, None]
+    xq = tq(x)
+    h = F.silu(F.linear(xq, W(qg, sg))) * F.linear(xq, W(qu, su))
+    hq = tq(h.to(torch.float16).float().numpy())
+    ref = F.linear(hq, W(qd, sd)).numpy()
+    assert np.allclose(out["y"], ref, rtol=1e-12, atol=1e-12)
+
+
 def golden_path(name):
     return os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", name)

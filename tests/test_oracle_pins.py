@@ -57,6 +57,10 @@ def test_pin_fp8():
     P.pin_fp8(oracle.e4m3_decode, oracle.dequantize_rows, oracle.moe_layer_fp8)
 
 
+def test_pin_w8a8():
+    P.pin_w8a8(oracle.e4m3_encode, oracle.quantize_rows_dynamic, oracle.moe_layer_w8a8)
+
+
 def test_pin_speaker():
     P.pin_speaker(oracle.speaker_prefix)
 
@@ -249,6 +253,69 @@ def _moe_fp8_scale_per_column(x, w_router, q_gate, s_gate, q_up, s_up, q_down, s
     return oracle.moe_layer(x, w_router, deq(q_gate, s_gate), deq(q_up, s_up), wd, k, **kw)
 
 
+def _e4m3_encode_ties_odd(v):
+    """Planted: ties go to the odd code."""
+    v = np.asarray(v, np.float64)
+    q = oracle.e4m3_encode(v).astype(np.int64)
+    grid = oracle.e4m3_decode(np.arange(127, dtype=np.uint8))
+    a = np.minimum(np.abs(v), 448.0)
+    mag = q & 0x7F
+    tie = np.zeros(a.shape, bool)
+    for c in (mag - 1, mag + 1):
+        ok = (c >= 0) & (c <= 126)
+        cc = np.clip(c, 0, 126)
+        tie |= ok & (np.abs(grid[cc] - a) == np.abs(grid[mag] - a)) & (grid[cc] != grid[mag])
+    alt = np.where(np.abs(grid[np.clip(mag + 1, 0, 126)] - a) == np.abs(grid[mag] - a), mag + 1, mag - 1)
+    mag = np.where(tie & (mag % 2 == 0), alt, mag)
+    return (mag | (q & 0x80)).astype(np.uint8)
+
+
+def _quantize_per_tensor(a):
+    """Planted: one scale for the whole matrix instead of one per token."""
+    a32 = np.asarray(a, np.float32)
+    amax = np.max(np.abs(a32))
+    s = np.float32(amax / np.float32(448.0)) if amax > 0 else np.float32(1.0)
+    q = oracle.e4m3_encode((a32 / s).astype(np.float32))
+    return q, np.full(a32.shape[:-1], s, np.float32)
+
+
+def _w8a8_layer_with(quantizer):
+    import oracle.fp8 as F8
+    saved = F8.quantize_rows_dynamic
+    def run(*args, **kw):
+        F8.quantize_rows_dynamic = quantizer
+        try:
+            return F8.moe_layer_w8a8(*args, **kw)
+        finally:
+            F8.quantize_rows_dynamic = saved
+    return run
+
+
+def _w8a8_no_f16_hidden(x, w_router, q_gate, s_gate, q_up, s_up, q_down, s_down, k, **kw):
+    """Planted: the hidden activation quantized straight from float64, without its f16 step."""
+    x = np.asarray(x, np.float64)
+    E = np.asarray(w_router).shape[0]
+    sel, gates, _, _ = oracle.route(x, w_router, k, kw.get("sel_bias"), kw.get("logit_bias"))
+    p = oracle.permute(sel, E, x)
+    qx, sx = oracle.quantize_rows_dynamic(p["x_perm"])
+    xq = oracle.e4m3_decode(qx) * sx[:, None].astype(np.float64)
+    off = p["offsets"]
+    h = np.zeros((xq.shape[0], np.asarray(q_gate).shape[1]))
+    y_perm = np.zeros_like(xq)
+    for e in range(E):
+        a, b = int(off[e]), int(off[e + 1])
+        if b > a:
+            h[a:b] = oracle.silu(xq[a:b] @ oracle.dequantize_rows(q_gate[e], s_gate[e]).T) * \
+                (xq[a:b] @ oracle.dequantize_rows(q_up[e], s_up[e]).T)
+    qh, sh = oracle.quantize_rows_dynamic(h)
+    hq = oracle.e4m3_decode(qh) * sh[:, None].astype(np.float64)
+    for e in range(E):
+        a, b = int(off[e]), int(off[e + 1])
+        if b > a:
+            y_perm[a:b] = hq[a:b] @ oracle.dequantize_rows(q_down[e], s_down[e]).T
+    return dict(y=oracle.combine(y_perm, p["inv_perm"], gates, kw.get("residual")))
+
+
 MUTANTS = {
     "shear reversed": lambda: P.pin_delay(_shear_reversed, oracle.delay_unshear, GOLDEN_DELAY),
     "shear too short": lambda: P.pin_delay(_shear_short, oracle.delay_unshear, GOLDEN_DELAY),
@@ -280,6 +347,12 @@ MUTANTS = {
     "fp8 down scales per column": lambda: P.pin_fp8(oracle.e4m3_decode, oracle.dequantize_rows,
                                                     _moe_fp8_scale_per_column),
     "speaker projection transposed": lambda: P.pin_speaker(_speaker_transposed),
+    "e4m3 ties to the odd code": lambda: P.pin_w8a8(_e4m3_encode_ties_odd, oracle.quantize_rows_dynamic,
+                                                    oracle.moe_layer_w8a8),
+    "w8a8 activations scaled per tensor": lambda: P.pin_w8a8(oracle.e4m3_encode, oracle.quantize_rows_dynamic,
+                                                             _w8a8_layer_with(_quantize_per_tensor)),
+    "w8a8 hidden activation without f16": lambda: P.pin_w8a8(oracle.e4m3_encode, oracle.quantize_rows_dynamic,
+                                                             _w8a8_no_f16_hidden),
     "dense layer drops residual": lambda: P.pin_stack_dense(_stack_dense_no_residual, oracle.embed_sum_rmsnorm,
                                                             oracle.rmsnorm, oracle.moe_layer_bruteforce),
 }
