@@ -349,6 +349,30 @@ ZMOE_API zmoe_status zmoe_moe_layer_f16h(const void* x, const float* h, const fl
                                          int32_t* expert_idx, float* gates, float* margin, void* x_norm,
                                          void* workspace, size_t ws_bytes, zmoe_stream_t stream);
 
+/* Bytes of workspace zmoe_moe_layer_w8a8 needs. */
+ZMOE_API size_t zmoe_moe_layer_w8a8_workspace_size(int T, int d, int f, int E, int k);
+
+/*
+ * The MoE layer in W8A8 fp8 for prefill-size batches ([COOKBOOK] Benchmark Results: the served ZONOS2
+ * runs fp8; the reading is the common fp8 serving scheme with dynamic per-token activation scales).
+ * Expert weights as in zmoe_moe_layer_fp8 (E4M3 codes, one fp32 scale per row: w = code * scale);
+ * router in bf16.  Each row entering an expert GEMM -- the permuted token row, then the hidden row h --
+ * is quantized per token: s = max|row| / 448 (fp32; 1 for an all-zero row), codes = the E4M3 value
+ * nearest row / s (ties to even, saturating at 448).  The GEMMs run on tcgen05 kind::f8f6f4 (CTA pairs);
+ * their fp32 sums are multiplied by the token scale and the weight row's scale; h is held in f16 between
+ * the GEMMs (an |h| beyond 65504 counts a device error) and quantized from that.
+ *   y[t] = h[t] + sum_i gate[t, i] * down_e( Q(silu(gate_e(Q(x[t]))) * up_e(Q(x[t]))) )   (h = 0 if NULL)
+ * Arguments as zmoe_moe_layer_fp8 (x or h with gamma: bf16 / f32); any T (built for >= 64 rows per expert
+ * on average); d % 256 == 0, f % 256 == 0.
+ */
+ZMOE_API zmoe_status zmoe_moe_layer_w8a8(const void* x, const float* h, const float* gamma, float eps,
+                                         const void* w_router, const float* logit_bias, const float* sel_bias,
+                                         const uint8_t* q_gate, const float* s_gate, const uint8_t* q_up,
+                                         const float* s_up, const uint8_t* q_down, const float* s_down, int T, int d,
+                                         int f, int E, int k, float* y, int32_t* expert_idx, float* gates,
+                                         float* margin, void* x_norm, void* workspace, size_t ws_bytes,
+                                         zmoe_stream_t stream);
+
 /* One layer of zmoe_decode_stack (bf16 weights, the layouts of zmoe_moe_layer). */
 typedef struct zmoe_stack_layer {
   const void* w_router;     /* bf16 [E, d]; NULL only for a dense FFN layer (E == 1, k == 1: gate 1) */

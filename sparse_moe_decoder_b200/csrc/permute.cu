@@ -192,6 +192,24 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ x, const int32_t* _
 int tiles_for(long long n) { return static_cast<int>((n + kTile - 1) / kTile); }
 
 }  // namespace
+
+// The index half of zmoe_permute (counts, offsets, perm, inv_perm; no row copy), for callers that move
+// the rows themselves (the fp8 path quantizes them on the way).  Workspace as zmoe_permute's.
+zmoe_status permute_indices(const int32_t* expert_idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                            int32_t* perm, int32_t* inv_perm, void* workspace, size_t ws_bytes, cudaStream_t s) {
+  const long long n = static_cast<long long>(T) * k;
+  if (n <= 0) return ZMOE_OK;
+  const int tiles = tiles_for(n);
+  if (!workspace || ws_bytes < static_cast<size_t>(tiles) * E * sizeof(int32_t))
+    return fail(ZMOE_ERR_WORKSPACE_TOO_SMALL, "permute (indices): workspace too small");
+  int32_t* tile_cnt = static_cast<int32_t*>(workspace);
+  unsigned int* err = device_error_counter();
+  permute_count_kernel<<<tiles, kTile, 0, s>>>(expert_idx, static_cast<int>(n), E, tile_cnt, err);
+  permute_scan_kernel<<<1, 128, 0, s>>>(tile_cnt, tiles, E, counts, offsets);
+  permute_scatter_kernel<<<tiles, kTile, 0, s>>>(expert_idx, static_cast<int>(n), k, E, tile_cnt, perm, inv_perm);
+  return check_launch("permute (indices)");
+}
+
 }  // namespace zmoe
 
 extern "C" {

@@ -254,6 +254,12 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// The same arrival without the release fence (relaxed): for a thread that only relays a completion it
+// has observed (a stage's bulk copies landed), where a cluster-scope release per arrival costs ~0.5 us.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // Has the phase of parity `parity` completed?  Acquire at cluster scope (for barriers that other CTAs
 // of the cluster arrive on).  Never suspends the thread: a thread suspended in try_wait is not woken
 // promptly by an arrival from another CTA (measured: ~0.5 us per wait), so these barriers are polled.
@@ -299,6 +305,16 @@ __device__ __forceinline__ void umma2_f16(uint32_t d_tmem, uint64_t adesc, uint6
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// The same pair MMA on 8-bit operands (kind::f8f6f4, K = 32 per instruction: 32 bytes, like kind::f16).
+__device__ __forceinline__ void umma2_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
 // Arrives once on the mbarrier at this shared-memory offset in every CTA of `cta_mask` when the
 // cta_group::2 tcgen05 operations issued so far by this thread have completed.
 __device__ __forceinline__ void umma2_commit_mc(uint64_t* bar, uint16_t cta_mask) {
@@ -324,6 +340,13 @@ __device__ __forceinline__ void tmem_alloc2(uint32_t* dst_smem, uint32_t ncols) 
 
 __device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+
+// Instruction descriptor of kind::f8f6f4 with E4M3 A and B (format code 0, K-major), fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                                   // D format: f32
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
 // Instruction descriptor of kind::f16 with f16 A and B (K-major), fp32 accumulator, M x N.

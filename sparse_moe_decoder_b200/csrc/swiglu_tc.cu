@@ -51,10 +51,10 @@ using namespace ptx;
 constexpr int BMC = 128;                        // rows of A per CTA (256 per pair)
 constexpr int BN = 256;                         // MMA N
 constexpr int BNC = 128;                        // rows of B per CTA
-constexpr int BK = 64;
+constexpr int KB_BYTES = 128;                   // bytes of K per row and stage (one 128-byte swizzle atom)
 constexpr int STAGES = 6;
-constexpr int A_BYTES = BMC * BK * 2;           // 16 KB
-constexpr int B_BYTES = BNC * BK * 2;           // 16 KB
+constexpr int A_BYTES = BMC * KB_BYTES;         // 16 KB
+constexpr int B_BYTES = BNC * KB_BYTES;         // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
 constexpr int kThreads = 192;
 constexpr uint32_t TMEM_COLS = 512;
@@ -62,11 +62,21 @@ constexpr unsigned long long kTimeoutNs = 2000000000ull;
 constexpr int kMaxE = 64;
 
 enum { kGateUp = 0, kDown = 1 };
+// Operand formats: bf16 with h as the bf16 pair; bf16 x / gate / up with h and W_down in f16; E4M3 with
+// per-row scales (W8A8).
+enum { kPair = 0, kF16 = 1, kE4M3 = 2 };
+
+// Elements of K per stage.
+__host__ __device__ constexpr int bk_of(int fmt) { return fmt == kE4M3 ? KB_BYTES : KB_BYTES / 2; }
 
 struct TcParams {
   const int32_t* offsets;
   void* out;                 // gate/up: h (f16 [M, f] or bf16 pair [M, 2f]); down: y_perm f32 [M, d]
   const float* down_scale;   // f16 down: [E], multiplies the finished sums; else null
+  const float* row_scale;    // E4M3: [M] per-token scale of A's rows (x or h)
+  const float* col_scale0;   // E4M3: row scales of the weights: gate [E f] (gate/up) or down [E d]
+  const float* col_scale1;   // E4M3 gate/up: up [E f]
+  unsigned int* amax;        // E4M3 gate/up: [M] bits of max |f16(h)| per row (atomic max)
   int E, K, out_ld;          // contraction length (A columns); row length of `out`
   int M_total;               // rows of x_perm / h / y_perm: offsets must be a monotone split of [0, M_total]
   int lo_offset;             // bf16 pair: column of h_lo in `out` (= f)
@@ -117,7 +127,7 @@ __device__ __forceinline__ uint16_t f32_to_f16_bits(float v) {
 // ------------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------------
-template <int MODE, bool F16H>
+template <int MODE, int FMT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_ffn_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
                   const __grid_constant__ CUtensorMap mapB1, TcParams p) {
@@ -169,6 +179,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = C.tmem_base;
   const int total = C.tile_start[p.E];
+  constexpr int BK = bk_of(FMT);
   const int nkb = p.K / BK;
 
   int issued = 0;   // k-blocks whose loads this CTA's producer issued (producer thread only)
@@ -205,7 +216,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (even) {
       if (lane == 0) {
         // ---------------- MMA issuer (even CTA) ----------------
-        constexpr uint32_t idesc = (MODE == kDown && F16H) ? idesc_f16_f32(2 * BMC, BN) : idesc_bf16_f32(2 * BMC, BN);
+        constexpr uint32_t idesc = FMT == kE4M3                      ? idesc_e4m3_f32(2 * BMC, BN)
+                                   : (MODE == kDown && FMT == kF16) ? idesc_f16_f32(2 * BMC, BN)
+                                                                    : idesc_bf16_f32(2 * BMC, BN);
         int kbt = 0, it = 0;
         bool ok = true;
         for (int t = pair; t < total && ok && !*abort_flag; t += npairs, ++it) {
@@ -228,9 +241,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t sa = smem_u32(stages + s * STAGE_BYTES);
             const uint32_t sb = sa + A_BYTES;
+            // four MMAs of 32 bytes of K each (K = 16 bf16 / f16 elements, or 32 E4M3 elements)
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              umma2_f16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < KB_BYTES / 32; ++kk) {
+              if (FMT == kE4M3)
+                umma2_f8(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+              else
+                umma2_f16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
             umma2_commit_mc(&C.empty[s], 0x3);
           }
           if (!ok) break;
@@ -254,7 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_cluster(mapa_shared(smem_u32(&C.pfull[s]), 0));
+          mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&C.pfull[s]), 0));
         }
       }
       if (!ok) set_abort(C, p.timeouts, peer);
@@ -281,6 +299,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (MODE == kGateUp) {
         uint16_t* h = static_cast<uint16_t*>(p.out) + static_cast<size_t>(row) * p.out_ld + nt * BNC;
         bool range_ok = true;
+        float hmax = 0.f;
+        const float rs = (FMT == kE4M3 && valid) ? p.row_scale[row] : 1.f;
+        const size_t col0 = static_cast<size_t>(e) * p.b_rows_per_expert + nt * BNC;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t g[32], u[32];
@@ -288,15 +309,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_ld32(taddr + 128 + c * 32, u);
           tmem_wait_ld();
           if (valid) {
-            if (F16H) {
+            if (FMT != kPair) {
               uint32_t hv[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-                const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                if (FMT == kE4M3) {
+                  const size_t j = col0 + c * 32 + 2 * i;
+                  g0 *= rs * __ldg(p.col_scale0 + j);
+                  g1 *= rs * __ldg(p.col_scale0 + j + 1);
+                  u0 *= rs * __ldg(p.col_scale1 + j);
+                  u1 *= rs * __ldg(p.col_scale1 + j + 1);
+                }
                 const float h0 = g0 / (1.f + expf(-g0)) * u0, h1 = g1 / (1.f + expf(-g1)) * u1;
                 range_ok = range_ok && fabsf(h0) < 65504.f && fabsf(h1) < 65504.f;
-                hv[i] = static_cast<uint32_t>(f32_to_f16_bits(h0)) | (static_cast<uint32_t>(f32_to_f16_bits(h1)) << 16);
+                const uint16_t b0 = f32_to_f16_bits(h0), b1 = f32_to_f16_bits(h1);
+                if (FMT == kE4M3)
+                  hmax = fmaxf(hmax, fmaxf(fabsf(__half2float(__ushort_as_half(b0))),
+                                           fabsf(__half2float(__ushort_as_half(b1)))));
+                hv[i] = static_cast<uint32_t>(b0) | (static_cast<uint32_t>(b1) << 16);
               }
               uint4* dst = reinterpret_cast<uint4*>(h + c * 32);
 #pragma unroll
@@ -322,21 +354,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         // an h beyond f16's range (65504) is a data error: counted, the stored value is +-inf
-        if (F16H && !range_ok) record_device_error(p.errors);
+        if (FMT != kPair && !range_ok) record_device_error(p.errors);
+        // the row's largest |h| so far, for its per-token E4M3 scale (non-negative floats order as integers)
+        if (FMT == kE4M3 && valid) atomicMax(p.amax + row, __float_as_uint(hmax));
       } else {
         float* y = static_cast<float*>(p.out) + static_cast<size_t>(row) * p.out_ld + nt * BN;
-        const float sc = F16H ? p.down_scale[e] : 1.f;
+        const float sc = FMT == kF16 ? p.down_scale[e] : ((FMT == kE4M3 && valid) ? p.row_scale[row] : 1.f);
+        const float* cs = FMT == kE4M3 ? p.col_scale0 + static_cast<size_t>(e) * p.b_rows_per_expert + nt * BN : nullptr;
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           uint32_t v[32];
           tmem_ld32(taddr + c * 32, v);
           tmem_wait_ld();
           if (valid) {
+            float o[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              o[j] = __uint_as_float(v[j]) * sc * (FMT == kE4M3 ? __ldg(cs + c * 32 + j) : 1.f);
             float4* dst = reinterpret_cast<float4*>(y + c * 32);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(__uint_as_float(v[4 * j]) * sc, __uint_as_float(v[4 * j + 1]) * sc,
-                                   __uint_as_float(v[4 * j + 2]) * sc, __uint_as_float(v[4 * j + 3]) * sc);
+            for (int j = 0; j < 8; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
           }
         }
       }
@@ -384,8 +421,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_outer) {
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {inner * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_outer};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(KB_BYTES / 2), box_outer};
   return encode_bf16_map(m, ptr, 2, dims, strides, box);
+}
+
+// The same for 1-byte elements (E4M3 codes): box of box_outer rows x 128 elements.
+bool make_map8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(KB_BYTES), box_outer};
+  return encode_map(m, ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // CTA pairs that can be resident at once (clusters of 2 are placed within one GPC), cached per kernel
@@ -413,16 +458,34 @@ int resident_pairs(K kern) {
   return n;
 }
 
-template <int MODE, bool F16H>
+template <int MODE, int FMT>
 zmoe_status launch_tc(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const TcParams& p,
                       cudaStream_t s) {
-  auto kern = tc_ffn_kernel<MODE, F16H>;
+  auto kern = tc_ffn_kernel<MODE, FMT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes)) !=
       cudaSuccess)
     return check_launch("grouped_swiglu (tcgen05): shared memory attribute");
   const int pairs = resident_pairs(kern);
   kern<<<2 * pairs, kThreads, kSmemBytes, s>>>(a, b0, b1, p);
   return check_launch("grouped_swiglu (tcgen05)");
+}
+
+TcParams params(const int32_t* offsets, void* out, int E, int K, int out_ld, int M_total, int lo_offset, int kb_wrap,
+                int b_rows, int n_tiles) {
+  TcParams p{};
+  p.offsets = offsets;
+  p.out = out;
+  p.E = E;
+  p.K = K;
+  p.out_ld = out_ld;
+  p.M_total = M_total;
+  p.lo_offset = lo_offset;
+  p.kb_wrap = kb_wrap;
+  p.b_rows_per_expert = b_rows;
+  p.n_tiles = n_tiles;
+  p.timeouts = device_timeout_counter();
+  p.errors = device_error_counter();
+  return p;
 }
 
 }  // namespace
@@ -445,13 +508,10 @@ zmoe_status grouped_swiglu_tc(const uint16_t* x_perm, const int32_t* offsets, in
       !make_map(&mu, w_up, d, static_cast<uint64_t>(E) * f, BNC) || !make_map(&mh, h, 2 * f, M_total, BMC) ||
       !make_map(&md, w_down, f, static_cast<uint64_t>(E) * d, BNC))
     return fail(ZMOE_ERR_CUDA, "grouped_swiglu (tcgen05): cuTensorMapEncodeTiled failed");
-  unsigned int* tmo = device_timeout_counter();
-  unsigned int* err = device_error_counter();
-  TcParams gu{offsets, h, nullptr, E, d, 2 * f, M_total, f, d / BK, f, f / BNC, tmo, err};
-  zmoe_status st = launch_tc<kGateUp, false>(mx, mg, mu, gu, s);
+  constexpr int BK = bk_of(kPair);
+  zmoe_status st = launch_tc<kGateUp, kPair>(mx, mg, mu, params(offsets, h, E, d, 2 * f, M_total, f, d / BK, f, f / BNC), s);
   if (st != ZMOE_OK) return st;
-  TcParams dn{offsets, y_perm, nullptr, E, 2 * f, d, M_total, 0, f / BK, d, d / BN, tmo, err};
-  return launch_tc<kDown, false>(mh, md, md, dn, s);
+  return launch_tc<kDown, kPair>(mh, md, md, params(offsets, y_perm, E, 2 * f, d, M_total, 0, f / BK, d, d / BN), s);
 }
 
 // f16 down weights (prepared, with per-expert scales): h in f16.
@@ -465,13 +525,48 @@ zmoe_status grouped_swiglu_tc_f16h(const uint16_t* x_perm, const int32_t* offset
       !make_map(&mu, w_up, d, static_cast<uint64_t>(E) * f, BNC) || !make_map(&mh, h, f, M_total, BMC) ||
       !make_map(&md, w_down_f16, f, static_cast<uint64_t>(E) * d, BNC))
     return fail(ZMOE_ERR_CUDA, "grouped_swiglu (tcgen05): cuTensorMapEncodeTiled failed");
-  unsigned int* tmo = device_timeout_counter();
-  unsigned int* err = device_error_counter();
-  TcParams gu{offsets, h, nullptr, E, d, f, M_total, 0, d / BK, f, f / BNC, tmo, err};
-  zmoe_status st = launch_tc<kGateUp, true>(mx, mg, mu, gu, s);
+  constexpr int BK = bk_of(kF16);
+  zmoe_status st = launch_tc<kGateUp, kF16>(mx, mg, mu, params(offsets, h, E, d, f, M_total, 0, d / BK, f, f / BNC), s);
   if (st != ZMOE_OK) return st;
-  TcParams dn{offsets, y_perm, down_scale, E, f, d, M_total, 0, f / BK, d, d / BN, tmo, err};
-  return launch_tc<kDown, true>(mh, md, md, dn, s);
+  TcParams dn = params(offsets, y_perm, E, f, d, M_total, 0, f / BK, d, d / BN);
+  dn.down_scale = down_scale;
+  return launch_tc<kDown, kF16>(mh, md, md, dn, s);
+}
+
+// W8A8: the gate/up GEMM on E4M3 x rows (per-token scales sx) and E4M3 weights (row scales); writes h in
+// f16 and each row's max |h| (amax, zeroed by the caller).
+zmoe_status grouped_gateup_tc_e4m3(const uint8_t* xq, const float* sx, const int32_t* offsets, int M_total,
+                                   const uint8_t* q_gate, const float* s_gate, const uint8_t* q_up, const float* s_up,
+                                   int E, int d, int f, uint16_t* h16, unsigned int* amax, cudaStream_t s) {
+  if (!grouped_swiglu_tc_supported(d, f) || E > kMaxE)
+    return fail(ZMOE_ERR_UNSUPPORTED, "grouped_swiglu (fp8): needs d % 256 == 0, f % 128 == 0, E <= 64");
+  CUtensorMap mx, mg, mu;
+  if (!make_map8(&mx, xq, d, M_total, BMC) || !make_map8(&mg, q_gate, d, static_cast<uint64_t>(E) * f, BNC) ||
+      !make_map8(&mu, q_up, d, static_cast<uint64_t>(E) * f, BNC))
+    return fail(ZMOE_ERR_CUDA, "grouped_swiglu (fp8): cuTensorMapEncodeTiled failed");
+  constexpr int BK = bk_of(kE4M3);
+  TcParams gu = params(offsets, h16, E, d, f, M_total, 0, d / BK, f, f / BNC);
+  gu.row_scale = sx;
+  gu.col_scale0 = s_gate;
+  gu.col_scale1 = s_up;
+  gu.amax = amax;
+  return launch_tc<kGateUp, kE4M3>(mx, mg, mu, gu, s);
+}
+
+// W8A8: the down GEMM on E4M3 h rows (per-token scales sh) and E4M3 W_down (row scales) -> y_perm f32.
+zmoe_status grouped_down_tc_e4m3(const uint8_t* hq, const float* sh, const int32_t* offsets, int M_total,
+                                 const uint8_t* q_down, const float* s_down, int E, int d, int f, float* y_perm,
+                                 cudaStream_t s) {
+  if (!grouped_swiglu_tc_supported(d, f) || E > kMaxE)
+    return fail(ZMOE_ERR_UNSUPPORTED, "grouped_swiglu (fp8): needs d % 256 == 0, f % 128 == 0, E <= 64");
+  CUtensorMap mh, md;
+  if (!make_map8(&mh, hq, f, M_total, BMC) || !make_map8(&md, q_down, f, static_cast<uint64_t>(E) * d, BNC))
+    return fail(ZMOE_ERR_CUDA, "grouped_swiglu (fp8): cuTensorMapEncodeTiled failed");
+  constexpr int BK = bk_of(kE4M3);
+  TcParams dn = params(offsets, y_perm, E, f, d, M_total, 0, f / BK, d, d / BN);
+  dn.row_scale = sh;
+  dn.col_scale0 = s_down;
+  return launch_tc<kDown, kE4M3>(mh, md, md, dn, s);
 }
 
 }  // namespace zmoe

@@ -58,6 +58,9 @@ SIGNATURES = {
     "zmoe_prepare_w_down_f16": (_I, [_P, _I, _I, _I, _P, _P, _P, _S, _P]),
     "zmoe_grouped_swiglu_f16h": (_I, [_P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "zmoe_moe_layer_f16h_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "zmoe_moe_layer_w8a8_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "zmoe_moe_layer_w8a8": (_I, [_P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P,
+                                 _P, _P, _P, _S, _P]),
     "zmoe_moe_layer_f16h": (_I, [_P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                                  _P, _S, _P]),
     "zmoe_decode_stack": (_I, [_P, _I, _I, _I, _F, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P]),
@@ -462,6 +465,36 @@ def zmoe_moe_layer_f16h(w_router: Optional[torch.Tensor], w_gate: torch.Tensor, 
                                      _ptr(outs.get("margin")), _ptr(outs.get("x_norm")), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream)),
            "zmoe_moe_layer_f16h")
+    return y
+
+
+def zmoe_moe_layer_w8a8(w_router: Optional[torch.Tensor], q_gate: torch.Tensor, s_gate: torch.Tensor,
+                        q_up: torch.Tensor, s_up: torch.Tensor, q_down: torch.Tensor, s_down: torch.Tensor, k: int,
+                        x: Optional[torch.Tensor] = None, h: Optional[torch.Tensor] = None,
+                        gamma: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                        logit_bias: Optional[torch.Tensor] = None, sel_bias: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, outs: Optional[dict] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The W8A8 fp8 layer (prefill sizes); f32 [T, d].  Weights: uint8 E4M3 codes [E, f, d] / [E, d, f]
+    with f32 row scales [E, f] / [E, d]."""
+    src = h if gamma is not None else x
+    if src is None:
+        raise ValueError("zmoe_moe_layer_w8a8: needs x, or h with gamma")
+    T, d = src.shape
+    E, f = q_gate.shape[0], q_gate.shape[1]
+    for t, n in ((q_gate, "q_gate"), (q_up, "q_up"), (q_down, "q_down")):
+        _need(t, n, torch.uint8, 3)
+    outs = outs or {}
+    y = out if out is not None else torch.empty((T, d), dtype=torch.float32, device=src.device)
+    ws_bytes = int(lib().zmoe_moe_layer_w8a8_workspace_size(T, d, f, E, k))
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=src.device)
+    _check(lib().zmoe_moe_layer_w8a8(_ptr(x), _ptr(h), _ptr(gamma), float(eps), _ptr(w_router), _ptr(logit_bias),
+                                     _ptr(sel_bias), _ptr(q_gate), _ptr(s_gate), _ptr(q_up), _ptr(s_up), _ptr(q_down),
+                                     _ptr(s_down), T, d, f, E, k, _ptr(y), _ptr(outs.get("expert_idx")),
+                                     _ptr(outs.get("gates")), _ptr(outs.get("margin")), _ptr(outs.get("x_norm")),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+           "zmoe_moe_layer_w8a8")
     return y
 
 
