@@ -47,7 +47,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--config", type=int, default=None, choices=[2, 3, 4, 5, 6, 7],
+    ap.add_argument("--config", type=int, default=None, choices=[2, 3, 4, 5, 6, 7, 8],
                     help="one workload alone; default: the headline workload (4) with workloads 2, 3 and 5 "
                          "measured in the same run and reported under 'also'")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -74,6 +74,9 @@ def load_peaks():
 
 
 WORKLOADS = {
+    8: "final MoE layer in W8A8 fp8: T=16384, d_model=2048, d_ff=3072, E=16, top-2, Zipf(1.2) logit skew; expert "
+       "weights E4M3 with one fp32 scale per row, token and hidden rows E4M3 with a dynamic per-token scale, "
+       "bf16 router, fp32 accumulate",
     7: "decode step with fp8 expert weights: one MoE layer, T=64, d_model=2048, d_ff=3072, E=16, top-1; expert "
        "weights E4M3 with one fp32 scale per row, bf16 router, f16 tensor-core operands, fp32 accumulate",
     2: "decode step: one MoE layer, T=64 tokens (64 streams x 1 position), d_model=2048, d_ff=3072, E=16, top-1, "
@@ -764,7 +767,96 @@ def summary_of(line):
     return out
 
 
+def run_w8a8(args):
+    """Workload 8: configuration 4's tokens and weights with the expert weights as E4M3 codes + row scales,
+    one zmoe_moe_layer_w8a8 call per step (router, permutation + token quantization, both E4M3 GEMMs on
+    CTA pairs, hidden quantization, combine)."""
+    import torch
+    world, rank, local_rank = args.world, args.rank, args.local_rank
+    from moe_inputs import make_config, quantize_e4m3_rows
+    from sparse_moe_decoder_b200 import zmoe_get_device_errors, zmoe_moe_layer_w8a8
+    L = make_config(4)
+    if rank > 0:
+        from moe_inputs import round_to_bf16
+        L.x = round_to_bf16(np.random.default_rng(rank_token_seed(rank)).standard_normal(L.x.shape, dtype=np.float32))
+    Q = [quantize_e4m3_rows(w) for w in (L.w_gate, L.w_up, L.w_down)]
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    qs = [dev(q) for q, _ in Q]
+    sc = [dev(s_) for _, s_ in Q]
+    w_r = torch.from_numpy(L.w_router).cuda().to(torch.bfloat16)
+    lb = dev(L.logit_bias) if L.logit_bias is not None else None
+    sb = dev(L.sel_bias) if L.sel_bias is not None else None
+    x = torch.from_numpy(L.x).cuda().to(torch.bfloat16)
+    T = L.T
+    idx = torch.empty((T, L.k), dtype=torch.int32, device="cuda")
+    y = torch.empty((T, L.d), dtype=torch.float32, device="cuda")
+    ws = torch.empty(int(__import__("sparse_moe_decoder_b200").zmoe.lib().zmoe_moe_layer_w8a8_workspace_size(
+        T, L.d, L.f, L.E, L.k)), dtype=torch.uint8, device="cuda")
+
+    def step(xin=None):
+        return zmoe_moe_layer_w8a8(w_r, qs[0], sc[0], qs[1], sc[1], qs[2], sc[2], L.k, x=x if xin is None else xin,
+                                   logit_bias=lb, sel_bias=sb, out=y, outs=dict(expert_idx=idx), workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    elapsed, = max_over_ranks([e0.elapsed_time(e1)], "cuda")
+    value = job_rate(T, world, args.steps, elapsed)
+    xh = torch.from_numpy(L.x).to(torch.bfloat16).pin_memory()
+    yh = torch.empty((T, L.d), dtype=torch.float32).pin_memory()
+    xd = torch.empty_like(x)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.steps):
+        xd.copy_(xh, non_blocking=True)
+        step(xd)
+        yh.copy_(y, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms, = max_over_ranks([a0.elapsed_time(a1)], "cuda")
+    errs = zmoe_get_device_errors()
+    peaks = load_peaks()
+    M = T * L.k
+    flops = 2.0 * M * 3 * L.d * L.f
+    ms = elapsed / args.steps
+    achieved = flops / (ms / 1e3) / 1e12
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    if rank != 0:
+        return None
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8 (e4m3 weights and activations)", "data": "synthetic",
+        "config": {"workload": WORKLOADS[8], "T": T, "d_model": L.d, "d_ff": L.f, "E": L.E, "k": L.k,
+                   "parallelism": f"dp{world} (replicated weights, no data-path collective)",
+                   "l2": "inputs larger than L2 (302 MB of E4M3 weights, 0.5 GB of per-step activations)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": achieved / fp8_peak, "traffic": None,
+                     "kernel": "whole zmoe_moe_layer_w8a8 call (route, permutation + token quantization, two E4M3 "
+                               "GEMMs on CTA pairs, hidden quantization, combine) against the GEMMs' FLOPs",
+                     "algorithmic_flops_per_launch": flops,
+                     "peak_source": peaks["source"] + " bf16 burst x 2 (the recipe's nominal fp8 / bf16 ratio)"},
+        "cpu_baseline": None,
+        "e2e": {"value": job_rate(T, world, args.steps, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * L.d * 2, "d2h_bytes_per_step": T * L.d * 4, "call": "zmoe_moe_layer_w8a8"},
+        "gpu_launches": 11 * args.steps, "clocks": clk.summary(), "device_errors": errs,
+    }
+
+
 def run_one(args):
+    if args.config == 8:
+        return run_w8a8(args)
     if args.config == 7:
         return run_fp8(args)
     if args.config >= 5:
@@ -773,7 +865,7 @@ def run_one(args):
 
 
 HEADLINE = 4
-ALSO = ((2, 200, 20), (3, None, None), (5, 100, 10))    # (workload, min steps, min warm-up)
+ALSO = ((2, 200, 20), (3, None, None), (5, 100, 10), (8, None, None))   # (workload, min steps, min warm-up)
 
 
 def main(argv=None):
