@@ -353,6 +353,14 @@ ZMOE_API zmoe_status zmoe_moe_layer_f16h(const void* x, const float* h, const fl
 ZMOE_API size_t zmoe_moe_layer_w8a8_workspace_size(int T, int d, int f, int E, int k);
 
 /*
+ * Where zmoe_moe_layer_w8a8 leaves its intermediates in the workspace (byte offsets, for inspection
+ * after the call): offsets[0..9] = counts int32 [E], offsets int32 [E + 1], perm int32 [T k], inv_perm
+ * int32 [T, k], the token rows' codes uint8 [T k, d] and scales f32 [T k], h f16 [T k, f], h's codes
+ * uint8 [T k, f] and scales f32 [T k], y_perm f32 [T k, d] (rows in expert order).  n >= 10.
+ */
+ZMOE_API zmoe_status zmoe_moe_layer_w8a8_workspace_layout(int T, int d, int f, int E, int k, size_t* offsets, int n);
+
+/*
  * The MoE layer in W8A8 fp8 for prefill-size batches ([COOKBOOK] Benchmark Results: the served ZONOS2
  * runs fp8; the reading is the common fp8 serving scheme with dynamic per-token activation scales).
  * Expert weights as in zmoe_moe_layer_fp8 (E4M3 codes, one fp32 scale per row: w = code * scale);

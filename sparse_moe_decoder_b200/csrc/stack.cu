@@ -171,6 +171,26 @@ __device__ __forceinline__ float warp_dot(const uint16_t* row, const float* v, i
   return acc;
 }
 
+// The same dot product with the vector held in registers: xr[j] = v[lane 8 + 256 j .. + 8) for the
+// j < kXChunks chunks that lie below n (n <= 256 kXChunks).  Same summation order as warp_dot.
+constexpr int kXChunks = 8;   // d <= 2048 keeps x in registers
+__device__ __forceinline__ float warp_dot_xr(const uint16_t* row, const float (&xr)[kXChunks][8], int n, int lane) {
+  float acc = 0.f;
+#pragma unroll
+  for (int j = 0; j < kXChunks; ++j) {
+    const int c = lane * 8 + j * 256;
+    if (c < n) {
+      float w[8];
+      unpack_bf16x8(*reinterpret_cast<const uint4*>(row + c), w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc = fmaf(w[i], xr[j][i], acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
+}
+
 // Sum over the CTA (all threads take part); every thread receives the total.
 __device__ __forceinline__ float cta_sum(float v, float* red) {
   v = warp_sum(v);
@@ -346,11 +366,21 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       }
     }
     __syncthreads();
+    // x in registers for the dot products of this layer (when d fits kXChunks chunks)
+    const bool x_in_regs = d <= 256 * kXChunks;
+    float xr[kXChunks][8];
+#pragma unroll
+    for (int j = 0; j < kXChunks; ++j) {
+      const int cidx = lane * 8 + j * 256;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) xr[j][i] = (x_in_regs && cidx < d) ? xs[cidx + i] : 0.f;
+    }
     // ---- router logits, one warp per expert ----
     if (Ly.w_r) {
       const uint16_t* wr = reinterpret_cast<const uint16_t*>(wr_s);
       for (int e = warp; e < E; e += kThreads / 32) {
-        const float v = warp_dot(wr + static_cast<size_t>(e) * d, xs, d, lane);
+        const uint16_t* row = wr + static_cast<size_t>(e) * d;
+        const float v = x_in_regs ? warp_dot_xr(row, xr, d, lane) : warp_dot(row, xs, d, lane);
         if (lane == 0) C.logit[e] = v;
       }
     }
@@ -490,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
         if (cw < nr) {
           const uint16_t* row = reinterpret_cast<const uint16_t*>(base + static_cast<size_t>(slot) * a.slot_bytes) +
                                 static_cast<size_t>(cw) * d;
-          const float v = warp_dot(row, xs, d, lane);
+          const float v = x_in_regs ? warp_dot_xr(row, xr, d, lane) : warp_dot(row, xs, d, lane);
           if ((i & 1) == 0) {
             if (lane == 0) C.gv[cw] = v;                     // the gate value waits for the up block
           } else if (lane == 0) {

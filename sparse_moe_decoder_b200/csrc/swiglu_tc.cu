@@ -119,6 +119,10 @@ __device__ __forceinline__ void set_abort(Ctrl& C, unsigned int* counter, uint32
   }
 }
 
+// silu(g) * u with the fast exponential and division (~2 ulp of fp32, far below the 11 bits of an f16 h or
+// the 16 of the bf16 pair): the epilogue computes one per h value, on one warp per SM sub-partition.
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.f + __expf(-g)) * u; }
+
 __device__ __forceinline__ uint16_t f32_to_f16_bits(float v) {
   const __half h = __float2half_rn(v);
   return *reinterpret_cast<const uint16_t*>(&h);
@@ -322,7 +326,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                   u0 *= rs * __ldg(p.col_scale1 + j);
                   u1 *= rs * __ldg(p.col_scale1 + j + 1);
                 }
-                const float h0 = g0 / (1.f + expf(-g0)) * u0, h1 = g1 / (1.f + expf(-g1)) * u1;
+                const float h0 = silu_mul(g0, u0), h1 = silu_mul(g1, u1);
                 range_ok = range_ok && fabsf(h0) < 65504.f && fabsf(h1) < 65504.f;
                 const uint16_t b0 = f32_to_f16_bits(h0), b1 = f32_to_f16_bits(h1);
                 if (FMT == kE4M3)
@@ -339,7 +343,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 16; ++i) {
                 const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
                 const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-                const float h0 = g0 / (1.f + expf(-g0)) * u0, h1 = g1 / (1.f + expf(-g1)) * u1;
+                const float h0 = silu_mul(g0, u0), h1 = silu_mul(g1, u1);
                 hi[i] = pack_bf16x2(h0, h1);
                 lo[i] = pack_bf16x2(h0 - __uint_as_float(hi[i] << 16), h1 - __uint_as_float(hi[i] & 0xFFFF0000u));
               }

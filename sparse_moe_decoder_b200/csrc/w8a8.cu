@@ -160,6 +160,17 @@ size_t zmoe_moe_layer_w8a8_workspace_size(int T, int d, int f, int E, int k) {
   return w8_ws(T, E, d, f, k).total;
 }
 
+zmoe_status zmoe_moe_layer_w8a8_workspace_layout(int T, int d, int f, int E, int k, size_t* offsets, int n) {
+  using namespace zmoe;
+  ZMOE_REQUIRE(offsets && n >= 10, "zmoe_moe_layer_w8a8_workspace_layout: needs 10 offsets");
+  ZMOE_REQUIRE(T > 0 && d > 0 && f > 0 && E >= 1 && E <= 64 && (k == 1 || k == 2),
+               "zmoe_moe_layer_w8a8_workspace_layout: bad sizes");
+  const W8Ws W = w8_ws(T, E, d, f, k);
+  const size_t o[10] = {W.counts, W.offsets, W.perm, W.inv_perm, W.xq, W.sx, W.h16, W.hq, W.sh, W.y_perm};
+  for (int i = 0; i < 10; ++i) offsets[i] = o[i];
+  return ZMOE_OK;
+}
+
 zmoe_status zmoe_moe_layer_w8a8(const void* x, const float* h, const float* gamma, float eps, const void* w_router,
                                 const float* logit_bias, const float* sel_bias, const uint8_t* q_gate,
                                 const float* s_gate, const uint8_t* q_up, const float* s_up, const uint8_t* q_down,

@@ -59,6 +59,7 @@ SIGNATURES = {
     "zmoe_grouped_swiglu_f16h": (_I, [_P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "zmoe_moe_layer_f16h_workspace_size": (_S, [_I, _I, _I, _I, _I]),
     "zmoe_moe_layer_w8a8_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "zmoe_moe_layer_w8a8_workspace_layout": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t), _I]),
     "zmoe_moe_layer_w8a8": (_I, [_P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P,
                                  _P, _P, _P, _S, _P]),
     "zmoe_moe_layer_f16h": (_I, [_P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
@@ -496,6 +497,25 @@ def zmoe_moe_layer_w8a8(w_router: Optional[torch.Tensor], q_gate: torch.Tensor, 
                                      _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
            "zmoe_moe_layer_w8a8")
     return y
+
+
+def w8a8_intermediates(workspace: torch.Tensor, T: int, d: int, f: int, E: int, k: int) -> dict:
+    """Views of zmoe_moe_layer_w8a8's intermediates inside its workspace (after the call)."""
+    o = (ctypes.c_size_t * 10)()
+    _check(lib().zmoe_moe_layer_w8a8_workspace_layout(T, d, f, E, k, o, 10), "zmoe_moe_layer_w8a8_workspace_layout")
+    M = T * k
+    shapes = (("counts", torch.int32, (E,)), ("offsets", torch.int32, (E + 1,)), ("perm", torch.int32, (M,)),
+              ("inv_perm", torch.int32, (T, k)), ("xq", torch.uint8, (M, d)), ("sx", torch.float32, (M,)),
+              ("h16", torch.float16, (M, f)), ("hq", torch.uint8, (M, f)), ("sh", torch.float32, (M,)),
+              ("y_perm", torch.float32, (M, d)))
+    out = {}
+    for i, (name, dt, shape) in enumerate(shapes):
+        n = 1
+        for v in shape:
+            n *= v
+        nbytes = n * torch.tensor([], dtype=dt).element_size()
+        out[name] = workspace[o[i]:o[i] + nbytes].view(dt).view(shape)
+    return out
 
 
 def zmoe_decode_stack_workspace_size(n_layers: int, d: int, f: int, E_max: int) -> int:
