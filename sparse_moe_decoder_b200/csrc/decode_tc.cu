@@ -92,8 +92,6 @@ constexpr uint32_t kIdescF16x32 =
 constexpr int kRingBytes = 184 * 1024;
 
 constexpr int kScratch0 = 2 * kMaxAssign * 4;
-// fused layer: weight stages (32 KB each) per CTA prefetched into L2 while routing runs (38 MB in all)
-constexpr int kPrefetchStages = 8;
 
 struct DecArgs {
   const int32_t* offsets;   // [E + 1] (grouped-SwiGLU entry; the fused layer forms its own)
@@ -125,8 +123,6 @@ struct DecArgs {
   // hand_limit_ns; hand_extra is 0 except under zmoe_debug_inject_timeout
   unsigned int hand_extra;
   unsigned long long hand_limit_ns;
-  // fused layer: weight stages of the CTA's expected phase-A range to prefetch into L2 during routing
-  int prefetch_stages;
 };
 
 struct LayerArgs {
@@ -1158,20 +1154,6 @@ __global__ void __launch_bounds__(Lay<FP8>::THREADS, 1)
   const int S[2] = {2 * (p.d / Lay<FP8>::KSTAGE), p.f / Lay<FP8>::KSTAGE};
   init_ctrl<FP8>(C);
   __syncthreads();
-  // Routing takes ~14 us at T = 64, during which HBM would idle.  Prefetch into L2 the first weight
-  // stages of the phase-A range this CTA would get if every expert received one token block (at decode
-  // sizes nearly every expert does; the units and their order are then known before routing).  A wrong
-  // guess costs bandwidth, never results: the loads themselves are unchanged.
-  if (threadIdx.x == 0 && p.prefetch_stages > 0) {
-    const int ub = p.f / BM;
-    const long long total = static_cast<long long>(p.E) * ub * S[0];
-    const long long s0 = total * blockIdx.x / gridDim.x;
-    for (int j = 0; j < p.prefetch_stages && s0 + j < total; ++j) {
-      const long long st = s0 + j;
-      const int u = static_cast<int>(st / S[0]), w = static_cast<int>(st % S[0]);
-      tma_prefetch_3d((w & 1) ? &mapWu : &mapWg, 0, (u / ub) * p.f + (u % ub) * BM, (w >> 1) * CH);
-    }
-  }
   // the ring is idle until the SwiGLU roles start: phase 0 keeps its scratch there
   int* ids = reinterpret_cast<int*>(base);
   int* rel = ids + kMaxAssign;
@@ -1471,7 +1453,6 @@ zmoe_status moe_layer_fused(const uint16_t* x, const float* h_in, const float* g
   a.out = y;
   a.comb_cnt = reinterpret_cast<unsigned int*>(w + W.ffn.comb);
   a.x_ready = L.gbar;                                  // second grid arrival: x_perm complete
-  a.prefetch_stages = kPrefetchStages;
   a.x_target = 2u * static_cast<unsigned int>(num_sms());
   a.s_gate = s_gate;
   a.s_up = s_up;
