@@ -191,6 +191,25 @@ __device__ __forceinline__ float warp_dot_xr(const uint16_t* row, const float (&
   return acc;
 }
 
+// The same for phase B's h (f <= 256 kHChunks).
+constexpr int kHChunks = 12;   // f <= 3072 keeps h in registers
+__device__ __forceinline__ float warp_dot_hr(const uint16_t* row, const float (&hr)[kHChunks][8], int n, int lane) {
+  float acc = 0.f;
+#pragma unroll
+  for (int j = 0; j < kHChunks; ++j) {
+    const int c = lane * 8 + j * 256;
+    if (c < n) {
+      float w[8];
+      unpack_bf16x8(*reinterpret_cast<const uint4*>(row + c), w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc = fmaf(w[i], hr[j][i], acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
+}
+
 // Sum over the CTA (all threads take part); every thread receives the total.
 __device__ __forceinline__ float cta_sum(float v, float* red) {
   v = warp_sum(v);
@@ -550,17 +569,31 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       }
       ok = bar_and(1, kConsumers * 32, ok && !*abort_flag);
       if (ok) ok = __all_sync(0xffffffffu, wait_bounded(&C.hb, static_cast<uint32_t>(l & 1), abort_flag));
-      // phase B: the owned d-rows of each chosen expert
+      // phase B: the owned d-rows of each chosen expert; this expert's h in registers when f fits
+      const bool h_in_regs = f <= 256 * kHChunks;
+      float hr[kHChunks][8];
+      int hr_u = -1;
       for (int i = nA; i < nIt && ok; ++i) {
         const int qq = q + i, slot = qq % kSlots;
         ok = __all_sync(0xffffffffu, wait_bounded(&C.full[slot], static_cast<uint32_t>((qq / kSlots) & 1), abort_flag));
         if (!ok) break;
         const int j = i - nA, u = j / GB, m = (j % GB) * RB;        // m: first row, relative to n0
         const int nr = (nRB - m) < RB ? (nRB - m) : RB;
+        if (h_in_regs && u != hr_u) {
+          const float* hu = hs + static_cast<size_t>(u) * f;
+#pragma unroll
+          for (int jj = 0; jj < kHChunks; ++jj) {
+            const int cidx = lane * 8 + jj * 256;
+#pragma unroll
+            for (int ii = 0; ii < 8; ++ii) hr[jj][ii] = cidx < f ? hu[cidx + ii] : 0.f;
+          }
+          hr_u = u;
+        }
         if (cw < nr) {
           const uint16_t* row = reinterpret_cast<const uint16_t*>(base + static_cast<size_t>(slot) * a.slot_bytes) +
                                 static_cast<size_t>(cw) * f;
-          const float v = warp_dot(row, hs + static_cast<size_t>(u) * f, f, lane);
+          const float v = h_in_regs ? warp_dot_hr(row, hr, f, lane)
+                                    : warp_dot(row, hs + static_cast<size_t>(u) * f, f, lane);
           if (lane == 0) C.ypart[u][m + cw] = v;
         }
         __syncwarp();
