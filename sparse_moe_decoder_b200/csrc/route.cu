@@ -74,74 +74,14 @@ __device__ __forceinline__ float group_sum(float v) {
   return v;
 }
 
-template <typename T, int EP>
-__global__ void __launch_bounds__(kWarps * 32) route_kernel(
-    const T* __restrict__ x, const T* __restrict__ w, const float* __restrict__ logit_bias,
-    const float* __restrict__ sel_bias, int T_, int d, int E, int k, int32_t* __restrict__ expert_idx,
-    float* __restrict__ gates, float* __restrict__ margin) {
-  constexpr int TB = 64 / EP;   // tokens per CTA
-  constexpr int G = EP / 2;     // lanes holding one token's logits
-  __shared__ float2 part[kWarps][32];
-
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int t0 = blockIdx.x * TB;
-
-  float acc[TB * EP];
-#pragma unroll
-  for (int i = 0; i < TB * EP; ++i) acc[i] = 0.f;
-
-  for (int c = warp; c * 256 < d; c += kWarps) {
-    const int k0 = c * 256 + lane * 8;
-    if (k0 < d) {
-      float xv[TB][8];
-#pragma unroll
-      for (int tb = 0; tb < TB; ++tb) {
-        if (t0 + tb < T_) {
-          load8v<T>(x + static_cast<size_t>(t0 + tb) * d + k0, xv[tb]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) xv[tb][i] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < EP; ++e) {
-        if (e < E) {
-          float wv[8];
-          load8v<T>(w + static_cast<size_t>(e) * d + k0, wv);
-#pragma unroll
-          for (int tb = 0; tb < TB; ++tb) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[tb * EP + e] = fmaf(wv[i], xv[tb][i], acc[tb * EP + e]);
-          }
-        }
-      }
-    }
-  }
-
-  // Reduce-scatter over the warp: after the step with offset o, a lane keeps the upper half
-  // of its current values when (lane & o) != 0.  After 5 steps lane l holds entries 2l, 2l+1.
-#pragma unroll
-  for (int o = 16, n = 64; o > 0; o >>= 1, n >>= 1) {
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < n / 2; ++i) {
-      const float send = upper ? acc[i] : acc[i + n / 2];
-      const float keep = upper ? acc[i + n / 2] : acc[i];
-      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-  part[warp][lane] = make_float2(acc[0], acc[1]);
-  __syncthreads();
-  if (warp != 0) return;
-
-  float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-  for (int w2 = 0; w2 < kWarps; ++w2) {
-    l0 += part[w2][lane].x;
-    l1 += part[w2][lane].y;
-  }
-  const int tok = t0 + (2 * lane) / EP;
+// Top-k, gates and margin of one token from the logits its G = EP / 2 lanes hold: lane l of the group
+// holds the (unbiased) logits l0, l1 of experts 2 (l % G) and 2 (l % G) + 1.  Lane 0 of the group writes.
+template <int EP>
+__device__ __forceinline__ void finish_topk(float l0, float l1, int tok, int lane, int T_, int E, int k,
+                                            const float* __restrict__ logit_bias, const float* __restrict__ sel_bias,
+                                            int32_t* __restrict__ expert_idx, float* __restrict__ gates,
+                                            float* __restrict__ margin) {
+  constexpr int G = EP / 2;
   const int ea = (2 * lane) % EP, eb = ea + 1;
   const bool va = ea < E, vb = eb < E;
   const float NEG = -INFINITY;
@@ -213,11 +153,168 @@ __global__ void __launch_bounds__(kWarps * 32) route_kernel(
   }
 }
 
+template <typename T, int EP>
+__global__ void __launch_bounds__(kWarps * 32) route_kernel(
+    const T* __restrict__ x, const T* __restrict__ w, const float* __restrict__ logit_bias,
+    const float* __restrict__ sel_bias, int T_, int d, int E, int k, int32_t* __restrict__ expert_idx,
+    float* __restrict__ gates, float* __restrict__ margin) {
+  constexpr int TB = 64 / EP;   // tokens per CTA
+  constexpr int G = EP / 2;     // lanes holding one token's logits
+  __shared__ float2 part[kWarps][32];
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int t0 = blockIdx.x * TB;
+
+  float acc[TB * EP];
+#pragma unroll
+  for (int i = 0; i < TB * EP; ++i) acc[i] = 0.f;
+
+  for (int c = warp; c * 256 < d; c += kWarps) {
+    const int k0 = c * 256 + lane * 8;
+    if (k0 < d) {
+      float xv[TB][8];
+#pragma unroll
+      for (int tb = 0; tb < TB; ++tb) {
+        if (t0 + tb < T_) {
+          load8v<T>(x + static_cast<size_t>(t0 + tb) * d + k0, xv[tb]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) xv[tb][i] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        if (e < E) {
+          float wv[8];
+          load8v<T>(w + static_cast<size_t>(e) * d + k0, wv);
+#pragma unroll
+          for (int tb = 0; tb < TB; ++tb) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[tb * EP + e] = fmaf(wv[i], xv[tb][i], acc[tb * EP + e]);
+          }
+        }
+      }
+    }
+  }
+
+  // Reduce-scatter over the warp: after the step with offset o, a lane keeps the upper half
+  // of its current values when (lane & o) != 0.  After 5 steps lane l holds entries 2l, 2l+1.
+#pragma unroll
+  for (int o = 16, n = 64; o > 0; o >>= 1, n >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float send = upper ? acc[i] : acc[i + n / 2];
+      const float keep = upper ? acc[i + n / 2] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  part[warp][lane] = make_float2(acc[0], acc[1]);
+  __syncthreads();
+  if (warp != 0) return;
+
+  float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+  for (int w2 = 0; w2 < kWarps; ++w2) {
+    l0 += part[w2][lane].x;
+    l1 += part[w2][lane].y;
+  }
+  finish_topk<EP>(l0, l1, t0 + (2 * lane) / EP, lane, T_, E, k, logit_bias, sel_bias, expert_idx, gates, margin);
+}
+
+// Prefill sizes (bf16, E <= 16): persistent CTAs stage the whole router matrix in shared memory once;
+// each warp takes TB = 4 tokens at a time over the whole d (lane l: elements [c 256 + 8 l, + 8) of every
+// chunk c), so no partial sums cross warps and each router byte read from memory serves every token of
+// the CTA.  The per-token sums then take the same reduce-scatter and top-k as route_kernel.
+template <int EP>
+__global__ void __launch_bounds__(kWarps * 32) route_rows_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ w, const float* __restrict__ logit_bias,
+    const float* __restrict__ sel_bias, int T_, int d, int E, int k, int32_t* __restrict__ expert_idx,
+    float* __restrict__ gates, float* __restrict__ margin) {
+  constexpr int TB = 64 / EP;
+  extern __shared__ uint4 wsm[];   // [E][d / 8] 16-byte vectors of bf16
+  const int vecs = E * (d / 8);
+  for (int i = threadIdx.x; i < vecs; i += blockDim.x) wsm[i] = __ldg(reinterpret_cast<const uint4*>(w) + i);
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int groups = (T_ + TB - 1) / TB;
+  const int dv = d / 8;
+  for (int gi = blockIdx.x * kWarps + warp; gi < groups; gi += gridDim.x * kWarps) {
+    const int t0 = gi * TB;
+    float acc[TB * EP];
+#pragma unroll
+    for (int i = 0; i < TB * EP; ++i) acc[i] = 0.f;
+    // x chunks are loaded one chunk ahead of the arithmetic (the raw 16-byte vectors stay packed)
+    uint4 xn[TB];
+    const int nch = (d + 255) / 256;
+    auto load_chunk = [&](int c, uint4 (&dst)[TB]) {
+      const int k0 = c * 256 + lane * 8;
+#pragma unroll
+      for (int tb = 0; tb < TB; ++tb)
+        dst[tb] = (k0 < d && t0 + tb < T_) ? __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + tb) * d + k0))
+                                           : make_uint4(0u, 0u, 0u, 0u);
+    };
+    load_chunk(0, xn);
+    for (int c = 0; c < nch; ++c) {
+      const int k0 = c * 256 + lane * 8;
+      float xv[TB][8];
+#pragma unroll
+      for (int tb = 0; tb < TB; ++tb) unpack_bf16x8(xn[tb], xv[tb]);
+      if (c + 1 < nch) load_chunk(c + 1, xn);
+      if (k0 < d) {
+#pragma unroll
+        for (int e = 0; e < EP; ++e) {
+          if (e < E) {
+            float wv[8];
+            unpack_bf16x8(wsm[e * dv + (k0 >> 3)], wv);
+#pragma unroll
+            for (int tb = 0; tb < TB; ++tb) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[tb * EP + e] = fmaf(wv[i], xv[tb][i], acc[tb * EP + e]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16, n = 64; o > 0; o >>= 1, n >>= 1) {
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < n / 2; ++i) {
+        const float send = upper ? acc[i] : acc[i + n / 2];
+        const float keep = upper ? acc[i + n / 2] : acc[i];
+        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    finish_topk<EP>(acc[0], acc[1], t0 + (2 * lane) / EP, lane, T_, E, k, logit_bias, sel_bias, expert_idx, gates,
+                    margin);
+  }
+}
+
+// Tokens from which the prefill router kernel is used (below, the one-CTA-per-4-tokens kernel needs no
+// staging of the router matrix).
+constexpr int kRowsMinT = 512;
+
 template <typename T>
 void launch_route(const void* x, const void* w, const float* lb, const float* sb, int T_, int d, int E, int k,
                   int32_t* idx, float* g, float* mg, cudaStream_t s) {
   const T* xp = static_cast<const T*>(x);
   const T* wp = static_cast<const T*>(w);
+  const size_t wbytes = static_cast<size_t>(E) * d * sizeof(T);
+  if (sizeof(T) == 2 && E <= 16 && T_ >= kRowsMinT && wbytes <= 96 * 1024) {
+    auto kern = route_rows_kernel<16>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(wbytes)) ==
+        cudaSuccess) {
+      const int groups = (T_ + 3) / 4;
+      int grid = 2 * num_sms();   // two CTAs per SM (128 registers, <= 96 KB each), persistent over the groups
+      if (grid * kWarps > groups) grid = (groups + kWarps - 1) / kWarps;
+      kern<<<grid, kWarps * 32, wbytes, s>>>(reinterpret_cast<const uint16_t*>(xp), reinterpret_cast<const uint16_t*>(wp),
+                                              lb, sb, T_, d, E, k, idx, g, mg);
+      return;
+    }
+    cudaGetLastError();
+  }
   if (E <= 16) {
     route_kernel<T, 16><<<(T_ + 3) / 4, kWarps * 32, 0, s>>>(xp, wp, lb, sb, T_, d, E, k, idx, g, mg);
   } else if (E <= 32) {
