@@ -191,6 +191,19 @@ __device__ __forceinline__ float warp_dot_xr(const uint16_t* row, const float (&
   return acc;
 }
 
+// v[c .. c + 8) from shared memory as two 16-byte loads (zeros when c >= n).
+__device__ __forceinline__ void load_chunk8(const float* v, int c, int n, float (&out)[8]) {
+  if (c < n) {
+    const float4 a = *reinterpret_cast<const float4*>(v + c);
+    const float4 b = *reinterpret_cast<const float4*>(v + c + 4);
+    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+    out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = 0.f;
+  }
+}
+
 // The same for phase B's h (f <= 256 kHChunks).
 constexpr int kHChunks = 12;   // f <= 3072 keeps h in registers
 __device__ __forceinline__ float warp_dot_hr(const uint16_t* row, const float (&hr)[kHChunks][8], int n, int lane) {
@@ -208,6 +221,17 @@ __device__ __forceinline__ float warp_dot_hr(const uint16_t* row, const float (&
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   return acc;
+}
+
+// Order-preserving map of a float onto uint32 (larger float -> larger key; -0 maps like +0).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f + 0.f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The inverse of order_key.
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
 // Sum over the CTA (all threads take part); every thread receives the total.
@@ -389,11 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
     const bool x_in_regs = d <= 256 * kXChunks;
     float xr[kXChunks][8];
 #pragma unroll
-    for (int j = 0; j < kXChunks; ++j) {
-      const int cidx = lane * 8 + j * 256;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) xr[j][i] = (x_in_regs && cidx < d) ? xs[cidx + i] : 0.f;
-    }
+    for (int j = 0; j < kXChunks; ++j) load_chunk8(xs, lane * 8 + j * 256, x_in_regs ? d : 0, xr[j]);
     // ---- router logits, one warp per expert ----
     if (Ly.w_r) {
       const uint16_t* wr = reinterpret_cast<const uint16_t*>(wr_s);
@@ -405,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
     }
     __syncthreads();
     // ---- top-k (larger score first, ties to the lower index) and gates, by warp 0: lane l holds experts
-    // l and l + 32; maxima, arg-maxima and the softmax sum by butterflies ----
+    // l and l + 32; maxima and arg-maxima by warp reductions, the softmax sum by a butterfly ----
     if (warp == 0) {
       if (!Ly.w_r) {
         if (lane == 0) {
@@ -414,16 +434,19 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
           C.nu = 1;
         }
       } else {
-        float qv[2], sv[2];
+        // scores as order-preserving keys (0: no expert; 1: a NaN score, chosen only when nothing else is
+        // left), so that each choice is a warp max then a warp min of the expert index among the maxima
+        float qv[2];
+        uint32_t sk[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const int e = lane + 32 * j;
           qv[j] = e < E ? C.logit[e] + C.qb[e] : -INFINITY;
-          sv[j] = e < E ? qv[j] + C.sb[e] : -INFINITY;
+          const float sv = e < E ? qv[j] + C.sb[e] : 0.f;
+          sk[j] = e >= E ? 0u : (sv != sv ? 1u : order_key(sv));
         }
-        float m = fmaxf(qv[0], qv[1]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const uint32_t qk = max(qv[0] != qv[0] ? 0u : order_key(qv[0]), qv[1] != qv[1] ? 0u : order_key(qv[1]));
+        const float m = key_float(__reduce_max_sync(0xffffffffu, qk));   // the largest logit (NaN ignored)
         float z = (lane < E ? expf(qv[0] - m) : 0.f) + (lane + 32 < E ? expf(qv[1] - m) : 0.f);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
@@ -432,28 +455,17 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
 #pragma unroll
         for (int i = 0; i < kMaxK; ++i) {
           if (i >= k) break;
-          // the lane's best candidate not chosen yet, then the warp's (larger score, else lower index)
-          float bs = -INFINITY;
-          int be = 0x7fffffff;
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int e = lane + 32 * j;
-            if (e < E && (i == 0 || e != sel[0]) && (sv[j] > bs || (sv[j] == bs && e < be))) {
-              bs = sv[j];
-              be = e;
-            }
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            if (os > bs || (os == bs && oe < be)) {
-              bs = os;
-              be = oe;
-            }
-          }
+          const bool hi = sk[1] > sk[0];   // the lane's best (its lower expert on a tie)
+          const uint32_t kb = hi ? sk[1] : sk[0];
+          const uint32_t mk = __reduce_max_sync(0xffffffffu, kb);
+          const int be = static_cast<int>(
+              __reduce_min_sync(0xffffffffu, kb == mk ? static_cast<uint32_t>(hi ? lane + 32 : lane) : 0xffffu));
           sel[i] = be;
           qsel[i] = __shfl_sync(0xffffffffu, (be >> 5) ? qv[1] : qv[0], be & 31);
+          if ((be & 31) == lane) {   // not chosen twice
+            if (be >> 5) sk[1] = 0u;
+            else sk[0] = 0u;
+          }
         }
         if (lane == 0) {
           if (k == 1) {
@@ -582,11 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
         if (h_in_regs && u != hr_u) {
           const float* hu = hs + static_cast<size_t>(u) * f;
 #pragma unroll
-          for (int jj = 0; jj < kHChunks; ++jj) {
-            const int cidx = lane * 8 + jj * 256;
-#pragma unroll
-            for (int ii = 0; ii < 8; ++ii) hr[jj][ii] = cidx < f ? hu[cidx + ii] : 0.f;
-          }
+          for (int jj = 0; jj < kHChunks; ++jj) load_chunk8(hu, lane * 8 + jj * 256, f, hr[jj]);
           hr_u = u;
         }
         if (cw < nr) {
