@@ -21,6 +21,10 @@
 #include "common.cuh"
 
 namespace zmoe {
+
+bool launch_route_tc(const void* x, const void* w, const float* lb, const float* sb, int T, int d, int E, int k,
+                     int32_t* idx, float* g, float* mg, cudaStream_t s);
+
 namespace {
 
 constexpr int kWarps = 8;
@@ -292,7 +296,7 @@ __global__ void __launch_bounds__(kWarps * 32) route_rows_kernel(
   }
 }
 
-// Tokens from which the prefill router kernel is used (below, the one-CTA-per-4-tokens kernel needs no
+// Tokens from which the persistent CUDA-core router kernel is used (below, the one-CTA-per-4-tokens kernel needs no
 // staging of the router matrix).
 constexpr int kRowsMinT = 512;
 
@@ -302,6 +306,8 @@ void launch_route(const void* x, const void* w, const float* lb, const float* sb
   const T* xp = static_cast<const T*>(x);
   const T* wp = static_cast<const T*>(w);
   const size_t wbytes = static_cast<size_t>(E) * d * sizeof(T);
+  // the tensor-core router (bf16, E <= 32, d % 64 == 0, T >= 2048)
+  if (sizeof(T) == 2 && launch_route_tc(x, w, lb, sb, T_, d, E, k, idx, g, mg, s)) return;
   if (sizeof(T) == 2 && E <= 16 && T_ >= kRowsMinT && wbytes <= 96 * 1024) {
     auto kern = route_rows_kernel<16>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(wbytes)) ==

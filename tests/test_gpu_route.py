@@ -80,3 +80,44 @@ def test_route_without_router_single_expert():
     x = torch.randn(37, 256, device="cuda").to(torch.bfloat16)
     idx, g, mg = zmoe_route(x, None, 1)
     assert (host(idx) == 0).all() and (host(g) == 1.0).all() and np.isinf(host(mg)).all()
+
+
+@pytest.mark.parametrize("T,d,E,k", [(2048, 2048, 16, 1), (3001, 2048, 16, 2), (2100, 256, 20, 2), (4096, 2048, 32, 1),
+                                     (2049, 1024, 32, 2), (2048, 2048, 1, 1), (2500, 192, 3, 2)])
+def test_route_tensor_core_shapes(T, d, E, k):
+    """Sizes taken by the tensor-core router (bf16, E <= 32, d % 64 == 0, T >= 2048): ragged last tile,
+    experts padded to 16 or 32 columns, fewer k-stages than the ring holds."""
+    require_gpu()
+    L = make_moe_layer(T, d, 8, E, k, "bf16", seed=T + d + E, sel_bias_var=0.3, zipf_s=1.2)
+    exempt = check_route(L, f"T={T} d={d} E={E} k={k}")
+    print(f"T={T} d={d} E={E} k={k}: {exempt} low-margin tokens exempt")
+
+
+def test_route_tensor_core_exact_ties_lowest_index():
+    """Exact ties at a tensor-core size: duplicated router rows give bit-identical logit columns, and
+    the lower expert index wins."""
+    require_gpu()
+    E, d, T = 12, 512, 2304
+    rng = np.random.default_rng(5)
+    w = rng.standard_normal((E, d)).astype(np.float32)
+    w[7] = w[2]
+    w[9] = w[2]
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    xb, wb = to_dev(x, torch.bfloat16), to_dev(w, torch.bfloat16)
+    idx, g, _ = zmoe_route(xb, wb, 2)
+    sel, gates, _, _ = oracle.route(host(xb.float()), host(wb.float()), 2)
+    idx, g = host(idx), host(g)
+    assert ((sel == 2) | (sel == 7) | (sel == 9)).any(), "the tie must reach the top-2 somewhere"
+    # 2 beats its copies 7 and 9: 9 is never among two choices, and 7 only as [2, 7]
+    assert not (idx == 9).any()
+    has7 = (idx == 7).any(axis=1)
+    assert (idx[has7, 0] == 2).all() and (idx[has7, 1] == 7).all()
+    _, _, margin, _ = oracle.route(host(xb.float()), host(wb.float()), 2)
+    ok = margin >= MARGIN_EXEMPT
+    # the tied pair itself has margin 0 in the oracle; where experts 2 and 7 are the top two, the GPU
+    # must list 2 first and 7 second
+    tied = (sel[:, 0] == 2) & (sel[:, 1] == 7)
+    assert tied.any()
+    assert np.array_equal(idx[tied], sel[tied])
+    assert np.array_equal(idx[ok], sel[ok])
+    assert np.allclose(g[tied], 0.5, atol=1e-6)
