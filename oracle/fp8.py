@@ -9,11 +9,12 @@ the decoded weights.  float64.
 
 At prefill sizes the layer runs W8A8 (fp8 weights AND fp8 activations, the scheme fp8 serving stacks
 use for dynamic activation quantization): the rows entering each expert GEMM are quantized per token
-with a dynamic scale s = max|row| / 448 and codes = the E4M3 value nearest row / s (ties to even,
-magnitudes saturating at 448); the first GEMM's input is the permuted token row, the second's the
-hidden activation h, which is held at 16 bits (f16) between the two GEMMs and quantized from that.
-The scale and the quotient are computed in fp32 (the precision in which the kernel takes the same
-decision), everything else in float64.
+with a dynamic scale s = max|row| / 448 and codes = the E4M3 value nearest row x (1 / s) (ties to
+even, magnitudes saturating at 448); the first GEMM's input is the permuted token row, the second's
+the hidden activation h, which is held at 16 bits (f16) between the two GEMMs and quantized from that.
+The scale, its reciprocal and the scaled row are computed in fp32 (the precision in which the kernel
+takes the same decision: one reciprocal per row, then a multiplication per element, the usual form of
+a dynamic-quantization kernel), everything else in float64.
 """
 from __future__ import annotations
 
@@ -70,12 +71,13 @@ def e4m3_encode(v: np.ndarray) -> np.ndarray:
 
 
 def quantize_rows_dynamic(a: np.ndarray):
-    """Per-row dynamic E4M3 quantization: s = fp32(max|row| / 448) (1 for an all-zero row) and
-    codes = e4m3_encode(fp32(row / s)).  Returns (codes uint8, s float32)."""
+    """Per-row dynamic E4M3 quantization: s = fp32(max|row| / 448) (1 for an all-zero row),
+    r = fp32(1 / s) and codes = e4m3_encode(fp32(row x r)).  Returns (codes uint8, s float32)."""
     a32 = np.asarray(a, np.float32)
     amax = np.max(np.abs(a32), axis=-1)
     s = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
-    q = e4m3_encode((a32 / s[..., None]).astype(np.float32))
+    r = (np.float32(1.0) / s).astype(np.float32)
+    q = e4m3_encode((a32 * r[..., None]).astype(np.float32))
     return q, s
 
 

@@ -4,8 +4,8 @@
 // The ZONOS2 serving stack runs the model in fp8 (ZONOS2 page of the sglang-omni cookbook, "Benchmark
 // Results").  Reading taken for prefill sizes: the common fp8 serving scheme with dynamic activation
 // quantization: each row entering an expert GEMM (the permuted token row, then the hidden row h) gets
-//   s = max|row| / 448  (fp32; 1 for an all-zero row),   codes = E4M3 nearest row / s (ties to even,
-//   saturating at 448),
+//   s = max|row| / 448  (fp32; 1 for an all-zero row),   codes = E4M3 nearest row x fp32(1 / s) (ties
+//   to even, saturating at 448; one correctly rounded reciprocal per row, one product per element),
 // and the tensor cores run kind::f8f6f4 at twice the bf16 rate; the fp32 sums are multiplied by the row's
 // token scale and the weight row's scale.  h is held in f16 between the two GEMMs (the first GEMM's
 // epilogue also records each row's max |h|), then quantized per token.
@@ -40,19 +40,23 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 // The per-token scale of a row whose largest magnitude is amax.
 __device__ __forceinline__ float token_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f; }
 
-// 8 values (fp32) divided by s and encoded: 8 codes in a uint2, the first value in the lowest byte.
-__device__ __forceinline__ uint2 encode8(const float* v, float s) {
+// 8 values (fp32) multiplied by r = fp32(1 / s) and encoded: 8 codes in a uint2, the first value in the
+// lowest byte.
+__device__ __forceinline__ uint2 encode8(const float* v, float r) {
   uint32_t w[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const uint16_t a = e4m3x2(__fdiv_rn(v[4 * i], s), __fdiv_rn(v[4 * i + 1], s));
-    const uint16_t b = e4m3x2(__fdiv_rn(v[4 * i + 2], s), __fdiv_rn(v[4 * i + 3], s));
+    const uint16_t a = e4m3x2(__fmul_rn(v[4 * i], r), __fmul_rn(v[4 * i + 1], r));
+    const uint16_t b = e4m3x2(__fmul_rn(v[4 * i + 2], r), __fmul_rn(v[4 * i + 3], r));
     w[i] = static_cast<uint32_t>(a) | (static_cast<uint32_t>(b) << 16);
   }
   return make_uint2(w[0], w[1]);
 }
 
-// xq[r] = E4M3(x[perm[r]] / sx[r]), sx[r] = max|x[perm[r]]| / 448, one warp per permuted row.
+constexpr int kRowChunks = 12;   // a row of up to 12 x 256 elements stays in registers (8 per lane per chunk)
+
+// xq[r] = E4M3(x[perm[r]] x fp32(1 / sx[r])), sx[r] = max|x[perm[r]]| / 448, one warp per permuted row
+// (the row is read once into registers when d <= 256 kRowChunks).
 __global__ void __launch_bounds__(kThreads) gather_quantize_kernel(const uint16_t* __restrict__ x,
                                                                     const int32_t* __restrict__ perm,
                                                                     const int32_t* __restrict__ offsets, int E, int d,
@@ -60,28 +64,58 @@ __global__ void __launch_bounds__(kThreads) gather_quantize_kernel(const uint16_
   const int lane = threadIdx.x & 31;
   const long long rows = offsets[E];
   const long long warps = static_cast<long long>(gridDim.x) * (kThreads / 32);
+  const bool in_regs = d <= 256 * kRowChunks;
   for (long long r = blockIdx.x * static_cast<long long>(kThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
     const uint16_t* src = x + static_cast<size_t>(perm[r]) * d;
+    uint4 raw[kRowChunks];
     float amax = 0.f;
-    for (int c = lane * 8; c < d; c += 256) {
-      float v[8];
-      unpack_bf16x8(*reinterpret_cast<const uint4*>(src + c), v);
+    if (in_regs) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      for (int j = 0; j < kRowChunks; ++j) {
+        const int c = lane * 8 + j * 256;
+        raw[j] = c < d ? __ldg(reinterpret_cast<const uint4*>(src + c)) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int j = 0; j < kRowChunks; ++j) {
+        float v[8];
+        unpack_bf16x8(raw[j], v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      }
+    } else {
+      for (int c = lane * 8; c < d; c += 256) {
+        float v[8];
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(src + c), v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float s = token_scale(amax);
-    for (int c = lane * 8; c < d; c += 256) {
-      float v[8];
-      unpack_bf16x8(*reinterpret_cast<const uint4*>(src + c), v);
-      *reinterpret_cast<uint2*>(xq + static_cast<size_t>(r) * d + c) = encode8(v, s);
+    const float s = token_scale(amax), rs = __frcp_rn(s);
+    if (in_regs) {
+#pragma unroll
+      for (int j = 0; j < kRowChunks; ++j) {
+        const int c = lane * 8 + j * 256;
+        if (c < d) {
+          float v[8];
+          unpack_bf16x8(raw[j], v);
+          *reinterpret_cast<uint2*>(xq + static_cast<size_t>(r) * d + c) = encode8(v, rs);
+        }
+      }
+    } else {
+      for (int c = lane * 8; c < d; c += 256) {
+        float v[8];
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(src + c), v);
+        *reinterpret_cast<uint2*>(xq + static_cast<size_t>(r) * d + c) = encode8(v, rs);
+      }
     }
     if (lane == 0) sx[r] = s;
   }
 }
 
-// hq[r] = E4M3(h16[r] / sh[r]), sh[r] = amax[r] / 448 (amax: bits of max |h16[r]|), one warp per row.
+// hq[r] = E4M3(h16[r] x fp32(1 / sh[r])), sh[r] = amax[r] / 448 (amax: bits of max |h16[r]|), one warp
+// per row.
 __global__ void __launch_bounds__(kThreads) quantize_h_kernel(const uint16_t* __restrict__ h16,
                                                                const unsigned int* __restrict__ amax,
                                                                const int32_t* __restrict__ offsets, int E, int f,
@@ -90,7 +124,7 @@ __global__ void __launch_bounds__(kThreads) quantize_h_kernel(const uint16_t* __
   const long long rows = offsets[E];
   const long long warps = static_cast<long long>(gridDim.x) * (kThreads / 32);
   for (long long r = blockIdx.x * static_cast<long long>(kThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
-    const float s = token_scale(__uint_as_float(amax[r]));
+    const float s = token_scale(__uint_as_float(amax[r])), rs = __frcp_rn(s);
     const uint16_t* src = h16 + static_cast<size_t>(r) * f;
     for (int c = lane * 8; c < f; c += 256) {
       const uint4 raw = *reinterpret_cast<const uint4*>(src + c);
@@ -101,7 +135,7 @@ __global__ void __launch_bounds__(kThreads) quantize_h_kernel(const uint16_t* __
         v[2 * i] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[i] & 0xFFFFu)));
         v[2 * i + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[i] >> 16)));
       }
-      *reinterpret_cast<uint2*>(hq + static_cast<size_t>(r) * f + c) = encode8(v, s);
+      *reinterpret_cast<uint2*>(hq + static_cast<size_t>(r) * f + c) = encode8(v, rs);
     }
     if (lane == 0) sh[r] = s;
   }

@@ -462,6 +462,24 @@ def pin_w8a8(e4m3_encode, quantize_rows_dynamic, moe_layer_w8a8):
     assert s[0] == np.float32(2 ** -3) and list(q[0]) == [0x7E, 0xB8, 0x30, 0x00]
     q0, s0 = quantize_rows_dynamic(np.zeros((1, 8), np.float32))
     assert s0[0] == 1.0 and not q0.any()
+    # the scaled row is row x fp32(1 / s), each product rounded to fp32 (torch's fp32 arithmetic and its
+    # float8 conversion): rows with a value next to an E4M3 midpoint, picked where dividing by s instead
+    # rounds to the other neighbour
+    rows = []
+    while len(rows) < 6:
+        s_ = np.float32(rng.random() + 0.5)
+        amax_ = np.float32(448.0) * s_
+        sq = np.float32(amax_ / np.float32(448.0))
+        v_ = np.float32(mids[rng.integers(1, 125)] * sq)
+        by_mul = np.float32(v_ * np.float32(np.float32(1.0) / sq))
+        if e4m3_encode(np.array([by_mul]))[0] != e4m3_encode(np.array([np.float32(v_ / sq)]))[0]:
+            rows.append([v_, amax_])
+    rows = np.array(rows, np.float32)
+    q, s = quantize_rows_dynamic(rows)
+    rt = torch.from_numpy(rows)
+    st = rt.abs().amax(dim=1) / torch.tensor(448.0, dtype=torch.float32)
+    ref_codes = (rt * (1.0 / st)[:, None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(s, st.numpy()) and np.array_equal(q, ref_codes)
     # one expert, W8A8, against torch
     d, f, T = 32, 96, 35     # 3360 hidden values: the f16 step moves ~0.4% of them across an E4M3 midpoint
     qg, qu, qd = (rng.integers(0, 0x7E, size=sh).astype(np.uint8) | (rng.integers(0, 2, size=sh) << 7).astype(np.uint8)
@@ -475,7 +493,7 @@ def pin_w8a8(e4m3_encode, quantize_rows_dynamic, moe_layer_w8a8):
         a32 = torch.from_numpy(np.asarray(a32, np.float32))
         s_ = a32.abs().amax(dim=1) / torch.tensor(448.0, dtype=torch.float32)
         s_ = torch.where(s_ > 0, s_, torch.ones_like(s_))
-        return (a32 / s_[:, None]).to(torch.float8_e4m3fn).double() * s_.double()[:, None]
+        return (a32 * (1.0 / s_)[:, None]).to(torch.float8_e4m3fn).double() * s_.double()[:, None]
 
     W = lambda q_, s_: torch.from_numpy(q_[0]).view(torch.float8_e4m3fn).double() * torch.from_numpy(s_[0]).double()[:, None]
     xq = tq(x)

@@ -279,6 +279,14 @@ def _quantize_per_tensor(a):
     return q, np.full(a32.shape[:-1], s, np.float32)
 
 
+def _quantize_by_division(a):
+    """Planted: the scaled row formed as row / s instead of row x fp32(1 / s)."""
+    a32 = np.asarray(a, np.float32)
+    amax = np.max(np.abs(a32), axis=-1)
+    s = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    return oracle.e4m3_encode((a32 / s[..., None]).astype(np.float32)), s
+
+
 def _w8a8_layer_with(quantizer):
     import oracle.fp8 as F8
     saved = F8.quantize_rows_dynamic
@@ -351,6 +359,8 @@ MUTANTS = {
                                                     oracle.moe_layer_w8a8),
     "w8a8 activations scaled per tensor": lambda: P.pin_w8a8(oracle.e4m3_encode, oracle.quantize_rows_dynamic,
                                                              _w8a8_layer_with(_quantize_per_tensor)),
+    "w8a8 quotient by division": lambda: P.pin_w8a8(oracle.e4m3_encode, _quantize_by_division,
+                                                    _w8a8_layer_with(_quantize_by_division)),
     "w8a8 hidden activation without f16": lambda: P.pin_w8a8(oracle.e4m3_encode, oracle.quantize_rows_dynamic,
                                                              _w8a8_no_f16_hidden),
     "dense layer drops residual": lambda: P.pin_stack_dense(_stack_dense_no_residual, oracle.embed_sum_rmsnorm,
