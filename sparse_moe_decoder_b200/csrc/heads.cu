@@ -27,6 +27,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kRowsPerStage = kWarps;   // one head row per warp per stage
 constexpr int kTok = 8;           // tokens per pass over the weights
 constexpr int kMaxStages = 8;
+constexpr int kXC = 8;            // a single bf16 token row of d <= 256 kXC is held in registers
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
 struct HeadArgs {
@@ -50,6 +51,7 @@ struct __align__(8) HeadCtrl {
   uint64_t full[kMaxStages];
   uint64_t xbar;             // token rows (+ gamma) of the current pass
   unsigned long long best[kTok][2];   // this CTA's best key per token for its first two codebooks
+  float red[kWarps][kTok];   // per-warp partial sums of squares (the final norm)
   int abort;
 };
 
@@ -156,7 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
   bool ok = true;
   for (int t0 = 0; t0 < a.T && ok; t0 += kTok) {
     const int nt = (a.T - t0) < kTok ? (a.T - t0) : kTok;
-    // token rows of this pass (and gamma, first pass) by bulk copy: one round trip, not one per load
+    // the pass's token rows (and gamma, first pass) by bulk copy, one round trip, then its first weight
+    // stages, which do not depend on x and land while x is formed
     const int pass = t0 / kTok;
     if (threadIdx.x == 0) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -170,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
       for (uint32_t o = 0; o < gb; o += 32768u)
         bulk_load(reinterpret_cast<unsigned char*>(gam) + o, reinterpret_cast<const unsigned char*>(a.gamma) + o,
                   gb - o < 32768u ? gb - o : 32768u, &C.xbar);
+      for (int s = 0; s < nst && s < a.stages; ++s) issue_stage(a, C, ring, slot_bytes, (q + s) % a.stages, r0, r1, s);
     }
     ok = __syncthreads_and(mbar_wait(&C.xbar, static_cast<uint32_t>(pass & 1), abort_flag, kTimeoutNs));
     if (!ok) {
@@ -178,38 +182,80 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
         const uint64_t t1 = globaltimer();
         while (!mbar_try_wait(&C.xbar, static_cast<uint32_t>(pass & 1)) && globaltimer() - t1 < kTimeoutNs) {
         }
+        // the weight stages issued above must land before the CTA leaves
+        for (int s2 = 0; s2 < nst && s2 < a.stages; ++s2) {
+          const int slot = (q + s2) % a.stages;
+          const uint32_t par = static_cast<uint32_t>(((q + s2) / a.stages) & 1);
+          const uint64_t t2 = globaltimer();
+          while (!mbar_try_wait(&C.full[slot], par) && globaltimer() - t2 < kTimeoutNs) {
+          }
+        }
       }
       break;
     }
     if (threadIdx.x < 2 * kTok) (&C.best[0][0])[threadIdx.x] = 0ull;
-    // one warp per token: optional RMSNorm, rounding to the weights' type
-    if (warp < nt) {
-      const int t = t0 + warp;
-      const float* hr = raw + static_cast<size_t>(warp) * d;
-      float inv = 1.f;
-      if (a.gamma) {
-        float ss = 0.f;
-        for (int c = lane; c < d; c += 32) ss = fmaf(hr[c], hr[c], ss);
+    // optional RMSNorm of each token row, by the whole CTA (sums of squares per thread, then per warp,
+    // then over the warps), and rounding to the weights' type
+    float inv[kTok];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        inv = rsqrtf(ss / static_cast<float>(d) + a.eps);
+    for (int t = 0; t < kTok; ++t) inv[t] = 1.f;
+    if (a.gamma) {
+      float ss[kTok];
+#pragma unroll
+      for (int t = 0; t < kTok; ++t) ss[t] = 0.f;
+      for (int c = threadIdx.x; c < d; c += kThreads) {
+#pragma unroll
+        for (int t = 0; t < kTok; ++t)
+          if (t < nt) ss[t] = fmaf(raw[static_cast<size_t>(t) * d + c], raw[static_cast<size_t>(t) * d + c], ss[t]);
       }
-      for (int c = lane; c < d; c += 32) {
-        float v = a.gamma ? hr[c] * inv * gam[c] : hr[c];
+#pragma unroll
+      for (int t = 0; t < kTok; ++t) {
+        if (t < nt) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) ss[t] += __shfl_xor_sync(0xffffffffu, ss[t], o);
+          if (lane == 0) C.red[warp][t] = ss[t];
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int t = 0; t < kTok; ++t) {
+        if (t < nt) {
+          float tot = 0.f;
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) tot += C.red[w][t];
+          inv[t] = rsqrtf(tot / static_cast<float>(d) + a.eps);
+        }
+      }
+    }
+    for (int c = threadIdx.x; c < d; c += kThreads) {
+#pragma unroll
+      for (int t = 0; t < kTok; ++t) {
+        if (t >= nt) continue;
+        const size_t i = static_cast<size_t>(t) * d + c;
+        const float v = a.gamma ? raw[i] * inv[t] * gam[c] : raw[i];
         if (a.elem == 2) {
           const uint16_t b = f32_to_bf16_bits(v);
-          reinterpret_cast<uint16_t*>(xs)[static_cast<size_t>(warp) * d + c] = b;
-          if (a.x_out && blockIdx.x == 0) a.x_out[static_cast<size_t>(t) * d + c] = b;
+          reinterpret_cast<uint16_t*>(xs)[i] = b;
+          if (a.x_out && blockIdx.x == 0) a.x_out[static_cast<size_t>(t0) * d + i] = b;
         } else {
-          reinterpret_cast<float*>(xs)[static_cast<size_t>(warp) * d + c] = v;   // in place over raw
-          if (a.x_out && blockIdx.x == 0) reinterpret_cast<float*>(a.x_out)[static_cast<size_t>(t) * d + c] = v;
+          reinterpret_cast<float*>(xs)[i] = v;   // in place over raw (read above by this thread only)
+          if (a.x_out && blockIdx.x == 0) reinterpret_cast<float*>(a.x_out)[static_cast<size_t>(t0) * d + i] = v;
         }
       }
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      for (int s = 0; s < nst && s < a.stages; ++s) issue_stage(a, C, ring, slot_bytes, (q + s) % a.stages, r0, r1, s);
+    // one bf16 token: its row in registers (lane's 8-column chunks), the weights alone from shared memory
+    const bool x1 = nt == 1 && a.elem == 2 && d <= 256 * kXC;
+    float xr[kXC][8];
+#pragma unroll
+    for (int j = 0; j < kXC; ++j) {
+      const int c = lane * 8 + j * 256;
+      if (x1 && c < d) {
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(xs + static_cast<size_t>(c) * 2), xr[j]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xr[j][i] = 0.f;
+      }
     }
     int s = 0;
     for (; s < nst; ++s) {
@@ -223,7 +269,20 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
         float acc[kTok];
 #pragma unroll
         for (int t = 0; t < kTok; ++t) acc[t] = 0.f;
-        for (int c = lane * 8; c < d; c += 256) dot8(wrow, a.elem, c, xs, d, nt, acc);
+        if (x1) {   // the same summation order as dot8 for one token
+#pragma unroll
+          for (int j = 0; j < kXC; ++j) {
+            const int c = lane * 8 + j * 256;
+            if (c < d) {
+              float w8[8];
+              unpack_bf16x8(*reinterpret_cast<const uint4*>(wrow + static_cast<size_t>(c) * 2), w8);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[0] = fmaf(w8[i], xr[j][i], acc[0]);
+            }
+          }
+        } else {
+          for (int c = lane * 8; c < d; c += 256) dot8(wrow, a.elem, c, xs, d, nt, acc);
+        }
 #pragma unroll
         for (int t = 0; t < kTok; ++t) {
           if (t < nt) {   // warp-uniform
