@@ -18,13 +18,14 @@
 // 128..255 in the odd CTA's.  Per CTA and 64-wide k-block that is 16 KB of A and 16 KB of B for
 // 2 x 128 x 256 x 64 FLOPs, two thirds of the bytes per FLOP of a one-CTA 128 x 256 tile, so a 6-stage
 // ring (192 KB) holds more time of MMA work in flight.  Per CTA, 192 threads:
-//   warp 0      TMA producer of this CTA's halves (2D tiled loads, 128-byte swizzle, no multicast);
+//   warp 0      TMA producer of this CTA's halves (2D tiled loads of the pair, cta_group::2, 128-byte
+//               swizzle, no multicast): both CTAs' bytes of a stage complete on the even CTA's stage
+//               barrier, which the even producer arms for both;
 //   warp 1      even CTA: allocates 512 TMEM columns (two 256-column fp32 accumulators, with the odd
-//               CTA), waits for both CTAs' stage bytes and issues the MMAs from one lane; a commit
-//               multicast to both CTAs frees a stage and, per tile, hands the accumulator to both
-//               epilogues; odd CTA: allocates with the even CTA and forwards the completion of each
-//               of its stages to the even CTA's barrier.  Barriers that the other CTA arrives on are
-//               polled without suspending the thread (a suspended waiter wakes ~0.5 us late on a
+//               CTA), waits for the stage and issues the MMAs from one lane; a commit multicast to both
+//               CTAs frees a stage and, per tile, hands the accumulator to both epilogues; odd CTA:
+//               allocates with the even CTA.  Barriers that the other CTA's copies or threads complete
+//               are polled without suspending the thread (a suspended waiter wakes ~0.5 us late on a
 //               remote arrival, which starved the MMAs);
 //   warps 2..5  epilogue: tcgen05.ld of this CTA's 128 accumulator rows (a 32-lane quarter per warp),
 //               SiLU * up -> h (gate/up) or the scaled fp32 result (down); masked stores of valid rows;
@@ -89,7 +90,6 @@ struct TcParams {
 
 struct __align__(8) Ctrl {
   uint64_t full[STAGES];     // this CTA's bytes of the stage have landed
-  uint64_t pfull[STAGES];    // even CTA: the odd CTA's bytes of the stage have landed (forwarded)
   uint64_t empty[STAGES];    // the MMAs reading the stage are done (commit multicast to both CTAs)
   uint64_t tfull[2];         // accumulator ready (commit multicast to both CTAs)
   uint64_t tempty[2];        // even CTA: accumulator read by both CTAs' epilogues (8 warp arrivals)
@@ -150,7 +150,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&C.full[s], 1);
-      mbar_init(&C.pfull[s], 1);
       mbar_init(&C.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -207,10 +206,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_expect_tx(&C.full[s], STAGE_BYTES);
+          // both CTAs' bytes complete on the even CTA's barrier, which the even producer arms for both
+          const uint32_t fbar = mapa_shared(smem_u32(&C.full[s]), 0);
+          if (even) mbar_expect_tx(&C.full[s], 2 * STAGE_BYTES);
           unsigned char* sa = stages + s * STAGE_BYTES;
-          tma_load_2d(sa, &mapA, &C.full[s], kb * BK, arow);
-          tma_load_2d(sa + A_BYTES, mB, &C.full[s], (kb % p.kb_wrap) * BK, brow);
+          tma_load_2d_pair(sa, &mapA, fbar, kb * BK, arow);
+          tma_load_2d_pair(sa + A_BYTES, mB, fbar, (kb % p.kb_wrap) * BK, brow);
         }
         if (!ok) break;
       }
@@ -237,8 +238,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int kb = 0; kb < nkb; ++kb, ++kbt) {
             const int s = kbt % STAGES;
             const uint32_t ph = static_cast<uint32_t>(kbt / STAGES) & 1u;
-            if (!mbar_wait(&C.full[s], ph, abort_flag, kTimeoutNs) ||
-                !mbar_wait_cluster(&C.pfull[s], ph, abort_flag, kTimeoutNs)) {
+            if (!mbar_wait_cluster(&C.full[s], ph, abort_flag, kTimeoutNs)) {
               ok = false;
               break;
             }
@@ -265,21 +265,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         while (!mbar_try_wait(&C.drain, 0) && globaltimer() - t0 < kTimeoutNs) {
         }
       }
-    } else if (lane == 0) {
-      // ---------------- odd CTA: forward each stage's completion to the even CTA ----------------
-      int kbt = 0;
-      bool ok = true;
-      for (int t = pair; t < total && ok && !*abort_flag; t += npairs) {
-        for (int kb = 0; kb < nkb; ++kb, ++kbt) {
-          const int s = kbt % STAGES;
-          if (!mbar_wait(&C.full[s], static_cast<uint32_t>(kbt / STAGES) & 1u, abort_flag, kTimeoutNs)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&C.pfull[s]), 0));
-        }
-      }
-      if (!ok) set_abort(C, p.timeouts, peer);
     }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
@@ -391,10 +376,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // warp meets the CTA barrier (and warp 1 the TMEM release) converged.
   __syncwarp();
   __syncthreads();
-  if (warp == 0 && lane == 0 && *abort_flag) {
-    // After an abort, loads the MMA warp never consumed may still be landing in this CTA's ring.  The
-    // latest phase of stage s belongs to the last k-block issued into it; wait (bounded) until that
-    // phase has completed, i.e. until its bytes have arrived.
+  if (warp == 0 && lane == 0 && *abort_flag && !even) {
+    // After an abort, loads this CTA issued may still be landing in its ring; they complete on the even
+    // CTA's barriers, which this CTA cannot wait on: give them a bounded time (far above a load's
+    // latency) before the cluster barrier below lets the CTA go.
+    const uint64_t t0 = globaltimer();
+    while (issued > 0 && globaltimer() - t0 < 200000ull) {
+    }
+  }
+  if (warp == 0 && lane == 0 && *abort_flag && even) {
+    // After an abort, loads the MMA warp never consumed may still be landing in this CTA's ring (and the
+    // odd CTA's).  The latest phase of stage s belongs to the last k-block issued into it; wait (bounded)
+    // until that phase has completed, i.e. until both CTAs' bytes of it have arrived.
     for (int s = 0; s < STAGES; ++s) {
       const int last = issued - 1 - ((issued - 1 - s) % STAGES + STAGES) % STAGES;
       if (last < 0) continue;
