@@ -49,19 +49,20 @@ struct HeadArgs {
 
 struct __align__(8) HeadCtrl {
   uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];   // every warp is done with the slot (one arrival per warp)
   uint64_t xbar;             // token rows (+ gamma) of the current pass
-  unsigned long long best[kTok][2];   // this CTA's best key per token for its first two codebooks
+  unsigned long long best[kWarps][kTok][2];   // each warp's best key per token for the CTA's two codebooks
   float red[kWarps][kTok];   // per-warp partial sums of squares (the final norm)
   int abort;
 };
 
-constexpr size_t kCtrlBytes = 512;
+constexpr size_t kCtrlBytes = 1536;
 static_assert(sizeof(HeadCtrl) <= kCtrlBytes, "the control block must fit ahead of the token rows");
 
-// Dynamic shared memory: control | raw token rows f32 [kTok][d] | gamma f32 [d] | x [kTok][d] in the
-// weights' type (bf16 x lives apart; f32 x is formed in place over the raw rows) | weight ring.
+// Dynamic shared memory: control | token rows f32 [kTok][d] (x is formed in place, rounded to the weights'
+// type but kept as f32) | gamma f32 [d] | weight ring.
 struct HeadSmem {
-  size_t raw, gam, x, ring, total;
+  size_t raw, gam, ring, total;
 };
 
 __host__ __device__ inline size_t a128(size_t b) { return (b + 127) & ~static_cast<size_t>(127); }
@@ -71,8 +72,7 @@ __host__ __device__ inline HeadSmem head_smem(int d, int elem, int stages, int t
   HeadSmem S;
   S.raw = kCtrlBytes;
   S.gam = S.raw + a128(static_cast<size_t>(tok) * d * 4);
-  S.x = S.gam + a128(static_cast<size_t>(d) * 4);
-  S.ring = S.x + (elem == 2 ? a128(static_cast<size_t>(tok) * d * 2) : 0);
+  S.ring = S.gam + a128(static_cast<size_t>(d) * 4);
   S.total = S.ring + static_cast<size_t>(stages) * d * elem * kRowsPerStage;
   return S;
 }
@@ -83,33 +83,31 @@ __device__ __forceinline__ uint32_t ordered_bits(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Columns [c, c + 8) of one head row against the pass's token rows x (typed like the weights).
-__device__ __forceinline__ void dot8(const unsigned char* wrow, int elem, int c, const unsigned char* xs, int d, int nt,
+// Columns [c, c + 8) of one head row against the pass's token rows x (f32 in shared memory).
+__device__ __forceinline__ void dot8(const unsigned char* wrow, int elem, int c, const float* xs, int d, int nt,
                                      float (&acc)[kTok]) {
   float w8[8];
   if (elem == 2) {
     unpack_bf16x8(*reinterpret_cast<const uint4*>(wrow + static_cast<size_t>(c) * 2), w8);
-#pragma unroll
-    for (int t = 0; t < kTok; ++t) {
-      if (t < nt) {
-        float x8[8];   // 16-byte reads at a 16-byte lane stride: no bank conflicts
-        unpack_bf16x8(*reinterpret_cast<const uint4*>(xs + (static_cast<size_t>(t) * d + c) * 2), x8);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[t] = fmaf(w8[i], x8[i], acc[t]);
-      }
-    }
   } else {
     const float4 a = *reinterpret_cast<const float4*>(wrow + static_cast<size_t>(c) * 4);
     const float4 b = *reinterpret_cast<const float4*>(wrow + static_cast<size_t>(c) * 4 + 16);
     w8[0] = a.x; w8[1] = a.y; w8[2] = a.z; w8[3] = a.w;
     w8[4] = b.x; w8[5] = b.y; w8[6] = b.z; w8[7] = b.w;
+  }
 #pragma unroll
-    for (int t = 0; t < kTok; ++t) {
-      if (t < nt) {
-        const float* xr = reinterpret_cast<const float*>(xs) + static_cast<size_t>(t) * d + c;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[t] = fmaf(w8[i], xr[i], acc[t]);
-      }
+  for (int t = 0; t < kTok; ++t) {
+    if (t < nt) {
+      const float4 p = *reinterpret_cast<const float4*>(xs + static_cast<size_t>(t) * d + c);
+      const float4 q = *reinterpret_cast<const float4*>(xs + static_cast<size_t>(t) * d + c + 4);
+      acc[t] = fmaf(w8[0], p.x, acc[t]);
+      acc[t] = fmaf(w8[1], p.y, acc[t]);
+      acc[t] = fmaf(w8[2], p.z, acc[t]);
+      acc[t] = fmaf(w8[3], p.w, acc[t]);
+      acc[t] = fmaf(w8[4], q.x, acc[t]);
+      acc[t] = fmaf(w8[5], q.y, acc[t]);
+      acc[t] = fmaf(w8[6], q.z, acc[t]);
+      acc[t] = fmaf(w8[7], q.w, acc[t]);
     }
   }
 }
@@ -137,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
   const HeadSmem L = head_smem(d, a.elem, a.stages, a.T < kTok ? a.T : kTok);
   float* raw = reinterpret_cast<float*>(smem + L.raw);
   float* gam = reinterpret_cast<float*>(smem + L.gam);
-  unsigned char* xs = a.elem == 2 ? smem + L.x : smem + L.raw;   // f32 x is formed in place
+  float* xs = raw;   // x is formed in place
   unsigned char* ring = smem + L.ring;
   const size_t row_bytes = static_cast<size_t>(d) * a.elem;
   const size_t slot_bytes = row_bytes * kRowsPerStage;
@@ -147,7 +145,10 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
   const int nst = (r1 - r0 + kRowsPerStage - 1) / kRowsPerStage;
   volatile int* abort_flag = &C.abort;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < a.stages; ++s) mbar_init(&C.full[s], 1);
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&C.full[s], 1);
+      mbar_init(&C.empty[s], kWarps);
+    }
     mbar_init(&C.xbar, 1);
     C.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -193,7 +194,6 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
       }
       break;
     }
-    if (threadIdx.x < 2 * kTok) (&C.best[0][0])[threadIdx.x] = 0ull;
     // optional RMSNorm of each token row, by the whole CTA (sums of squares per thread, then per warp,
     // then over the warps), and rounding to the weights' type
     float inv[kTok];
@@ -233,12 +233,13 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
         if (t >= nt) continue;
         const size_t i = static_cast<size_t>(t) * d + c;
         const float v = a.gamma ? raw[i] * inv[t] * gam[c] : raw[i];
+        // in place over raw (element i was read above by this thread only)
         if (a.elem == 2) {
           const uint16_t b = f32_to_bf16_bits(v);
-          reinterpret_cast<uint16_t*>(xs)[i] = b;
+          xs[i] = bf16_to_f32(b);
           if (a.x_out && blockIdx.x == 0) a.x_out[static_cast<size_t>(t0) * d + i] = b;
         } else {
-          reinterpret_cast<float*>(xs)[i] = v;   // in place over raw (read above by this thread only)
+          xs[i] = v;
           if (a.x_out && blockIdx.x == 0) reinterpret_cast<float*>(a.x_out)[static_cast<size_t>(t0) * d + i] = v;
         }
       }
@@ -251,25 +252,35 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
     for (int j = 0; j < kXC; ++j) {
       const int c = lane * 8 + j * 256;
       if (x1 && c < d) {
-        unpack_bf16x8(*reinterpret_cast<const uint4*>(xs + static_cast<size_t>(c) * 2), xr[j]);
+        const float4 p = *reinterpret_cast<const float4*>(xs + c);
+        const float4 q = *reinterpret_cast<const float4*>(xs + c + 4);
+        xr[j][0] = p.x; xr[j][1] = p.y; xr[j][2] = p.z; xr[j][3] = p.w;
+        xr[j][4] = q.x; xr[j][5] = q.y; xr[j][6] = q.z; xr[j][7] = q.w;
       } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) xr[j][i] = 0.f;
       }
     }
+    // lane t < nt of every warp keeps the warp's best key of token t for codebooks n0 and n0 + 1
+    unsigned long long best0 = 0ull, best1 = 0ull;
+    int issued = nst < a.stages ? nst : a.stages;   // thread 0: stages of this pass issued so far
     int s = 0;
     for (; s < nst; ++s) {
       const int slot = (q + s) % a.stages;
       const uint32_t par = static_cast<uint32_t>(((q + s) / a.stages) & 1);
-      ok = __syncthreads_and(mbar_wait(&C.full[slot], par, abort_flag, kTimeoutNs));
-      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(&C.full[slot], par, abort_flag, kTimeoutNs));
+      if (!ok) {   // stop the other warps' waits too
+        if (lane == 0 && atomicExch(&C.abort, 1) == 0) atomicAdd(a.timeouts, 1u);
+        break;
+      }
       const int rs = r0 + s * kRowsPerStage;
       if (rs + warp < r1) {
         const unsigned char* wrow = ring + static_cast<size_t>(slot) * slot_bytes + static_cast<size_t>(warp) * row_bytes;
         float acc[kTok];
 #pragma unroll
         for (int t = 0; t < kTok; ++t) acc[t] = 0.f;
-        if (x1) {   // the same summation order as dot8 for one token
+        if (x1) {   // four partial sums (chunks j mod 4), added pairwise: short dependency chains
+          float p4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int j = 0; j < kXC; ++j) {
             const int c = lane * 8 + j * 256;
@@ -277,9 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
               float w8[8];
               unpack_bf16x8(*reinterpret_cast<const uint4*>(wrow + static_cast<size_t>(c) * 2), w8);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) acc[0] = fmaf(w8[i], xr[j][i], acc[0]);
+              for (int i = 0; i < 8; ++i) p4[j & 3] = fmaf(w8[i], xr[j][i], p4[j & 3]);
             }
           }
+          acc[0] = (p4[0] + p4[1]) + (p4[2] + p4[3]);
         } else {
           for (int c = lane * 8; c < d; c += 256) dot8(wrow, a.elem, c, xs, d, nt, acc);
         }
@@ -290,32 +302,46 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
             for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
           }
         }
+        // every lane holds every sum: lane t takes token t's
+        float lg = acc[0];
+#pragma unroll
+        for (int t = 1; t < kTok; ++t)
+          if (lane == t) lg = acc[t];
         const int row = rs + warp;
         const int n = row / V, v = row - n * V;
-#pragma unroll
-        for (int t = 0; t < kTok; ++t) {
-          if (lane == t && t < nt) {
-            const float lg = acc[t];
-            const size_t tn = static_cast<size_t>(t0 + t) * N + n;
-            if (a.logits) a.logits[tn * V + v] = lg;
-            if (lg == lg)   // NaN never wins; the CTA's maximum first, in shared memory
-              atomicMax(&C.best[t][n - n0], (static_cast<unsigned long long>(ordered_bits(lg)) << 32) |
-                                                static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(v)));
+        if (lane < nt) {
+          if (a.logits) a.logits[(static_cast<size_t>(t0 + lane) * N + n) * V + v] = lg;
+          if (lg == lg) {   // NaN never wins
+            const unsigned long long key = (static_cast<unsigned long long>(ordered_bits(lg)) << 32) |
+                                           static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(v));
+            if (n == n0) best0 = key > best0 ? key : best0;
+            else best1 = key > best1 ? key : best1;
           }
         }
       }
-      __syncthreads();   // every warp is done with this slot (and with its shared-memory maxima)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&C.empty[slot]);
+      // thread 0 refills the slot once every warp is done with it
       if (threadIdx.x == 0 && s + a.stages < nst) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue_stage(a, C, ring, slot_bytes, slot, r0, r1, s + a.stages);
+        if (!mbar_wait(&C.empty[slot], par, abort_flag, kTimeoutNs)) {
+          ok = false;
+          if (atomicExch(&C.abort, 1) == 0) atomicAdd(a.timeouts, 1u);
+        } else {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          issue_stage(a, C, ring, slot_bytes, slot, r0, r1, s + a.stages);
+          ++issued;
+        }
       }
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
     }
+    ok = __syncthreads_and(ok && !*abort_flag);
     if (!ok) {
       if (threadIdx.x == 0) {
         if (atomicExch(&C.abort, 1) == 0) atomicAdd(a.timeouts, 1u);
-        // copies issued but not consumed must land before the CTA leaves
-        const int issued = (nst < s + a.stages) ? nst : s + a.stages;
-        for (int s2 = s; s2 < issued; ++s2) {
+        // copies issued but not consumed must land before the CTA leaves: the last stage issued into
+        // each slot (the slot's latest phase)
+        for (int s2 = issued > a.stages ? issued - a.stages : 0; s2 < issued; ++s2) {
           const int slot = (q + s2) % a.stages;
           const uint32_t par = static_cast<uint32_t>(((q + s2) / a.stages) & 1);
           const uint64_t t1 = globaltimer();
@@ -325,12 +351,21 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(HeadArgs a) {
       }
       break;
     }
-    // one global atomic per (token, codebook) this CTA touched: order-independent, so deterministic
+    // the CTA's best key per (token, codebook) over its warps, then one global atomic each:
+    // order-independent, so deterministic
+    if (lane < kTok) {
+      C.best[warp][lane][0] = best0;
+      C.best[warp][lane][1] = best1;
+    }
+    __syncthreads();
     if (threadIdx.x < 2 * nt) {
       const int t = threadIdx.x >> 1, j = threadIdx.x & 1;
-      const unsigned long long key = C.best[t][j];
+      unsigned long long key = 0ull;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) key = C.best[w][t][j] > key ? C.best[w][t][j] : key;
       if (key != 0ull && n0 + j < N) atomicMax(a.keys + static_cast<size_t>(t0 + t) * N + n0 + j, key);
     }
+    __syncthreads();   // C.best is rewritten by the next pass
     q += nst;
   }
   // the last CTA to finish turns the keys into ids
