@@ -149,14 +149,19 @@ __device__ __forceinline__ void abort_cta(StackCtrl& C, unsigned int* timeouts) 
 }
 
 // Dot product of a bf16 row in shared memory with an f32 vector in shared memory over n elements
-// (n % 8 == 0), by one warp; every lane returns the result (fixed butterfly order).
+// (n % 8 == 0), by one warp; every lane returns the result.  Lane l takes the 8-element chunks
+// [l 8 + 256 j, + 8) into four partial sums (chunk j into sum j mod 4: four short dependency chains
+// instead of one long one), adds them as (s0 + s1) + (s2 + s3), then the warp in a fixed butterfly.
 __device__ __forceinline__ float warp_dot(const uint16_t* row, const float* v, int n, int lane) {
-  float acc = 0.f;
-  for (int c = lane * 8; c < n; c += 256) {
+  float p[4] = {0.f, 0.f, 0.f, 0.f};
+  int j = 0;
+  for (int c = lane * 8; c < n; c += 256, ++j) {
     float w[8];
     unpack_bf16x8(*reinterpret_cast<const uint4*>(row + c), w);
     const float4 a = *reinterpret_cast<const float4*>(v + c);
     const float4 b = *reinterpret_cast<const float4*>(v + c + 4);
+    const int q = j & 3;
+    float acc = q == 0 ? p[0] : (q == 1 ? p[1] : (q == 2 ? p[2] : p[3]));
     acc = fmaf(w[0], a.x, acc);
     acc = fmaf(w[1], a.y, acc);
     acc = fmaf(w[2], a.z, acc);
@@ -165,7 +170,12 @@ __device__ __forceinline__ float warp_dot(const uint16_t* row, const float* v, i
     acc = fmaf(w[5], b.y, acc);
     acc = fmaf(w[6], b.z, acc);
     acc = fmaf(w[7], b.w, acc);
+    if (q == 0) p[0] = acc;
+    else if (q == 1) p[1] = acc;
+    else if (q == 2) p[2] = acc;
+    else p[3] = acc;
   }
+  float acc = (p[0] + p[1]) + (p[2] + p[3]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   return acc;
@@ -175,7 +185,7 @@ __device__ __forceinline__ float warp_dot(const uint16_t* row, const float* v, i
 // j < kXChunks chunks that lie below n (n <= 256 kXChunks).  Same summation order as warp_dot.
 constexpr int kXChunks = 8;   // d <= 2048 keeps x in registers
 __device__ __forceinline__ float warp_dot_xr(const uint16_t* row, const float (&xr)[kXChunks][8], int n, int lane) {
-  float acc = 0.f;
+  float p[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int j = 0; j < kXChunks; ++j) {
     const int c = lane * 8 + j * 256;
@@ -183,9 +193,10 @@ __device__ __forceinline__ float warp_dot_xr(const uint16_t* row, const float (&
       float w[8];
       unpack_bf16x8(*reinterpret_cast<const uint4*>(row + c), w);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc = fmaf(w[i], xr[j][i], acc);
+      for (int i = 0; i < 8; ++i) p[j & 3] = fmaf(w[i], xr[j][i], p[j & 3]);
     }
   }
+  float acc = (p[0] + p[1]) + (p[2] + p[3]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   return acc;
@@ -207,7 +218,7 @@ __device__ __forceinline__ void load_chunk8(const float* v, int c, int n, float 
 // The same for phase B's h (f <= 256 kHChunks).
 constexpr int kHChunks = 12;   // f <= 3072 keeps h in registers
 __device__ __forceinline__ float warp_dot_hr(const uint16_t* row, const float (&hr)[kHChunks][8], int n, int lane) {
-  float acc = 0.f;
+  float p[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int j = 0; j < kHChunks; ++j) {
     const int c = lane * 8 + j * 256;
@@ -215,9 +226,10 @@ __device__ __forceinline__ float warp_dot_hr(const uint16_t* row, const float (&
       float w[8];
       unpack_bf16x8(*reinterpret_cast<const uint4*>(row + c), w);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc = fmaf(w[i], hr[j][i], acc);
+      for (int i = 0; i < 8; ++i) p[j & 3] = fmaf(w[i], hr[j][i], p[j & 3]);
     }
   }
+  float acc = (p[0] + p[1]) + (p[2] + p[3]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   return acc;
