@@ -757,7 +757,7 @@ def summary_of(line):
     if "us_per_token" in line["config"]:
         out["us_per_token"] = line["config"]["us_per_token"]
     r = line.get("roofline") or {}
-    for k in ("bound", "achieved", "peak", "unit", "frac", "kernel"):
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic", "kernel"):
         if k in r:
             out[f"roofline_{k}"] = r[k]
     out["e2e_value"] = (line.get("e2e") or {}).get("value")
@@ -867,7 +867,7 @@ def run_one(args):
 
 
 HEADLINE = 4
-ALSO = ((2, 200, 20), (3, None, None), (5, 100, 10), (8, None, None))   # (workload, min steps, min warm-up)
+ALSO = ((2, 200, 20), (3, None, None), (5, 100, 10), (6, 100, 10), (7, 200, 20), (8, None, None))   # (workload, min steps, min warm-up)
 
 
 def main(argv=None):
