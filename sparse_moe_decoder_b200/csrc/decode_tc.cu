@@ -901,12 +901,20 @@ __device__ __forceinline__ bool route_item(const LayerArgs& L, const DecArgs& p,
     ss = block_sum(ss, C);
     const float inv = rsqrtf(ss / static_cast<float>(d) + L.eps);
     for (int v = threadIdx.x; v < d / 8; v += nthreads()) {
+      // 16-byte shared-memory accesses (a lane's 8 floats are 32 bytes: scalar ones conflict 8 ways)
+      const float4 h0 = reinterpret_cast<const float4*>(hr)[2 * v], h1 = reinterpret_cast<const float4*>(hr)[2 * v + 1];
+      const float4 g0 = reinterpret_cast<const float4*>(R.gam)[2 * v], g1 = reinterpret_cast<const float4*>(R.gam)[2 * v + 1];
+      const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+      const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
       uint16_t b[8];
+      float xv[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        b[i] = f32_to_bf16_bits(hr[8 * v + i] * inv * R.gam[8 * v + i]);
-        R.xs[8 * v + i] = bf16_to_f32(b[i]);
+        b[i] = f32_to_bf16_bits(hv[i] * inv * gv[i]);
+        xv[i] = bf16_to_f32(b[i]);
       }
+      reinterpret_cast<float4*>(R.xs)[2 * v] = make_float4(xv[0], xv[1], xv[2], xv[3]);
+      reinterpret_cast<float4*>(R.xs)[2 * v + 1] = make_float4(xv[4], xv[5], xv[6], xv[7]);
       if (g == 0) {
         uint4 pk;
         pk.x = b[0] | (static_cast<uint32_t>(b[1]) << 16);
@@ -934,9 +942,8 @@ __device__ __forceinline__ bool route_item(const LayerArgs& L, const DecArgs& p,
 #pragma unroll
     for (int j = 0; j < 16; ++j) acc[j] = 0.f;
     for (int v = threadIdx.x; v < d / 8; v += nthreads()) {
-      float xv[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) xv[i] = R.xs[8 * v + i];
+      const float4 xa = reinterpret_cast<const float4*>(R.xs)[2 * v], xb = reinterpret_cast<const float4*>(R.xs)[2 * v + 1];
+      const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
       for (int j = 0; j < 16; ++j)
         if (j0 + j < ne) {
