@@ -366,12 +366,12 @@ ZMOE_API zmoe_status zmoe_moe_layer_w8a8_workspace_layout(int T, int d, int f, i
  * Expert weights as in zmoe_moe_layer_fp8 (E4M3 codes, one fp32 scale per row: w = code * scale);
  * router in bf16.  Each row entering an expert GEMM -- the permuted token row, then the hidden row h --
  * is quantized per token: s = max|row| / 448 (fp32; 1 for an all-zero row), codes = the E4M3 value
- * nearest row / s (ties to even, saturating at 448).  The GEMMs run on tcgen05 kind::f8f6f4 (CTA pairs);
+ * nearest row x fp32(1 / s) (each product rounded to fp32; ties to even, saturating at 448).  The GEMMs run on tcgen05 kind::f8f6f4 (CTA pairs);
  * their fp32 sums are multiplied by the token scale and the weight row's scale; h is held in f16 between
  * the GEMMs (an |h| beyond 65504 counts a device error) and quantized from that.
  *   y[t] = h[t] + sum_i gate[t, i] * down_e( Q(silu(gate_e(Q(x[t]))) * up_e(Q(x[t]))) )   (h = 0 if NULL)
- * Arguments as zmoe_moe_layer_fp8 (x or h with gamma: bf16 / f32); any T (built for >= 64 rows per expert
- * on average); d % 256 == 0, f % 256 == 0.
+ * Arguments as zmoe_moe_layer_fp8 (x or h with gamma: bf16 / f32; the codes and the scale arrays 16-byte
+ * aligned); any T (built for >= 64 rows per expert on average); d % 256 == 0, f % 256 == 0.
  */
 ZMOE_API zmoe_status zmoe_moe_layer_w8a8(const void* x, const float* h, const float* gamma, float eps,
                                          const void* w_router, const float* logit_bias, const float* sel_bias,

@@ -299,17 +299,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           if (valid) {
             if (FMT != kPair) {
+              // E4M3: the chunk's 32 gate and 32 up weight-row scales, as 16-byte loads (the same for every
+              // row of the tile: broadcast from L1)
+              float sg[32], su[32];
+              if (FMT == kE4M3) {
+                const float4* pg = reinterpret_cast<const float4*>(p.col_scale0 + col0 + c * 32);
+                const float4* pu = reinterpret_cast<const float4*>(p.col_scale1 + col0 + c * 32);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                  const float4 a = __ldg(pg + q), b = __ldg(pu + q);
+                  sg[4 * q] = a.x; sg[4 * q + 1] = a.y; sg[4 * q + 2] = a.z; sg[4 * q + 3] = a.w;
+                  su[4 * q] = b.x; su[4 * q + 1] = b.y; su[4 * q + 2] = b.z; su[4 * q + 3] = b.w;
+                }
+              }
               uint32_t hv[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
                 float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
                 if (FMT == kE4M3) {
-                  const size_t j = col0 + c * 32 + 2 * i;
-                  g0 *= rs * __ldg(p.col_scale0 + j);
-                  g1 *= rs * __ldg(p.col_scale0 + j + 1);
-                  u0 *= rs * __ldg(p.col_scale1 + j);
-                  u1 *= rs * __ldg(p.col_scale1 + j + 1);
+                  g0 *= rs * sg[2 * i];
+                  g1 *= rs * sg[2 * i + 1];
+                  u0 *= rs * su[2 * i];
+                  u1 *= rs * su[2 * i + 1];
                 }
                 const float h0 = silu_mul(g0, u0), h1 = silu_mul(g1, u1);
                 range_ok = range_ok && fabsf(h0) < 65504.f && fabsf(h1) < 65504.f;
@@ -357,9 +369,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           if (valid) {
             float o[32];
+            if (FMT == kE4M3) {
+              // the chunk's 32 weight-row scales as 16-byte loads
+              const float4* pc = reinterpret_cast<const float4*>(cs + c * 32);
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              o[j] = __uint_as_float(v[j]) * sc * (FMT == kE4M3 ? __ldg(cs + c * 32 + j) : 1.f);
+              for (int q = 0; q < 8; ++q) {
+                const float4 a = __ldg(pc + q);
+                o[4 * q] = __uint_as_float(v[4 * q]) * sc * a.x;
+                o[4 * q + 1] = __uint_as_float(v[4 * q + 1]) * sc * a.y;
+                o[4 * q + 2] = __uint_as_float(v[4 * q + 2]) * sc * a.z;
+                o[4 * q + 3] = __uint_as_float(v[4 * q + 3]) * sc * a.w;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(v[j]) * sc;
+            }
             float4* dst = reinterpret_cast<float4*>(y + c * 32);
 #pragma unroll
             for (int j = 0; j < 8; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);

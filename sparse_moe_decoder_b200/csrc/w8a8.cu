@@ -226,7 +226,7 @@ zmoe_status zmoe_moe_layer_w8a8(const void* x, const float* h, const float* gamm
   ZMOE_REQUIRE(gamma ? h != nullptr : x != nullptr, "zmoe_moe_layer_w8a8: needs x, or h with gamma");
   ZMOE_REQUIRE((!x || aligned16(x)) && (!h || aligned16(h)) && aligned16(y) && (!w_router || aligned16(w_router)) &&
                    aligned16(q_gate) && aligned16(q_up) && aligned16(q_down) && (!x_norm || aligned16(x_norm)) &&
-                   (!gamma || aligned16(gamma)),
+                   (!gamma || aligned16(gamma)) && aligned16(s_gate) && aligned16(s_up) && aligned16(s_down),
                "zmoe_moe_layer_w8a8: pointers must be 16-byte aligned");
   if (!grouped_swiglu_tc_supported(d, f))
     return fail(ZMOE_ERR_UNSUPPORTED, "zmoe_moe_layer_w8a8: no tensor-core kernel for this d, f");
