@@ -17,7 +17,7 @@
 // other halves from the odd CTA's, and leaves D rows 0..127 in the even CTA's tensor memory and rows
 // 128..255 in the odd CTA's.  Per CTA and 64-wide k-block that is 16 KB of A and 16 KB of B for
 // 2 x 128 x 256 x 64 FLOPs, two thirds of the bytes per FLOP of a one-CTA 128 x 256 tile, so a 6-stage
-// ring (192 KB) holds more time of MMA work in flight.  Per CTA, 192 threads:
+// ring (192 KB) holds more time of MMA work in flight.  Per CTA, 320 threads:
 //   warp 0      TMA producer of this CTA's halves (2D tiled loads of the pair, cta_group::2, 128-byte
 //               swizzle, no multicast): both CTAs' bytes of a stage complete on the even CTA's stage
 //               barrier, which the even producer arms for both;
@@ -27,7 +27,8 @@
 //               allocates with the even CTA.  Barriers that the other CTA's copies or threads complete
 //               are polled without suspending the thread (a suspended waiter wakes ~0.5 us late on a
 //               remote arrival, which starved the MMAs);
-//   warps 2..5  epilogue: tcgen05.ld of this CTA's 128 accumulator rows (a 32-lane quarter per warp),
+//   warps 2..9  epilogue: tcgen05.ld of this CTA's 128 accumulator rows (a 32-lane quarter and half of
+//               the column chunks per warp: two warps per quarter, so the epilogue keeps up with the MMAs),
 //               SiLU * up -> h (gate/up) or the scaled fp32 result (down); masked stores of valid rows;
 //               then an arrival on the even CTA's accumulator-free barrier.
 // Tiles are the flattened (expert, 256-row m-tile, n-tile) space computed on the device from `offsets`,
@@ -57,7 +58,8 @@ constexpr int STAGES = 6;
 constexpr int A_BYTES = BMC * KB_BYTES;         // 16 KB
 constexpr int B_BYTES = BNC * KB_BYTES;         // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;   // warp 0 producer, warp 1 MMA, warps 2..9 epilogue
+constexpr int kEpiWarps = 8;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 constexpr int kMaxE = 64;
@@ -154,7 +156,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&C.tfull[b], 1);
-      mbar_init(&C.tempty[b], 8);
+      mbar_init(&C.tempty[b], 2 * kEpiWarps);   // every epilogue warp of both CTAs
     }
     mbar_init(&C.drain, 1);
     C.abort = 0;
@@ -267,8 +269,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..9) ----------------
+    // a warp reads the TMEM lanes of its quarter (warp % 4) and one half of each tile's column chunks
     const int quarter = warp & 3;
+    const int chalf = (warp - 2) >> 2;
     const uint32_t tempty0 = mapa_shared(smem_u32(&C.tempty[0]), 0);
     const uint32_t tempty1 = mapa_shared(smem_u32(&C.tempty[1]), 0);
     int it = 0;
@@ -292,7 +296,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const float rs = (FMT == kE4M3 && valid) ? p.row_scale[row] : 1.f;
         const size_t col0 = static_cast<size_t>(e) * p.b_rows_per_expert + nt * BNC;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 2 * chalf; c < 2 * chalf + 2; ++c) {
           uint32_t g[32], u[32];
           tmem_ld32(taddr + c * 32, g);
           tmem_ld32(taddr + 128 + c * 32, u);
@@ -363,7 +367,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const float sc = FMT == kF16 ? p.down_scale[e] : ((FMT == kE4M3 && valid) ? p.row_scale[row] : 1.f);
         const float* cs = FMT == kE4M3 ? p.col_scale0 + static_cast<size_t>(e) * p.b_rows_per_expert + nt * BN : nullptr;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 4 * chalf; c < 4 * chalf + 4; ++c) {
           uint32_t v[32];
           tmem_ld32(taddr + c * 32, v);
           tmem_wait_ld();
