@@ -96,7 +96,7 @@ struct __align__(16) StackCtrl {
   float gsel[kMaxK];
   int ids[kMaxN];
   float red[kThreads / 32];
-  float logit[kMaxE];
+  float lpart[kThreads / 32][kMaxE];   // per-warp partial router logits
   float qb[kMaxE];           // the layer's logit bias (0 when none)
   float sb[kMaxE];           // the layer's selection bias (0 when none)
   float gv[kConsumers];      // gate value of warp w's row of the current block
@@ -233,6 +233,37 @@ __device__ __forceinline__ float warp_dot_hr(const uint16_t* row, const float (&
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   return acc;
+}
+
+// Warp reduce-scatter of 16 per-lane values p[0..16): on return lane l holds in p[0] the warp's sum of
+// value l >> 1 (both lanes of a pair hold it).  Five steps of lane distance 16, 8, 4, 2, 1; at each the
+// lane keeps the half of its values that its lane bit selects and adds the partner's copy of that half,
+// so every sum is formed once, in a fixed order.
+__device__ __forceinline__ float warp_reduce_scatter16(float (&p)[16], int lane) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool hi = (lane & 16) != 0;
+    const float send = hi ? p[i] : p[i + 8], keep = hi ? p[i + 8] : p[i];
+    p[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool hi = (lane & 8) != 0;
+    const float send = hi ? p[i] : p[i + 4], keep = hi ? p[i + 4] : p[i];
+    p[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool hi = (lane & 4) != 0;
+    const float send = hi ? p[i] : p[i + 2], keep = hi ? p[i + 2] : p[i];
+    p[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  {
+    const bool hi = (lane & 2) != 0;
+    const float send = hi ? p[0] : p[1], keep = hi ? p[1] : p[0];
+    p[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  return p[0] + __shfl_xor_sync(0xffffffffu, p[0], 1);
 }
 
 // Order-preserving map of a float onto uint32 (larger float -> larger key; -0 maps like +0).
@@ -387,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       C.qb[threadIdx.x] = Ly.logit_bias ? Ly.logit_bias[threadIdx.x] : 0.f;
       C.sb[threadIdx.x] = Ly.sel_bias ? Ly.sel_bias[threadIdx.x] : 0.f;
     }
-    // ---- pre-norm: x = bf16(RMSNorm(h) * gamma), kept as f32 in xs ----
+    // ---- pre-norm: x = bf16(RMSNorm(h) * gamma), kept as f32 in hv (this thread's vectors) and xs ----
     if (l > 0 || !a.ids) {
 #pragma unroll
       for (int j = 0; j < kMaxVec; ++j) {
@@ -411,28 +442,43 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
     for (int j = 0; j < kMaxVec; ++j) {
       const int v = threadIdx.x + j * kThreads;
       if (v >= nvec) continue;
+      float g[8];
+      load_chunk8(gam, v * 8, d, g);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int n = v * 8 + i;
-        const uint16_t b = f32_to_bf16_bits(hv[j][i] * inv * gam[n]);
-        xs[n] = bf16_to_f32(b);
+        const uint16_t b = f32_to_bf16_bits(hv[j][i] * inv * g[i]);
         if (c == 0 && a.layer_x) a.layer_x[static_cast<size_t>(l) * d + n] = b;
         if (c == 0 && a.layer_h) a.layer_h[static_cast<size_t>(l) * d + n] = hv[j][i];
+        hv[j][i] = bf16_to_f32(b);
       }
+      *reinterpret_cast<float4*>(xs + v * 8) = make_float4(hv[j][0], hv[j][1], hv[j][2], hv[j][3]);
+      *reinterpret_cast<float4*>(xs + v * 8 + 4) = make_float4(hv[j][4], hv[j][5], hv[j][6], hv[j][7]);
     }
-    __syncthreads();
-    // x in registers for the dot products of this layer (when d fits kXChunks chunks)
-    const bool x_in_regs = d <= 256 * kXChunks;
-    float xr[kXChunks][8];
-#pragma unroll
-    for (int j = 0; j < kXChunks; ++j) load_chunk8(xs, lane * 8 + j * 256, x_in_regs ? d : 0, xr[j]);
-    // ---- router logits, one warp per expert ----
+    // ---- router logits: each thread's dot products over its own vectors of x, 16 experts at a time, a
+    // reduce-scatter per warp, then (warp 0, below) the 8 warps' partial sums in warp order ----
     if (Ly.w_r) {
       const uint16_t* wr = reinterpret_cast<const uint16_t*>(wr_s);
-      for (int e = warp; e < E; e += kThreads / 32) {
-        const uint16_t* row = wr + static_cast<size_t>(e) * d;
-        const float v = x_in_regs ? warp_dot_xr(row, xr, d, lane) : warp_dot(row, xs, d, lane);
-        if (lane == 0) C.logit[e] = v;
+      for (int e0 = 0; e0 < E; e0 += 16) {
+        float pl[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          pl[t] = 0.f;
+          if (e0 + t < E) {
+#pragma unroll
+            for (int j = 0; j < kMaxVec; ++j) {
+              const int v = threadIdx.x + j * kThreads;
+              if (v < nvec) {
+                float w[8];
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e0 + t) * d + v * 8), w);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) pl[t] = fmaf(w[i], hv[j][i], pl[t]);
+              }
+            }
+          }
+        }
+        const float s = warp_reduce_scatter16(pl, lane);
+        if ((lane & 1) == 0 && e0 + (lane >> 1) < E) C.lpart[warp][e0 + (lane >> 1)] = s;
       }
     }
     __syncthreads();
@@ -453,7 +499,12 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const int e = lane + 32 * j;
-          qv[j] = e < E ? C.logit[e] + C.qb[e] : -INFINITY;
+          float lg = 0.f;
+          if (e < E) {
+#pragma unroll
+            for (int w = 0; w < kThreads / 32; ++w) lg += C.lpart[w][e];
+          }
+          qv[j] = e < E ? lg + C.qb[e] : -INFINITY;
           const float sv = e < E ? qv[j] + C.sb[e] : 0.f;
           sk[j] = e >= E ? 0u : (sv != sv ? 1u : order_key(sv));
         }
@@ -553,6 +604,12 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       // ================================ consumers (warps 1..7) ================================
       // every consumer warp takes every item in order; warp cw contracts row cw of the block
       const int cw = warp - 1;
+      // x in registers for the phase-A dot products (when d fits kXChunks chunks), loaded while the
+      // first block is in flight
+      const bool x_in_regs = d <= 256 * kXChunks;
+      float xr[kXChunks][8];
+#pragma unroll
+      for (int j = 0; j < kXChunks; ++j) load_chunk8(xs, lane * 8 + j * 256, x_in_regs ? d : 0, xr[j]);
       // phase A: h of the owned f-rows of each chosen expert
       for (int i = 0; i < nA && ok; ++i) {
         const int qq = q + i, slot = qq % kSlots;
