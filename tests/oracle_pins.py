@@ -161,6 +161,25 @@ def pin_route(router_logits, softmax, select_topk, route):
         for t in range(40):
             want = sorted(range(7), key=lambda e: (-s[t, e], e))[:k]
             assert got[t].tolist() == want
+    # 8. the margin: hand-worked scores [3, 0.2, 0, -1] (the second gap is the smaller one), on the
+    # selection scores (a bias that reorders them moves it), and E = 2 with k = 2 (one gap only)
+    xs = np.array([[3.0, 0.2, 0.0, -1.0]])
+    m1, m2 = route(xs, np.eye(4), 1)[2][0], route(xs, np.eye(4), 2)[2][0]
+    assert abs(m1 - 2.8) < 1e-15 and abs(m2 - 0.2) < 1e-15, (m1, m2)
+    m = route(xs, np.eye(4), 2, sel_bias=np.array([0.0, 0.0, 2.5, 0.0]))[2][0]   # s = [3, 0.2, 2.5, -1]
+    assert abs(m - 0.5) < 1e-15, m                                               # min(3 - 2.5, 2.5 - 0.2)
+    m = route(np.array([[1.0, 4.0]]), np.eye(2), 2)[2][0]
+    assert abs(m - 3.0) < 1e-15, m
+    # brute force: the smallest gap between consecutive ranks 0..k of the sorted selection scores
+    x = rng.standard_normal((30, 6))
+    W = rng.standard_normal((5, 6))
+    sb = rng.standard_normal(5)
+    for k in (1, 2):
+        _, _, m, _ = route(x, W, k, sel_bias=sb)
+        for t in range(30):
+            st = sorted((float(np.dot(W[e], x[t])) + sb[e] for e in range(5)), reverse=True)
+            want = min(st[r] - st[r + 1] for r in range(k))
+            assert abs(m[t] - want) < 1e-12, (t, k, m[t], want)
 
 
 # ------------------------------------------------------------------------------------------

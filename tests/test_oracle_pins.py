@@ -157,6 +157,21 @@ def _route_ties_high(x, W, k, sel_bias=None, logit_bias=None):
         route_mod.select_topk = orig
 
 
+def _route_margin_top_gap_only(x, W, k, sel_bias=None, logit_bias=None):
+    """Planted: the margin is the gap between the two best scores only, whatever k."""
+    sel, g, m, p = oracle.route(x, W, k, sel_bias, logit_bias)
+    q = oracle.router_logits(x, W) + (0.0 if logit_bias is None else np.asarray(logit_bias))
+    s_ = -np.sort(-(q if sel_bias is None else q + np.asarray(sel_bias)), axis=1)
+    return sel, g, (s_[:, 0] - s_[:, 1]) if s_.shape[1] > 1 else m, p
+
+
+def _route_margin_on_logits(x, W, k, sel_bias=None, logit_bias=None):
+    """Planted: the margin taken on the unbiased logits instead of the selection scores."""
+    sel, g, _, p = oracle.route(x, W, k, sel_bias, logit_bias)
+    _, _, m, _ = oracle.route(x, W, k, None, logit_bias)
+    return sel, g, m, p
+
+
 def _permute_descending_t(expert_idx, E, x=None):
     idx = np.asarray(expert_idx)
     T, k = idx.shape
@@ -338,6 +353,10 @@ MUTANTS = {
                                                    _route_top1_renormalised),
     "ties to the higher index": lambda: P.pin_route(oracle.router_logits, oracle.softmax, _select_ties_high,
                                                     _route_ties_high),
+    "margin of the top two scores only": lambda: P.pin_route(oracle.router_logits, oracle.softmax,
+                                                             oracle.select_topk, _route_margin_top_gap_only),
+    "margin on the unbiased logits": lambda: P.pin_route(oracle.router_logits, oracle.softmax, oracle.select_topk,
+                                                         _route_margin_on_logits),
     "permutation not stable": lambda: P.pin_permute(_permute_descending_t),
     "silu is the sigmoid": lambda: P.pin_ffn(_silu_is_sigmoid, oracle.swiglu_ffn, oracle.grouped_swiglu),
     "gate and up swapped": lambda: P.pin_ffn(oracle.silu, _swiglu_swapped, oracle.grouped_swiglu),
