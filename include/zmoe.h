@@ -416,10 +416,12 @@ ZMOE_API size_t zmoe_decode_stack_workspace_size(int n_layers, int d, int f, int
  *   CTA repeats the pre-norm and routing, the weights stream through shared memory, two grid
  *   barriers per layer.  Same arithmetic as n_layers zmoe_moe_layer calls with T = 1 (fp32 sums in a
  *   fixed order; the router's summation order differs, so ids can differ only on near-ties).
- *   Limits: n_layers <= 32, d % 8 == 0, d <= 4096, f % 8 == 0, N <= 32, and the per-CTA buffers
- *   must fit one SM (14 ring slots of max(4 d, 2 f) bytes, the largest router E d 2 bytes, 8 d +
- *   8 f bytes): d = 2048, f = 3072, E = 16 fits; larger sizes return ZMOE_ERR_UNSUPPORTED.  Ids
- *   outside [0, V) count a device error and contribute nothing.
+ *   Limits: n_layers <= 32, d % 8 == 0, d <= 4096, f % 8 == 0, N <= 32, at most 64 of the d rows
+ *   per SM, and the per-CTA buffers must fit one SM's shared memory: a 4-slot ring of weight blocks
+ *   (a block = as many 2 d- or 2 f-byte rows as fit 32 KB, 1 to 7), max(E d 2, 8 f) bytes for the
+ *   router rows and then the chosen experts' h, 8 d bytes of gain and x, and ~2 KB of control.
+ *   d = 2048, f = 3072, E = 16 fits; larger sizes return ZMOE_ERR_UNSUPPORTED.  Ids outside [0, V)
+ *   count a device error and contribute nothing.
  */
 ZMOE_API zmoe_status zmoe_decode_stack(const zmoe_stack_layer* layers, int n_layers, int d, int f, float eps,
                                        const int32_t* ids, const void* tables, const float* gamma0, int N, int V,

@@ -147,3 +147,81 @@ def test_timeout_injection_checks_its_limit(L):
     assert L.zmoe_debug_inject_timeout(1, 10) == 1                  # below 1 us: ZMOE_ERR_INVALID_ARG
     assert L.zmoe_debug_inject_timeout(1, 3_000_000_000) == 1       # above 2 s
     assert L.zmoe_debug_inject_timeout(0, 0) == 0
+
+
+# Placeholder device pointers: 16-byte aligned, never dereferenced (every case fails on the host first).
+_A, _B, _C, _D, _S = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000
+
+
+def _w8a8_layer(L, T=4, d=256, f=256, E=16, k=1, x=_A, h=NULL, gamma=NULL, w_router=_B, q_gate=_C, s_gate=_S,
+                y=_D):
+    return L.zmoe_moe_layer_w8a8(x, h, gamma, 1e-6, w_router, NULL, NULL, q_gate, s_gate, _C, _S, _C, _S, T, d, f, E,
+                                 k, y, NULL, NULL, NULL, NULL, NULL, 0, NULL)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(T=-1), dict(E=65), dict(k=3), dict(k=2, E=1), dict(d=384), dict(f=128), dict(q_gate=NULL), dict(y=NULL),
+    dict(w_router=NULL), dict(x=NULL), dict(gamma=_S), dict(s_gate=_S + 4),
+])
+def test_w8a8_layer_bad_arguments_rejected_on_host(L, kw):
+    assert _w8a8_layer(L, **kw) == 1
+    assert len(L.zmoe_last_error()) > 0
+
+
+def _f16h_layer(L, T=4, d=256, f=256, E=16, k=1, x=_A, w_down_f16=_C, down_scale=_S, y=_D):
+    return L.zmoe_moe_layer_f16h(x, NULL, NULL, 1e-6, _B, NULL, NULL, _C, _C, w_down_f16, down_scale, T, d, f, E, k, y,
+                                 NULL, NULL, NULL, NULL, NULL, 0, NULL)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(T=-1), dict(E=0), dict(k=3), dict(d=2056), dict(f=264), dict(w_down_f16=NULL), dict(down_scale=NULL),
+    dict(x=_A + 8),
+])
+def test_f16h_layer_bad_arguments_rejected_on_host(L, kw):
+    assert _f16h_layer(L, **kw) == 1
+    assert len(L.zmoe_last_error()) > 0
+
+
+@pytest.mark.parametrize("args", [
+    dict(M=-1), dict(E=65), dict(d=200), dict(offsets=NULL), dict(h=NULL), dict(h=_D + 2),
+])
+def test_grouped_swiglu_f16h_bad_arguments_rejected_on_host(L, args):
+    a = dict(M=64, E=4, d=256, f=256, offsets=_S, h=_D)
+    a.update(args)
+    assert L.zmoe_grouped_swiglu_f16h(_A, a["offsets"], a["M"], _B, _B, _C, _S, a["E"], a["d"], a["f"], a["h"], _D,
+                                      NULL) == 1
+    assert len(L.zmoe_last_error()) > 0
+
+
+def test_prepare_w_down_f16_checks_its_arguments_and_workspace(L):
+    assert L.zmoe_prepare_w_down_f16(_A, 0, 256, 256, _B, _S, _C, 64, NULL) == 1        # E = 0
+    assert L.zmoe_prepare_w_down_f16(_A, 4, 252, 256, _B, _S, _C, 64, NULL) == 1        # d % 8
+    assert L.zmoe_prepare_w_down_f16(_A, 4, 256, 256, NULL, _S, _C, 64, NULL) == 1      # NULL output
+    assert L.zmoe_prepare_w_down_f16(_A + 8, 4, 256, 256, _B, _S, _C, 64, NULL) == 1    # unaligned
+    assert L.zmoe_prepare_w_down_f16(_A, 16, 256, 256, _B, _S, _C, 63, NULL) == 4       # 4 E bytes needed
+    assert b"workspace" in L.zmoe_last_error()
+
+
+def _stack_layers(n, **over):
+    arr = (Z.StackLayer * n)()
+    for i in range(n):
+        f = dict(w_router=_A, logit_bias=NULL, sel_bias=NULL, gamma=_S, w_gate=_B, w_up=_C, w_down=_D, E=16, k=1)
+        f.update(over)
+        arr[i] = Z.StackLayer(f["w_router"], f["logit_bias"], f["sel_bias"], f["gamma"], f["w_gate"], f["w_up"],
+                              f["w_down"], f["E"], f["k"])
+    return arr
+
+
+@pytest.mark.parametrize("case", [
+    dict(n=0), dict(n=33), dict(d=2044), dict(d=4104), dict(f=3070), dict(eps=-1.0), dict(h=NULL), dict(h=_D + 4),
+    dict(ids=_S, N=0), dict(ids=_S, N=33), dict(layer=dict(E=65)), dict(layer=dict(k=3)), dict(layer=dict(E=1, k=2)),
+    dict(layer=dict(w_router=NULL)), dict(layer=dict(w_down=NULL)), dict(layer=dict(w_gate=_B + 8)),
+])
+def test_decode_stack_bad_arguments_rejected_on_host(L, case):
+    n = case.get("n", 2)
+    arr = _stack_layers(max(n, 1), **case.get("layer", {}))
+    st = L.zmoe_decode_stack(ctypes.cast(arr, ctypes.c_void_p), n, case.get("d", 2048), case.get("f", 3072),
+                             case.get("eps", 1e-6), case.get("ids", NULL), _A, _S, case.get("N", 9), 1025,
+                             case.get("h", _D), NULL, NULL, NULL, NULL, _C, 1 << 20, NULL)
+    assert st == 1
+    assert len(L.zmoe_last_error()) > 0
