@@ -98,6 +98,22 @@ def test_full_ffn_stack_teacher_forced(stack28):
     assert np.array_equal(host(st.next_ids)[ok], ref["ids"][ok])
 
 
+@pytest.mark.parametrize("d,f,E,n_layers", [(512, 768, 20, 3), (256, 512, 64, 2), (3072, 1024, 8, 2)])
+def test_stack_other_shapes_teacher_forced(d, f, E, n_layers):
+    """The one-launch stack away from the model's sizes: E = 20 (the router's partial logits go in groups
+    of 16 experts, the last group ragged), E = 64 (four groups; top-k over two experts per lane),
+    d = 256 (one warp holds all of x), d = 3072 (two vectors of x per thread; phase A reads x from
+    shared memory)."""
+    require_gpu()
+    spec = StackSpec(seed=11, n_layers=n_layers, d=d, f=f, E=E)
+    st = stack_from_bits(bf16_bits(spec.tables()), spec.gamma0(), spec.layer_small,
+                         stack_expert_bits(spec, workers=1), spec.n_layers, spec.E, spec.d, spec.f, spec.k_of,
+                         spec.eps, T=1)
+    assert st.persistent, f"d = {d}, f = {f}, E = {E} runs as one zmoe_decode_stack launch"
+    check_teacher_forced(spec, st, 2)
+    assert zmoe_get_device_errors() == 0
+
+
 def check_teacher_forced(spec, st, steps):
     codes = spec.codes(steps)
     cache = {}
