@@ -3,8 +3,6 @@
 import hashlib
 import os
 
-import pytest
-
 import bench
 
 

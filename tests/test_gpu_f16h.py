@@ -16,7 +16,7 @@ import oracle
 from moe_inputs import make_config, make_moe_layer
 from sparse_moe_decoder_b200 import (MoELayerRunner, MoEWeights, zmoe_get_device_errors, zmoe_grouped_swiglu_f16h,
                                      zmoe_prepare_w_down_f16)
-from tests.gpu_util import MARGIN_EXEMPT, assert_close, host, rel_err, require_gpu, to_dev
+from tests.gpu_util import MARGIN_EXEMPT, assert_close, host, require_gpu, to_dev
 
 pytestmark = pytest.mark.gpu
 

@@ -7,12 +7,11 @@ grouped SwiGLU runs many tiles per CTA.
 """
 import numpy as np
 import pytest
-import torch
 
 import oracle
 from moe_inputs import make_config
 from sparse_moe_decoder_b200 import MoELayerRunner, MoEWeights
-from tests.gpu_util import MARGIN_EXEMPT, TOL, assert_close, host, rel_err, require_gpu, tdtype, to_dev
+from tests.gpu_util import MARGIN_EXEMPT, assert_close, host, rel_err, require_gpu, tdtype, to_dev
 
 pytestmark = pytest.mark.gpu
 

@@ -6,7 +6,7 @@ import torch
 import oracle
 from moe_inputs import CODEBOOK_SIZE, PAD_ID, StackSpec, make_codes, round_to_bf16
 from sparse_moe_decoder_b200 import zmoe_embed_sum_rmsnorm, zmoe_get_device_errors, zmoe_rmsnorm
-from tests.gpu_util import TOL, assert_close, host, require_gpu, to_dev
+from tests.gpu_util import assert_close, host, require_gpu, to_dev
 
 pytestmark = pytest.mark.gpu
 

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from moe_inputs import make_config, make_moe_layer, round_to_bf16
+from moe_inputs import make_config, make_moe_layer
 from sparse_moe_decoder_b200 import zmoe_grouped_swiglu
 from tests.gpu_util import TOL, assert_close, host, rel_err, require_gpu, tdtype, to_dev
 
