@@ -162,8 +162,7 @@ __global__ void __launch_bounds__(kWarps * 32) route_kernel(
     const T* __restrict__ x, const T* __restrict__ w, const float* __restrict__ logit_bias,
     const float* __restrict__ sel_bias, int T_, int d, int E, int k, int32_t* __restrict__ expert_idx,
     float* __restrict__ gates, float* __restrict__ margin) {
-  constexpr int TB = 64 / EP;   // tokens per CTA
-  constexpr int G = EP / 2;     // lanes holding one token's logits
+  constexpr int TB = 64 / EP;   // tokens per CTA (EP / 2 lanes hold one token's logits)
   __shared__ float2 part[kWarps][32];
 
   const int lane = threadIdx.x & 31;
