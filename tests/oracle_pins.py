@@ -406,6 +406,10 @@ def pin_heads(head_logits, greedy, output_heads, rmsnorm):
     assert np.allclose(out["x"], rmsnorm(h, g, 1e-6), rtol=1e-15)
     assert np.array_equal(out["ids"], np.argmax(head_logits(rmsnorm(h, g, 1e-6), W), axis=-1))
     assert (out["margin"] >= 0).all()
+    # the margin is the gap between the two largest logits: identity head rows make the logits h itself
+    out = output_heads(np.array([[0.5, 2.0, -1.0, 1.9], [2.0, 2.0, 0.0, 1.0]]), np.eye(4)[None], None, 1e-6)
+    assert out["ids"].tolist() == [[1], [0]]
+    assert abs(out["margin"][0, 0] - 0.1) < 1e-15 and out["margin"][1, 0] == 0.0, out["margin"]
 
 
 def pin_speaker(speaker_prefix):

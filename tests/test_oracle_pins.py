@@ -240,6 +240,14 @@ def _greedy_ties_high(logits):
     return (L.shape[-1] - 1 - np.argmax(L[..., ::-1], axis=-1)).astype(np.int64)
 
 
+def _heads_margin_top_and_third(h, w_heads, gamma, eps, x_rounded=None):
+    """Planted: the heads' margin taken between the largest and the third largest logit."""
+    out = oracle.output_heads(h, w_heads, gamma, eps, x_rounded)
+    s_ = np.sort(out["logits"], axis=-1)
+    out["margin"] = s_[..., -1] - s_[..., -3]
+    return out
+
+
 def _head_logits_transposed(x, w):
     """Planted: the head contracted over the wrong axis of W (rows and columns swapped)."""
     w = np.asarray(w, np.float64)
@@ -368,6 +376,8 @@ MUTANTS = {
                                            oracle.moe_layer_bruteforce),
     "greedy ties to the higher id": lambda: P.pin_heads(oracle.head_logits, _greedy_ties_high, oracle.output_heads,
                                                          oracle.rmsnorm),
+    "heads margin of the top and third logits": lambda: P.pin_heads(oracle.head_logits, oracle.greedy,
+                                                                   _heads_margin_top_and_third, oracle.rmsnorm),
     "head contracted on the wrong axis": lambda: P.pin_heads(_head_logits_transposed, oracle.greedy,
                                                               oracle.output_heads, oracle.rmsnorm),
     "e4m3 exponent bias 8": lambda: P.pin_fp8(_e4m3_decode_bias8, oracle.dequantize_rows, oracle.moe_layer_fp8),
